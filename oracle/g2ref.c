@@ -1,0 +1,196 @@
+/*
+ * g2ref.c -- fp64 CPU oracle for the Gemma 2 per-layer attention forward.
+ *
+ * TEST INFRASTRUCTURE (see g2ref.h): loaded only by the tests, the smoke
+ * check and the benchmark's CPU-baseline leg. Plain loops, no blocking, no
+ * fusion: one query row at a time, in the order of the Gemma 2 card's
+ * per-layer attention pseudo-code ("Method" section): scale the queries,
+ * score every key, soft-cap, mask, softmax, mix the values.
+ */
+#include "g2ref.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+static double widen(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int check_args(int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                      int64_t q_offset, double softcap, int64_t window) {
+    if (B <= 0 || T <= 0 || S <= 0 || H <= 0 || Hkv <= 0 || d <= 0) return -1;
+    if (H % Hkv != 0) return -1;
+    if (q_offset < 0 || window < 0 || softcap < 0) return -1;
+    return 0;
+}
+
+/* Mask of the card's pseudo-code: causal, and for a local layer also within
+ * the window. The window keeps the key at distance 0 (the query itself) and
+ * the window-1 keys before it: "Gemma 2 Guide" code builds the local mask with
+ * tril(diagonal=-W) and the card's paper-vs-code notes state the lower bound
+ * as "position greater than pos - W". */
+static int visible(int64_t p, int64_t j, int64_t window) {
+    if (j > p) return 0;
+    if (window > 0 && p - j >= window) return 0;
+    return 1;
+}
+
+/* Capped logit of key j for the (already scaled) query qs.
+ * Soft-cap formula: "Gemma 2 Guide", section 1, cap_val * tanh(logits / cap_val),
+ * with cap_val = 50 for attention; the card applies it to every logit before
+ * the mask. softcap == 0 means the cap is switched off. */
+static double capped_logit(const double* qs, const uint16_t* krow, int64_t d, double softcap) {
+    double x = 0.0;
+    for (int64_t c = 0; c < d; ++c) x += qs[c] * widen(krow[c]);
+    if (softcap > 0.0) x = softcap * tanh(x / softcap);
+    return x;
+}
+
+/* One query row (b, i, h): fills s[0..S) with the masked capped logits and,
+ * when out_row/lse are given, the mixed values and the log-sum-exp. */
+static void one_row(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                    int64_t b, int64_t i, int64_t h,
+                    int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                    int64_t q_offset, double query_scale, double softcap, int64_t window,
+                    double* qs, double* s, double* w, double* out_row, double* lse) {
+    const int64_t group = H / Hkv;
+    const int64_t g = h / group;
+    const int64_t p = i + q_offset;
+    const uint16_t* qrow = q + ((b * T + i) * H + h) * d;
+
+    /* queries = queries * query_scale */
+    for (int64_t c = 0; c < d; ++c) qs[c] = query_scale * widen(qrow[c]);
+
+    /* logits -> soft-cap -> where(mask, logits, -inf) */
+    for (int64_t j = 0; j < S; ++j) {
+        const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
+        double sj = capped_logit(qs, krow, d, softcap);
+        s[j] = visible(p, j, window) ? sj : -INFINITY;
+    }
+
+    /* softmax over keys */
+    double m = -INFINITY;
+    for (int64_t j = 0; j < S; ++j)
+        if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < S; ++j) {
+        w[j] = (s[j] == -INFINITY) ? 0.0 : exp(s[j] - m);
+        l += w[j];
+    }
+    for (int64_t j = 0; j < S; ++j) w[j] /= l;
+
+    /* mix the values */
+    if (out_row) {
+        for (int64_t c = 0; c < d; ++c) out_row[c] = 0.0;
+        for (int64_t j = 0; j < S; ++j) {
+            if (w[j] == 0.0) continue; /* masked: weight exactly 0 */
+            const uint16_t* vrow = v + ((b * S + j) * Hkv + g) * d;
+            for (int64_t c = 0; c < d; ++c) out_row[c] += w[j] * widen(vrow[c]);
+        }
+    }
+    if (lse) *lse = m + log(l);
+}
+
+int g2ref_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+               double* out, double* lse,
+               int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+               int64_t q_offset, double query_scale, double softcap, int64_t window) {
+    if (check_args(B, T, S, H, Hkv, d, q_offset, softcap, window)) return -1;
+    const int64_t nrows = B * T * H;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* qs = (double*)malloc(sizeof(double) * (size_t)d);
+        double* s = (double*)malloc(sizeof(double) * (size_t)S);
+        double* w = (double*)malloc(sizeof(double) * (size_t)S);
+        if (!qs || !s || !w) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t r = 0; r < nrows; ++r) {
+                const int64_t b = r / (T * H);
+                const int64_t i = (r / H) % T;
+                const int64_t h = r % H;
+                one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale, softcap,
+                        window, qs, s, w, out + ((b * T + i) * H + h) * d,
+                        lse + (b * H + h) * T + i);
+            }
+        }
+        free(qs);
+        free(s);
+        free(w);
+    }
+    return err ? -1 : 0;
+}
+
+int g2ref_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                    double* out, double* lse, const int64_t* rows, int64_t n,
+                    int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                    int64_t q_offset, double query_scale, double softcap, int64_t window) {
+    if (check_args(B, T, S, H, Hkv, d, q_offset, softcap, window)) return -1;
+    for (int64_t r = 0; r < n; ++r) {
+        const int64_t b = rows[3 * r], i = rows[3 * r + 1], h = rows[3 * r + 2];
+        if (b < 0 || b >= B || i < 0 || i >= T || h < 0 || h >= H) return -1;
+    }
+    int err = 0;
+#pragma omp parallel
+    {
+        double* qs = (double*)malloc(sizeof(double) * (size_t)d);
+        double* s = (double*)malloc(sizeof(double) * (size_t)S);
+        double* w = (double*)malloc(sizeof(double) * (size_t)S);
+        if (!qs || !s || !w) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < n; ++r) {
+                one_row(q, k, v, rows[3 * r], rows[3 * r + 1], rows[3 * r + 2], T, S, H, Hkv,
+                        d, q_offset, query_scale, softcap, window, qs, s, w, out + r * d,
+                        lse + r);
+            }
+        }
+        free(qs);
+        free(s);
+        free(w);
+    }
+    return err ? -1 : 0;
+}
+
+int g2ref_row_detail(const uint16_t* q, const uint16_t* k,
+                     double* s, double* w, int64_t b, int64_t i, int64_t h,
+                     int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                     int64_t q_offset, double query_scale, double softcap, int64_t window) {
+    if (check_args(B, T, S, H, Hkv, d, q_offset, softcap, window)) return -1;
+    if (b < 0 || b >= B || i < 0 || i >= T || h < 0 || h >= H) return -1;
+    double* qs = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!qs) return -1;
+    one_row(q, k, NULL, b, i, h, T, S, H, Hkv, d, q_offset, query_scale, softcap, window, qs,
+            s, w, NULL, NULL);
+    free(qs);
+    return 0;
+}
+
+void g2ref_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int g2ref_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
