@@ -1,0 +1,332 @@
+// api.cu -- C ABI of libg2attn (declared in include/g2attn.h): argument
+// checks, TMA descriptor encoding, launch configuration and the kernels
+// (compiled as one translation unit so the device error word is unique).
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "../../include/g2attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// Host-side helpers
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool finite_f(float x) { return isfinite(x) != 0; }
+
+unsigned long long wait_limit_ns() {
+    // Bounded waits inside the kernels give up after this long (default 4 s).
+    static unsigned long long v = [] {
+        const char* e = getenv("G2ATTN_WAIT_TIMEOUT_US");
+        unsigned long long us = e ? strtoull(e, nullptr, 10) : 0ull;
+        if (us == 0ull) us = 4000000ull;
+        return us * 1000ull;
+    }();
+    return v;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor map over a packed (rows, heads, d) tensor, viewed as
+// {d, rows, heads} so one box covers `box_rows` rows of `box_heads` heads.
+bool make_map(CUtensorMap* map, const void* ptr, int d, long long rows, int heads, int box_rows,
+              int box_heads) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(heads)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(heads) * d * 2,  // next row
+                             static_cast<cuuint64_t>(d) * 2};         // next head
+    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_heads)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    return n;
+}
+
+void fill_cap(float query_scale, float softcap, float& k_exp, float& cap_l2, float& scale_l2,
+              int& has_cap) {
+    has_cap = softcap > 0.f;
+    k_exp = has_cap ? 2.0f * query_scale * kLog2e / softcap : 0.f;
+    cap_l2 = has_cap ? softcap * kLog2e : 0.f;
+    scale_l2 = query_scale * kLog2e;
+}
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, long long total_q,
+                   long long total_k, g2::PfParams& P, cudaStream_t stream) {
+    using C = g2::PfCfg<D>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, D, total_q, P.H, g2::PF_QPOS, 2) ||
+        !make_map(&mk, k, D, total_k, P.Hkv, g2::PF_BN, 1) ||
+        !make_map(&mv, v, D, total_k, P.Hkv, C::VROWS, 1))
+        return G2ATTN_ERR_CUDA;
+    const int sms = num_sms();
+    if (sms <= 0) return G2ATTN_ERR_CUDA;
+    auto kern = g2::prefill_fwd_sm100<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+        return G2ATTN_ERR_CUDA;
+    const int grid = P.num_units < sms ? P.num_units : sms;
+    kern<<<grid, g2::PF_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, P);
+    return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+}
+
+int dispatch_prefill(int d, const void* q, const void* k, const void* v, long long tq,
+                     long long tk, g2::PfParams& P, cudaStream_t st) {
+    switch (d) {
+        case 64: return launch_prefill<64>(q, k, v, tq, tk, P, st);
+        case 128: return launch_prefill<128>(q, k, v, tq, tk, P, st);
+        case 256: return launch_prefill<256>(q, k, v, tq, tk, P, st);
+        default: return G2ATTN_ERR_UNSUPPORTED;
+    }
+}
+
+int check_common(int H, int Hkv, int d, float query_scale, float softcap, int window) {
+    if (H <= 0 || Hkv <= 0) return G2ATTN_ERR_INVALID_ARG;
+    if (!finite_f(query_scale) || !finite_f(softcap) || softcap < 0.f || window < 0)
+        return G2ATTN_ERR_INVALID_ARG;
+    if (H != 2 * Hkv) return G2ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return G2ATTN_ERR_UNSUPPORTED;
+    return G2ATTN_OK;
+}
+
+// Decode split plan: chunk of keys per CTA. Depends only on the sizes, so the
+// workspace size query and the launch agree without a device query.
+int decode_chunk(int num_seqs, int H, int max_len) {
+    int chunk = g2::DEC_MAX_CHUNK;
+    const long long kv_heads = static_cast<long long>(num_seqs) * (H / 2 > 0 ? H / 2 : 1);
+    while (chunk > 64 && kv_heads * ((max_len + chunk - 1) / chunk) < 1184) chunk >>= 1;
+    return chunk;
+}
+
+size_t decode_ws_bytes(int num_seqs, int H, int d, int max_len, int chunk) {
+    const size_t splits = static_cast<size_t>((max_len + chunk - 1) / chunk);
+    const size_t slots = static_cast<size_t>(num_seqs) * H * splits;
+    size_t ml = slots * 2 * sizeof(float);
+    ml = (ml + 255) & ~static_cast<size_t>(255);
+    return ml + slots * static_cast<size_t>(d) * sizeof(float);
+}
+
+template <int D>
+int launch_decode(g2::DecParams& P, cudaStream_t stream) {
+    dim3 grid(P.max_splits, P.Hkv, P.num_seqs);
+    g2::decode_split<D><<<grid, g2::DEC_THREADS, 0, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
+    const int warps = P.num_seqs * P.H;
+    g2::decode_merge<D><<<(warps + 3) / 4, 128, 0, stream>>>(P);
+    return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+}
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        g2::mbar_init(&bar, 1);
+        abort_flag = 0;
+        g2::fence_mbar_init();
+    }
+    __syncthreads();
+    // Nothing ever arrives on `bar`: the wait must give up after limit_ns.
+    if (threadIdx.x == 0)
+        g2::mbar_wait(&bar, 0, &abort_flag, limit_ns, g2::SITE_SELFTEST);
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+int g2attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                   int T, int S, int H, int Hkv, int d, int q_offset, float query_scale,
+                   float softcap, int window, g2attn_stream_t stream) {
+    if (!q || !k || !v || !out) return G2ATTN_ERR_INVALID_ARG;
+    if (B <= 0 || T <= 0 || S <= 0 || q_offset < 0 ||
+        static_cast<long long>(q_offset) + T > S)
+        return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (lse && !aligned16(lse)))
+        return G2ATTN_ERR_MISALIGNED;
+    const long long tq = static_cast<long long>(B) * T, tk = static_cast<long long>(B) * S;
+    if (tq > INT32_MAX || tk > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    g2::PfParams P{};
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    P.num_seqs = B;
+    P.T = T;
+    P.S = S;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.q_offset = q_offset;
+    P.window = window;
+    P.varlen = 0;
+    P.total_q = static_cast<int>(tq);
+    P.max_units_per_seq_tiles = (T + g2::PF_QPOS - 1) / g2::PF_QPOS;
+    const long long units = static_cast<long long>(P.max_units_per_seq_tiles) * B * Hkv;
+    if (units > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    P.num_units = static_cast<int>(units);
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    P.timeout_ns = wait_limit_ns();
+    return dispatch_prefill(d, q, k, v, tq, tk, P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int g2attn_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                          const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                          int total_q, int total_k, int max_T, int max_S, int H, int Hkv, int d,
+                          float query_scale, float softcap, int window, g2attn_stream_t stream) {
+    if (!q || !k || !v || !out || !cu_seqlens_q || !cu_seqlens_k) return G2ATTN_ERR_INVALID_ARG;
+    if (num_seqs <= 0 || total_q <= 0 || total_k <= 0 || max_T <= 0 || max_S <= 0 ||
+        max_T > max_S || max_T > total_q || max_S > total_k)
+        return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (num_seqs > g2::PfCfg<64>::MAX_SEQ_TABLE) return G2ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+        return G2ATTN_ERR_MISALIGNED;
+    g2::PfParams P{};
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    P.cu_q = cu_seqlens_q;
+    P.cu_k = cu_seqlens_k;
+    P.num_seqs = num_seqs;
+    P.T = max_T;
+    P.S = max_S;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.window = window;
+    P.varlen = 1;
+    P.total_q = total_q;
+    // Units are enumerated on the device from cu_seqlens_q; the grid is sized
+    // from an upper bound and surplus units are skipped by the kernel.
+    const long long ub = (static_cast<long long>(total_q) / g2::PF_QPOS + num_seqs) * Hkv;
+    if (ub > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    P.num_units = static_cast<int>(ub);
+    P.max_units_per_seq_tiles = (max_T + g2::PF_QPOS - 1) / g2::PF_QPOS;
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    P.timeout_ns = wait_limit_ns();
+    return dispatch_prefill(d, q, k, v, total_q, total_k, P,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t g2attn_decode_workspace_size(int num_seqs, int H, int d, int max_cache_len) {
+    if (num_seqs <= 0 || H <= 0 || d <= 0 || max_cache_len <= 0) return 0;
+    return decode_ws_bytes(num_seqs, H, d, max_cache_len, decode_chunk(num_seqs, H, max_cache_len));
+}
+
+int g2attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                  const int* cu_seqlens_k, void* out, float* lse, int num_seqs, int total_k,
+                  int max_cache_len, int H, int Hkv, int d, float query_scale, float softcap,
+                  int window, void* workspace, size_t workspace_bytes, g2attn_stream_t stream) {
+    if (!q || !k_cache || !v_cache || !cu_seqlens_k || !out) return G2ATTN_ERR_INVALID_ARG;
+    if (num_seqs <= 0 || total_k <= 0 || max_cache_len <= 0) return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
+        (workspace && !aligned16(workspace)))
+        return G2ATTN_ERR_MISALIGNED;
+    const int chunk = decode_chunk(num_seqs, H, max_cache_len);
+    const size_t need = decode_ws_bytes(num_seqs, H, d, max_cache_len, chunk);
+    if (!workspace || workspace_bytes < need) return G2ATTN_ERR_WORKSPACE;
+    g2::DecParams P{};
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.k = static_cast<const __nv_bfloat16*>(k_cache);
+    P.v = static_cast<const __nv_bfloat16*>(v_cache);
+    P.cu_k = cu_seqlens_k;
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    const int splits = (max_cache_len + chunk - 1) / chunk;
+    size_t ml = static_cast<size_t>(num_seqs) * H * splits * 2 * sizeof(float);
+    ml = (ml + 255) & ~static_cast<size_t>(255);
+    P.ws_ml = static_cast<float*>(workspace);
+    P.ws_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + ml);
+    P.num_seqs = num_seqs;
+    P.total_k = total_k;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.window = window;
+    P.chunk = chunk;
+    P.max_splits = splits;
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (d) {
+        case 64: return launch_decode<64>(P, st);
+        case 128: return launch_decode<128>(P, st);
+        case 256: return launch_decode<256>(P, st);
+        default: return G2ATTN_ERR_UNSUPPORTED;
+    }
+}
+
+const char* g2attn_status_string(int status) {
+    switch (status) {
+        case G2ATTN_OK: return "ok";
+        case G2ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case G2ATTN_ERR_UNSUPPORTED: return "unsupported shape";
+        case G2ATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case G2ATTN_ERR_CUDA: return "CUDA call failed";
+        case G2ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case G2ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int g2attn_get_device_error(void) {
+    unsigned int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return G2ATTN_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g2::g_device_error, sizeof(v)) != cudaSuccess)
+        return G2ATTN_ERR_CUDA;
+    if (v == 0) return G2ATTN_OK;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g2::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return G2ATTN_ERR_CUDA;
+    return G2ATTN_ERR_DEVICE_TIMEOUT;
+}
+
+int g2attn_selftest_wait_timeout(int timeout_us) {
+    if (timeout_us < 1 || timeout_us > 1000000) return G2ATTN_ERR_INVALID_ARG;
+    int pre = g2attn_get_device_error();  // start from a clear word
+    if (pre == G2ATTN_ERR_CUDA) return pre;
+    selftest_wait_kernel<<<1, 32>>>(static_cast<unsigned long long>(timeout_us) * 1000ull);
+    if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
+    return g2attn_get_device_error();
+}
+
+}  // extern "C"

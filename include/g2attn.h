@@ -1,0 +1,147 @@
+/*
+ * g2attn.h -- libg2attn: Gemma 2 soft-capped local/global attention forward
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation (Gemma 2 card, "Method", per-layer attention pseudo-code; the
+ * soft-cap formula is the "Gemma 2 Guide", section 1): for every query row i
+ * at absolute position p = i + q_offset and query head h, with KV head
+ * g = h / 2 (two query heads share one KV head: the card's "num_groups = 2"):
+ *
+ *   x_j  = query_scale * (q[i,h,:] . k[j,g,:])
+ *   s_j  = softcap * tanh(x_j / softcap)        (softcap == 0: s_j = x_j)
+ *   key j is visible iff j <= p and (window == 0 or p - j < window)
+ *   out[i,h,:] = sum_j softmax_j(s)_j * v[j,g,:]        over visible j
+ *   lse[h,i]   = ln sum_{visible j} exp(s_j)
+ *
+ * window == 0 is a global layer (full causal span); window == W > 0 is a local
+ * layer that keeps the W most recent keys, the query's own key included
+ * (Gemma 2 uses W = 4096 on local layers and softcap = 50 on both).
+ *
+ * Common rules for every entry point:
+ *  - Tensors q, k, v, out, caches are bf16, row-major, head dimension
+ *    contiguous; lse is fp32. Every pointer is device memory owned by the
+ *    caller; the library never allocates or frees device memory and keeps no
+ *    pointer after the call returns. lse may be NULL (then it is not written).
+ *  - d must be 64, 128 or 256; H must equal 2 * Hkv.
+ *  - Tensor pointers must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream). Arguments are checked on the host before any launch; on an
+ *    argument error nothing is launched and nothing is written.
+ *  - The host never reads device memory; cu_seqlens arrays stay on the device.
+ *  - Return value: a g2attn_status code.
+ */
+#ifndef G2ATTN_H
+#define G2ATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define G2ATTN_API __attribute__((visibility("default")))
+#else
+#define G2ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* g2attn_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    G2ATTN_OK = 0,
+    G2ATTN_ERR_INVALID_ARG = 1,    /* a size, scale, cap or window is out of range */
+    G2ATTN_ERR_UNSUPPORTED = 2,    /* d or H/Hkv outside what the kernels implement */
+    G2ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
+    G2ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
+    G2ATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting (see g2attn_get_device_error) */
+    G2ATTN_ERR_WORKSPACE = 6       /* decode workspace NULL or smaller than required */
+} g2attn_status;
+
+/*
+ * Dense prefill of one attention layer.
+ *   q   (B, T, H, d)      queries of rows i = 0..T-1 at positions q_offset + i
+ *   k,v (B, S, Hkv, d)    keys and values at positions 0..S-1
+ *   out (B, T, H, d)      bf16 output
+ *   lse (B, H, T)         fp32 natural-log log-sum-exp of the capped logits
+ * Requires B, T, S >= 1, 0 <= q_offset, q_offset + T <= S, window >= 0,
+ * finite query_scale, finite softcap >= 0.
+ * Source: Gemma 2 card, "Method" (attention_layer pseudo-code: queries
+ * (B,T,H,d), keys/values (B,S,K,d), K = H/2, cap 50, causal and 4096 window).
+ */
+G2ATTN_API int g2attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
+                   int B, int T, int S, int H, int Hkv, int d, int q_offset,
+                   float query_scale, float softcap, int window, g2attn_stream_t stream);
+
+/*
+ * Packed variable-length prefill. Sequence s owns query rows
+ * cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and key rows cu_seqlens_k[s] ..
+ * cu_seqlens_k[s+1]-1; with T_s and S_s its lengths, its queries sit at the
+ * last T_s positions of its keys (q_offset_s = S_s - T_s; a chunked-prefill
+ * tail has T_s < S_s). Each sequence is the dense layer above with B = 1.
+ *   q   (total_q, H, d), k and v (total_k, Hkv, d), out like q,
+ *   lse (H, total_q) fp32.
+ *   cu_seqlens_q, cu_seqlens_k: device int32 arrays of num_seqs + 1 entries,
+ *   non-decreasing, starting at 0, ending at total_q / total_k, with
+ *   T_s <= S_s, T_s <= max_T and S_s <= max_S for every sequence (the kernel
+ *   cannot check these; a violation gives undefined results, never an
+ *   out-of-bounds access of q/k/v/out/lse, which are bounded by total_q/k).
+ * total_q and total_k are the packed extents (the host does not read the
+ * device arrays). Source: as g2attn_prefill; the packing is this library's.
+ */
+G2ATTN_API int g2attn_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                          const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                          int total_q, int total_k, int max_T, int max_S,
+                          int H, int Hkv, int d, float query_scale, float softcap, int window,
+                          g2attn_stream_t stream);
+
+/*
+ * Bytes of device workspace g2attn_decode needs for these sizes (split-KV
+ * partial results: per sequence, query head and split, a running max, a sum
+ * and d accumulators, fp32). Depends only on the arguments.
+ */
+G2ATTN_API size_t g2attn_decode_workspace_size(int num_seqs, int H, int d, int max_cache_len);
+
+/*
+ * Decode: one new query per sequence over that sequence's KV cache.
+ *   q (num_seqs, H, d); k_cache, v_cache (total_k, Hkv, d) packed by
+ *   cu_seqlens_k (device int32, num_seqs + 1 entries, L_s = difference,
+ *   1 <= L_s <= max_cache_len); the query of sequence s sits at position
+ *   L_s - 1, so it sees keys max(0, L_s - window) .. L_s - 1 on a local
+ *   layer and 0 .. L_s - 1 on a global one.
+ *   out (num_seqs, H, d) bf16; lse (num_seqs, H) fp32.
+ *   workspace: device memory of at least g2attn_decode_workspace_size(...)
+ *   bytes, 16-byte aligned, owned by the caller; no initial contents needed.
+ * Source: the Guide's serving notes (local layers only need the last 4,096
+ * cached tokens, "Interleaved Local Sliding Window and Global Attention").
+ */
+G2ATTN_API int g2attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                  const int* cu_seqlens_k, void* out, float* lse,
+                  int num_seqs, int total_k, int max_cache_len, int H, int Hkv, int d,
+                  float query_scale, float softcap, int window,
+                  void* workspace, size_t workspace_bytes, g2attn_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+G2ATTN_API const char* g2attn_status_string(int status);
+
+/*
+ * Sticky device-side error word of the current device: nonzero after a
+ * kernel gave up on a bounded wait (G2ATTN_ERR_DEVICE_TIMEOUT). Reading it
+ * synchronizes the device and clears it. Returns G2ATTN_OK when clear,
+ * G2ATTN_ERR_DEVICE_TIMEOUT when set, G2ATTN_ERR_CUDA if it cannot be read.
+ */
+G2ATTN_API int g2attn_get_device_error(void);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one tiny kernel that waits
+ * on a shared-memory barrier nothing will ever complete, with a limit of
+ * timeout_us microseconds (1..1000000), then reads and clears the device
+ * error word. Returns G2ATTN_ERR_DEVICE_TIMEOUT when the wait gave up as it
+ * should (the GPU context stays usable), another code otherwise. No fault,
+ * trap or hang is involved.
+ */
+G2ATTN_API int g2attn_selftest_wait_timeout(int timeout_us);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* G2ATTN_H */

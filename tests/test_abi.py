@@ -1,0 +1,111 @@
+"""The C ABI library: it loads, exports every entry point include/g2attn.h
+declares, and rejects bad arguments on the host before any launch (these
+checks run without a GPU: no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import global_soft_capped_b200 as g2
+from global_soft_capped_b200 import build as g2build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "g2attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    g2build.build()
+    return g2.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"G2ATTN_API\s+[\w\s\*]*?\b(g2attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_symbols() == sorted(g2.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {g2.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (g2attn_\w+)", out))
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings(lib):
+    names = {g2.g2attn_status_string(i) for i in range(7)}
+    assert len(names) == 7
+    assert g2.g2attn_status_string(99) == "unknown status"
+
+
+def test_workspace_size_is_host_only_and_monotone(lib):
+    a = g2.g2attn_decode_workspace_size(64, 32, 128, 8192)
+    b = g2.g2attn_decode_workspace_size(64, 32, 128, 16384)
+    assert 0 < a < b
+    assert g2.g2attn_decode_workspace_size(0, 32, 128, 8192) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: calls fail before launch
+
+
+def prefill_args(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, B=1, T=64, S=64, H=8, Hkv=4, d=256,
+             q_offset=0, query_scale=0.0625, softcap=50.0, window=0, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(B=0), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(T=0), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(q_offset=-1), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(q_offset=1), g2.G2ATTN_ERR_INVALID_ARG),          # q_offset + T > S
+    (dict(window=-1), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(softcap=-1.0), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(softcap=float("inf")), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(query_scale=float("nan")), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(H=6), g2.G2ATTN_ERR_UNSUPPORTED),                 # H != 2*Hkv
+    (dict(d=96), g2.G2ATTN_ERR_UNSUPPORTED),
+    (dict(k=ctypes.c_void_p((1 << 20) + 8)), g2.G2ATTN_ERR_MISALIGNED),
+])
+def test_prefill_rejects_before_launch(lib, kw, status):
+    assert g2.g2attn_prefill(*prefill_args(**kw)) == status
+
+
+def test_varlen_and_decode_reject_before_launch(lib):
+    cu = ctypes.c_void_p(1 << 21)
+    base = [FAKE, FAKE, FAKE, FAKE, None, cu, cu, 2, 128, 128, 64, 64, 8, 4, 128, 0.1, 50.0, 0,
+            None]
+    assert g2.g2attn_prefill_varlen(*base[:5], None, *base[6:]) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(base)
+    bad[10] = 100  # max_T > max_S
+    assert g2.g2attn_prefill_varlen(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(base)
+    bad[7] = 5000  # more sequences than the per-launch table holds
+    assert g2.g2attn_prefill_varlen(*bad) == g2.G2ATTN_ERR_UNSUPPORTED
+
+    dec = [FAKE, FAKE, FAKE, cu, FAKE, None, 4, 4096, 1024, 32, 16, 128, 0.083, 50.0, 4096,
+           FAKE, 16, None]
+    assert g2.g2attn_decode(*dec) == g2.G2ATTN_ERR_WORKSPACE          # 16 bytes is too small
+    bad = list(dec)
+    bad[15] = None
+    assert g2.g2attn_decode(*bad) == g2.G2ATTN_ERR_WORKSPACE
+    bad = list(dec)
+    bad[11] = 80
+    assert g2.g2attn_decode(*bad) == g2.G2ATTN_ERR_UNSUPPORTED
+    bad = list(dec)
+    bad[6] = 0
+    assert g2.g2attn_decode(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(g2, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(g2, "_lib", None)
+    with pytest.raises(RuntimeError, match="libg2attn.so is missing"):
+        g2.load_library()
