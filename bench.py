@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of libg2attn on B200: useful attention TFLOP/s (prefill) and KV GB/s (decode).
+
+One step = one pass of the prefill hot path over the 2B-shaped layer pair
+(B=1, T=S=8192, H=8, Hkv=4, d=256, query_scale 1/16, softcap 50): the local
+layer (window 4096) and the global layer, both through the C ABI. Useful FLOPs
+count 4*d per visible (query, key, head) triple only. Inputs live in HBM; the
+L2 is flushed (a 512 MiB write) between timed steps, outside the timed events.
+
+Printed (rank 0, one JSON line): the contract keys, plus
+  roofline      dominant kernel (prefill_fwd_sm100<256>) vs measured bf16 peak
+  cpu_baseline  the fp64 oracle on the host cores on a bounded row sample
+  e2e           the same metric with pinned-host inputs and outputs copied
+                inside the timed region
+  clocks        nvidia-smi samples taken during the timed region
+  layers        per-layer times of the step
+  extra         9B pair (local/global separately), 27B decode (KV GB/s,
+                tokens/s) and the 9B ragged varlen prefill
+
+`--impl reference` times the fp64 oracle (the reference arm of this build)
+on the host cores on bounded samples of the same workload.
+Multi-GPU (torchrun): every rank runs its own replica (the units are
+independent; there is no data-path collective); value = total useful FLOPs
+of all ranks / max-over-ranks device time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from global_soft_capped_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs, varlen_inputs  # noqa: E402
+
+METRIC = "useful attention TFLOP/s (prefill) and KV GB/s (decode) vs B200 roofline"
+WORKLOAD = "2b"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# work counts (host arithmetic on sizes only)
+# ---------------------------------------------------------------------------
+def visible_pairs(T, S, q_offset, window):
+    """Number of visible (query row, key) pairs of one (batch, head)."""
+    p = np.arange(T, dtype=np.int64) + q_offset
+    hi = np.minimum(p, S - 1)
+    lo = np.maximum(0, p - window + 1) if window > 0 else np.zeros_like(p)
+    return int(np.sum(hi - lo + 1))
+
+
+def prefill_flops(B, T, S, H, d, q_offset, window):
+    return 4.0 * d * H * B * visible_pairs(T, S, q_offset, window)
+
+
+def varlen_flops(Ts, Ss, H, d, window):
+    return sum(4.0 * d * H * visible_pairs(t, s, s - t, window) for t, s in zip(Ts, Ss))
+
+
+def decode_kv_bytes(lengths, Hkv, d, window):
+    rows = sum(min(L, window) if window > 0 else L for L in lengths)
+    return rows * Hkv * d * 2 * 2  # K and V, bf16
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("prefill_sm100.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "global_soft_capped_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, units_now):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, scaled by units processed; None if the kernel source changed."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        rec = json.load(open(path)).get(kernel_key)
+    except Exception:
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec["bytes_per_launch"] * units_now / rec["units"]
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"g2attn_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm = float(parts[1])
+                mx = float(parts[2])
+                pw = float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else 0.0
+            except ValueError:
+                continue
+            if pw > 150.0:  # under load
+                sms.append(sm)
+            for n, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "samples_under_load": len(sms), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, dev):
+    import global_soft_capped_b200 as g2
+    g2.load_library()
+    w = WORKLOADS[WORKLOAD]
+    q, k, v = prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed + rank)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    outs = {lay: torch.empty_like(qd) for lay in ("local", "global")}
+    lses = {lay: torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+            for lay in ("local", "global")}
+    windows = {"local": w.window_local, "global": 0}
+    flops = {lay: prefill_flops(w.B, w.T, w.S, w.H, w.d, 0, windows[lay]) for lay in windows}
+    step_flops = sum(flops.values())
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def layer(lay):
+        g2.prefill(qd, kd, vd, query_scale=w.query_scale, softcap=w.softcap,
+                   window=windows[lay], out=outs[lay], lse=lses[lay], stream=stream)
+
+    for _ in range(args.warmup):
+        layer("local")
+        layer("global")
+    torch.cuda.synchronize()
+
+    nsteps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(nsteps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        layer("local")
+        ev[i][1].record(stream)
+        layer("global")
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    loc = [ev[i][0].elapsed_time(ev[i][1]) for i in range(nsteps)]
+    glo = [ev[i][1].elapsed_time(ev[i][2]) for i in range(nsteps)]
+    total_ms = sum(loc) + sum(glo)
+    total_ms_t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(total_ms_t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(total_ms_t.item())
+    ms_per_step = total_ms / nsteps
+    value = step_flops * world / (ms_per_step * 1e-3) / 1e12
+
+    pk, pk_kind = peaks()
+    avg_loc, avg_glo = sum(loc) / nsteps, sum(glo) / nsteps
+    ach = (flops["local"] + flops["global"]) / ((avg_loc + avg_glo) * 1e-3) / 1e12
+    roof = {"kernel": "prefill_fwd_sm100<256>", "bound": "tensor", "achieved": round(ach, 2),
+            "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
+            "peak_kind": f"{pk_kind} bf16 dense (burst; kernel timed alone)",
+            "traffic": ncu_traffic("prefill_fwd_sm100<256>/2b_pair", 1.0),
+            "algorithmic": "4*d*H*B per visible (query,key) pair; 0.4811 TFLOP per step"}
+
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": nsteps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded iid N(0,1) bf16)",
+        "config": {"workload": "2b_prefill_pair", "B": w.B, "T": w.T, "S": w.S, "H": w.H,
+                   "Hkv": w.Hkv, "d": w.d, "window_local": w.window_local,
+                   "query_scale": w.query_scale, "softcap": w.softcap,
+                   "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between steps by a 512 MiB write outside the timed events"},
+        "gpu_launches": 2 * nsteps,
+        "wall_s_timed_region": round(t_wall, 3),
+        "roofline": roof,
+        "clocks": clk,
+        "layers": {"local": {"ms": round(avg_loc, 5),
+                             "tflops": round(flops["local"] / (avg_loc * 1e-3) / 1e12, 2)},
+                   "global": {"ms": round(avg_glo, 5),
+                              "tflops": round(flops["global"] / (avg_glo * 1e-3) / 1e12, 2)}},
+    }
+
+    # ---- e2e: pinned host inputs -> device -> both layers -> host outputs
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = {lay: torch.empty(q.shape, dtype=q.dtype).pin_memory() for lay in windows}
+    lh = {lay: torch.empty((w.B, w.H, w.T), dtype=torch.float32).pin_memory() for lay in windows}
+    e2e_steps = max(3, min(nsteps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(e2e_steps + 2):
+        if it == 2:
+            torch.cuda.synchronize()
+            e0.record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        for lay in ("local", "global"):
+            layer(lay)
+            oh[lay].copy_(outs[lay], non_blocking=True)
+            lh[lay].copy_(lses[lay], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = sum(oh[l].numel() * 2 + lh[l].numel() * 4 for l in windows)
+    result["e2e"] = {"value": round(step_flops * world / (e2e_ms * 1e-3) / 1e12, 3),
+                     "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                     "ms_per_step": round(e2e_ms, 4),
+                     "path": "pinned host q,k,v -> HBM -> g2attn_prefill x2 -> host out, lse"}
+
+    if not args.no_extra:
+        result["extra"] = extra_workloads(g2, dev, stream, flush)
+    del flush
+    return result
+
+
+def time_launches(fn, flush, stream, reps=10, warm=3):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts), min(ts)
+
+
+def extra_workloads(g2, dev, stream, flush):
+    pk, _ = peaks()
+    res = {}
+    # 9B batched pair, local and global reported separately
+    w = WORKLOADS["9b"]
+    q, k, v = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+    r9 = {}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        f = prefill_flops(w.B, w.T, w.S, w.H, w.d, 0, win)
+        med, best = time_launches(lambda: g2.prefill(q, k, v, query_scale=w.query_scale,
+                                                     softcap=w.softcap, window=win, out=out,
+                                                     lse=lse, stream=stream), flush, stream)
+        r9[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                   "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+    res["9b_prefill"] = r9
+    del q, k, v, out, lse
+
+    # 27B decode
+    w = WORKLOADS["27b_decode"]
+    lengths, cu, q, k, v = decode_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv, w.d, w.std,
+                                         w.seed)
+    q, k, v, cu = q.to(dev), k.to(dev), v.to(dev), cu.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], w.H), dtype=torch.float32, device=dev)
+    ws = g2.decode_workspace(q.shape[0], w.H, w.d, max(lengths), dev)
+    rd = {}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        nbytes = decode_kv_bytes(lengths, w.Hkv, w.d, win)
+        med, best = time_launches(lambda: g2.decode(q, k, v, cu, max(lengths),
+                                                    query_scale=w.query_scale, softcap=w.softcap,
+                                                    window=win, out=out, lse=lse, workspace=ws,
+                                                    stream=stream), flush, stream)
+        gbs = nbytes / (med * 1e-3) / 1e9
+        rd[lay] = {"ms": round(med, 4), "kv_GBps": round(gbs, 1),
+                   "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                   "tokens_per_s": round(len(lengths) / (med * 1e-3), 1), "kv_bytes": nbytes}
+    res["27b_decode"] = rd
+    del q, k, v, out, lse, ws
+
+    # 9B ragged packed prefill (16 sequences + chunked-prefill tail)
+    w = WORKLOADS["9b_varlen"]
+    Ts, Ss, cq, ck, q, k, v = varlen_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv, w.d,
+                                            w.std, w.seed, tail_T=w.tail_T, tail_S=w.tail_S)
+    q, k, v, cq, ck = q.to(dev), k.to(dev), v.to(dev), cq.to(dev), ck.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=dev)
+    rv = {}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        f = varlen_flops(Ts, Ss, w.H, w.d, win)
+        med, best = time_launches(lambda: g2.prefill_varlen(q, k, v, cq, ck, max(Ts), max(Ss),
+                                                            query_scale=w.query_scale,
+                                                            softcap=w.softcap, window=win,
+                                                            out=out, lse=lse, stream=stream),
+                                  flush, stream)
+        rv[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                   "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+    res["9b_varlen"] = rv
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline / reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def oracle_sample_rate(target_s=12.0, seed=0):
+    """Useful TFLOP/s of the oracle on a bounded sample of the 2B pair: query
+    rows spread over positions and heads of both layers; useful FLOPs of a
+    row = 4*d*(visible keys of that row)."""
+    import oracle
+    w = WORKLOADS[WORKLOAD]
+    q, k, v = prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed)
+    rng = np.random.default_rng(seed)
+    threads = oracle.max_threads()
+
+    def run(nrows):
+        t0 = time.perf_counter()
+        useful = 0.0
+        for win in (w.window_local, 0):
+            pos = rng.integers(0, w.T, nrows)
+            heads = rng.integers(0, w.H, nrows)
+            rows = np.stack([np.zeros(nrows, np.int64), pos, heads], 1)
+            oracle.attn_rows(q, k, v, rows, query_scale=w.query_scale, softcap=w.softcap,
+                             window=win)
+            vis = np.minimum(pos + 1, win) if win else pos + 1
+            useful += float(np.sum(4.0 * w.d * vis))
+        return time.perf_counter() - t0, useful
+
+    n = max(threads, 8)
+    dt, _ = run(n)
+    n = int(max(threads, min(200000, n * target_s / max(dt, 1e-3))))
+    dt, useful = run(n)
+    return useful / dt / 1e12, {"kind": "oracle", "cores": threads,
+                                "sample": f"{2 * n} query rows (half local, half global) of the "
+                                          f"2B pair, uniform positions and heads",
+                                "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    rates = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        rate, info = oracle_sample_rate(target_s=max(2.0, 60.0 / (args.warmup + args.steps)),
+                                        seed=i)
+        if i >= args.warmup:
+            rates.append(rate)
+    value = statistics.median(rates)
+    w = WORKLOADS[WORKLOAD]
+    useful_step = sum(prefill_flops(w.B, w.T, w.S, w.H, w.d, 0, win) for win in (w.window_local, 0))
+    info = dict(info, value=value, unit="TFLOP/s")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": useful_step / (value * 1e12) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded iid N(0,1) bf16)",
+            "config": {"workload": "2b_prefill_pair", "B": w.B, "T": w.T, "S": w.S, "H": w.H,
+                       "Hkv": w.Hkv, "d": w.d, "window_local": w.window_local},
+            "cpu_baseline": info,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the 9B/decode/varlen extras")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if world > 1 and rank != 0:
+            return
+        res = run_reference(args, rank, world)
+        print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    # the oracle's thread pool is created before any GPU work (never forked after it)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, info = oracle_sample_rate()
+        cpu = dict(info, value=rate, unit="TFLOP/s")
+    res = run_ours(args, rank, world, dev)
+    if rank == 0:
+        if cpu is not None:
+            res["cpu_baseline"] = cpu
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

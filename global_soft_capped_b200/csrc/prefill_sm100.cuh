@@ -420,7 +420,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             pf_unit(P, pre, u, U);
             const int p = U.p_min + pr;  // absolute query position of this row
             float m_ref = -INFINITY;     // log2-domain reference max of the row
-            float l = 0.f;
+            float l = 0.f;               // sum of the fp32 weights (for lse)
+            float lr = 0.f;              // sum of the bf16-rounded weights (normalises O)
             for (int jj = 0; jj < U.nkt; ++jj) {
                 const uint32_t gt = tile + jj;
                 const uint32_t buf = gt & 1;
@@ -484,11 +485,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     }
                     tmem_wait_st();
                     l *= f;
+                    lr *= f;
                     if (need) m_ref = m_new;
                 }
                 if (m_ref == -INFINITY) m_ref = mt;
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                float lsum = 0.f;
+                // The PV product sees bf16(p); normalising O by the sum of the
+                // same rounded weights makes them sum to one exactly, so their
+                // rounding errors cancel against the row's mean value.
+                float lsum = 0.f, lrsum = 0.f;
 #pragma unroll
                 for (int c = 0; c < PF_BN / 64; ++c) {
                     uint32_t pk[32];
@@ -498,10 +503,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         const float b = ex2_approx(s[c * 64 + 2 * i + 1] - m_use);
                         lsum += a + b;
                         pk[i] = pack_bf16x2(a, b);
+                        lrsum += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u);
                     }
                     tmem_st32(s_addr + c * 32, pk);
                 }
                 l += lsum;
+                lr += lrsum;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[buf]);
@@ -516,7 +523,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             tc_fence_after();
             const bool valid = pr < U.tvalid;
             const int h = 2 * U.g + hl;
-            const float inv_l = 1.0f / l;
+            const float inv_l = 1.0f / lr;
             const size_t orow = static_cast<size_t>(U.qbase + U.t0 + pr) * P.H + h;
             __nv_bfloat16* optr = P.out + orow * D;
             const uint32_t o_addr = tmem + lane_addr;

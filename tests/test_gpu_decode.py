@@ -66,5 +66,5 @@ def test_decode_is_last_row_of_prefill():
     qf[0, -1] = q[0]
     po, pl = g2.prefill(qf.cuda(), k[None].cuda(), v[None].cuda(), query_scale=0.09, window=100)
     torch.cuda.synchronize()
-    check(out, po[0, -1].double().cpu().numpy(), lse, pl[0, :, -1].double().cpu().numpy(),
-          "decode vs prefill last row")
+    check(out[0], po[0, -1].double().cpu().numpy(), lse[0],
+          pl[0, :, -1].double().cpu().numpy(), "decode vs prefill last row")

@@ -50,7 +50,7 @@ EDGE = [
     (1, 77, 500, 2, 1, 256, 423, 0, 50.0, 0.0625, 1.0),
     (3, 100, 100, 4, 2, 64, 0, 4096, 50.0, 0.125, 1.0),
     (1, 190, 190, 2, 1, 128, 0, 50, 0.0, 0.09, 1.0),      # no cap
-    (1, 128, 128, 2, 1, 64, 0, 0, 50.0, 1.0, 2.0),        # logits well past the cap
+    (1, 128, 128, 2, 1, 64, 0, 0, 50.0, 4.0, 1.0),        # logits well past the cap
     (1, 192, 192, 2, 1, 256, 0, 70, 50.0, 0.25, 1.0),
 ]
 
