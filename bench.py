@@ -418,6 +418,47 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_single(args, dev):
+    """One kernel case only (for profiling): `<workload>:<layer>`, layer local|global."""
+    import global_soft_capped_b200 as g2
+    g2.load_library()
+    name, lay = args.single.split(":")
+    w = WORKLOADS[name]
+    win = w.window_local if lay == "local" else 0
+    stream = torch.cuda.current_stream()
+    if w.kind == "prefill":
+        q, k, v = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std,
+                                                      w.seed))
+        fn = lambda: g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap,
+                                window=win, stream=stream)
+    elif w.kind == "decode":
+        lengths, cu, q, k, v = decode_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv, w.d,
+                                             w.std, w.seed)
+        q, k, v, cu = q.to(dev), k.to(dev), v.to(dev), cu.to(dev)
+        ws = g2.decode_workspace(q.shape[0], w.H, w.d, max(lengths), dev)
+        fn = lambda: g2.decode(q, k, v, cu, max(lengths), query_scale=w.query_scale,
+                               softcap=w.softcap, window=win, workspace=ws, stream=stream)
+    else:
+        Ts, Ss, cq, ck, q, k, v = varlen_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv,
+                                                w.d, w.std, w.seed, tail_T=w.tail_T,
+                                                tail_S=w.tail_S)
+        q, k, v, cq, ck = q.to(dev), k.to(dev), v.to(dev), cq.to(dev), ck.to(dev)
+        fn = lambda: g2.prefill_varlen(q, k, v, cq, ck, max(Ts), max(Ss),
+                                       query_scale=w.query_scale, softcap=w.softcap,
+                                       window=win, stream=stream)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    print(json.dumps({"single": args.single, "steps": args.steps,
+                      "ms_per_launch": a.elapsed_time(b) / max(args.steps, 1)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -426,7 +467,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the 9B/decode/varlen extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single", default=None,
+                    help="profile aid: run one case only, e.g. 9b:global or 27b_decode:local")
     args = ap.parse_args()
+    if args.single:
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        run_single(args, dev)
+        return
     if args.warmup < 3:
         args.warmup = 3
 
