@@ -4,7 +4,8 @@ Two layers:
 
 * The C entry points under their own names (``g2attn_prefill``,
   ``g2attn_prefill_varlen``, ``g2attn_decode_workspace_size``,
-  ``g2attn_decode``, ``g2attn_status_string``, ``g2attn_get_device_error``,
+  ``g2attn_decode``, ``g2attn_decode_noalloc``, ``g2attn_status_string``,
+  ``g2attn_get_device_error``,
   ``g2attn_selftest_wait_timeout``): plain argument marshalling of integers,
   floats and raw pointers through ctypes, returning the status code.
 * Tensor helpers (:func:`prefill`, :func:`prefill_varlen`, :func:`decode`)
@@ -36,6 +37,7 @@ EXPORTS = (
     "g2attn_prefill_varlen",
     "g2attn_decode_workspace_size",
     "g2attn_decode",
+    "g2attn_decode_noalloc",
     "g2attn_status_string",
     "g2attn_get_device_error",
     "g2attn_selftest_wait_timeout",
@@ -70,6 +72,8 @@ def load_library():
     lib.g2attn_decode_workspace_size.restype = SZ
     lib.g2attn_decode.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P, SZ, P]
     lib.g2attn_decode.restype = I
+    lib.g2attn_decode_noalloc.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P]
+    lib.g2attn_decode_noalloc.restype = I
     lib.g2attn_status_string.argtypes = [I]
     lib.g2attn_status_string.restype = ctypes.c_char_p
     lib.g2attn_get_device_error.argtypes = []
@@ -105,6 +109,15 @@ def g2attn_decode(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs, total_k
     return load_library().g2attn_decode(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs,
                                         total_k, max_cache_len, H, Hkv, d, query_scale, softcap,
                                         window, workspace, workspace_bytes, stream)
+
+
+def g2attn_decode_noalloc(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs, total_k,
+                          max_cache_len, H, Hkv, d, query_scale, softcap, window, stream):
+    """Decode with the library's static scratch instead of a caller workspace,
+    for callers that cannot allocate device memory at call time."""
+    return load_library().g2attn_decode_noalloc(q, k_cache, v_cache, cu_seqlens_k, out, lse,
+                                                num_seqs, total_k, max_cache_len, H, Hkv, d,
+                                                query_scale, softcap, window, stream)
 
 
 def g2attn_status_string(status):

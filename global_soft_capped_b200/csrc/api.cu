@@ -12,6 +12,11 @@
 #include "decode.cuh"
 #include "prefill_sm100.cuh"
 
+// Scratch of g2attn_decode_noalloc (see there): 24 MiB, reserved on every GPU
+// that loads the library until the process exits.
+constexpr size_t kNoAllocScratchBytes = 24u << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -167,6 +172,33 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
     __syncthreads();
 }
 
+// ---------------------------------------------------------------------------
+// Decode without any allocation: the split-KV partial results live in this
+// file-scope device array instead of a caller-provided workspace. It is
+// reserved on every GPU that loads the library, for the life of the process.
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. The host-side
+// name of the array is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return G2ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return G2ATTN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return G2ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -293,6 +325,31 @@ int g2attn_decode(const void* q, const void* k_cache, const void* v_cache,
         case 256: return launch_decode<256>(P, st);
         default: return G2ATTN_ERR_UNSUPPORTED;
     }
+}
+
+int g2attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                          const int* cu_seqlens_k, void* out, float* lse, int num_seqs,
+                          int total_k, int max_cache_len, int H, int Hkv, int d,
+                          float query_scale, float softcap, int window,
+                          g2attn_stream_t stream) {
+    // Size check first (host arithmetic only), so an oversized request is
+    // rejected before any CUDA call.
+    if (num_seqs > 0 && H > 0 && max_cache_len > 0 && (d == 64 || d == 128 || d == 256) &&
+        g2attn_decode_workspace_size(num_seqs, H, d, max_cache_len) > kNoAllocScratchBytes)
+        return G2ATTN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (!q || !k_cache || !v_cache || !cu_seqlens_k || !out || num_seqs <= 0 || total_k <= 0 ||
+        max_cache_len <= 0)
+        return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    // The decode kernels write every partial they later read, so the scratch
+    // needs no clearing between calls.
+    return g2attn_decode(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs, total_k,
+                         max_cache_len, H, Hkv, d, query_scale, softcap, window, scratch,
+                         kNoAllocScratchBytes, stream);
 }
 
 const char* g2attn_status_string(int status) {

@@ -120,6 +120,34 @@ G2ATTN_API int g2attn_decode(const void* q, const void* k_cache, const void* v_c
                   float query_scale, float softcap, int window,
                   void* workspace, size_t workspace_bytes, g2attn_stream_t stream);
 
+/*
+ * Decode without allocating: the same operation and arguments as
+ * g2attn_decode, minus the workspace. For callers that cannot allocate device
+ * memory at call time -- a serving loop whose device memory is planned up
+ * front by another allocator, a plug-in that is handed only its input and
+ * output pointers, or code that must not pay cudaMalloc's implicit device
+ * synchronisation. The split-KV partial results go to a static scratch array
+ * of 24 MiB inside the library, which every GPU that loads the library holds
+ * until the process exits; this call never calls cudaMalloc, cudaFree or any
+ * allocating routine. Inputs and outputs are still the caller's.
+ *   - Rejects with G2ATTN_ERR_WORKSPACE (before any CUDA call) when
+ *     g2attn_decode_workspace_size(num_seqs, H, d, max_cache_len) exceeds
+ *     24 MiB (25165824 bytes).
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one scratch array and leaves its
+ *     contents behind (nothing in it needs clearing: the kernels write every
+ *     partial before reading it). Calls that overlap on the GPU -- on
+ *     different streams, or from different host threads -- race on it and
+ *     must be serialised by the caller.
+ * The Gemma 2 pages have no counterpart to this entry point.
+ */
+G2ATTN_API int g2attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                          const int* cu_seqlens_k, void* out, float* lse,
+                          int num_seqs, int total_k, int max_cache_len, int H, int Hkv, int d,
+                          float query_scale, float softcap, int window, g2attn_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 G2ATTN_API const char* g2attn_status_string(int status);
 
