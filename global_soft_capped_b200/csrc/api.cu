@@ -91,6 +91,12 @@ void fill_cap(float query_scale, float softcap, float& k_exp, float& cap_l2, flo
     scale_l2 = query_scale * kLog2e;
 }
 
+void fill_poly(float query_scale, float softcap, g2::PfParams& P) {
+    P.u_scale = softcap > 0.f ? query_scale / softcap : 0.f;
+    const float a = fabsf(query_scale);
+    P.poly_acc_max = (softcap > 0.f && a > 0.f) ? g2::PF_POLY_U_MAX * softcap / a : INFINITY;
+}
+
 template <int D>
 int launch_prefill(const void* q, const void* k, const void* v, long long total_q,
                    long long total_k, g2::PfParams& P, cudaStream_t stream) {
@@ -234,6 +240,7 @@ int g2attn_prefill(const void* q, const void* k, const void* v, void* out, float
     if (units > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
     P.num_units = static_cast<int>(units);
     fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    fill_poly(query_scale, softcap, P);
     P.timeout_ns = wait_limit_ns();
     return dispatch_prefill(d, q, k, v, tq, tk, P, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -273,6 +280,7 @@ int g2attn_prefill_varlen(const void* q, const void* k, const void* v, void* out
     P.num_units = static_cast<int>(ub);
     P.max_units_per_seq_tiles = (max_T + g2::PF_QPOS - 1) / g2::PF_QPOS;
     fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    fill_poly(query_scale, softcap, P);
     P.timeout_ns = wait_limit_ns();
     return dispatch_prefill(d, q, k, v, total_q, total_k, P,
                             reinterpret_cast<cudaStream_t>(stream));

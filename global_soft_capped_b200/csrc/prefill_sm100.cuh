@@ -6,19 +6,25 @@
 // window on local layers, softmax over keys, grouped mix of the values);
 // cap formula from the "Gemma 2 Guide", section 1.
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialised):
-//   warp 0      TMA producer: Q tile once per work unit, then K/V tiles into a
+// Design (one persistent CTA per SM, 320 threads, warp-specialised):
+//   warps 0..7  softmax + epilogue: warps w and w+4 share MMA rows 32*(w%4)..+31
+//               (TMEM lanes of their sub-partition); warp w<4 takes key columns
+//               0..63 of every S tile and O columns 0..D/2-1, warp w+4 the rest.
+//               The pair exchanges its partial row maxima through shared memory
+//               once per tile (64-thread named barrier), so both halves use the
+//               same running max.
+//   warp 8      TMA producer: Q tile once per work unit, then K/V tiles into a
 //               ring of shared-memory slots (128-byte swizzle).
-//   warp 1      UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
+//   warp 9      UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
 //               O += P V with P read from TMEM; owns the TMEM allocation.
-//   warps 2..5  softmax + epilogue: thread r owns MMA row r (TMEM lane r).
 // A work unit is (sequence, KV head g, 64 query positions); its 128 MMA rows
 // are the two query heads 2g, 2g+1 that share KV head g (row = head_local*64 +
 // position), so each K/V tile feeds both heads. Only KV tiles that intersect
 // the causal band (and the window on local layers) are visited, and only
 // tiles that cross a band edge evaluate the mask.
-// Softmax: fp32, log2 domain. s2 = C*log2(e)*tanh(x/C) computed as
-// C*log2(e)*(1 - 2/(1 + 2^(2*x*log2(e)/C))) with ex2/rcp, then a running max
+// Softmax: fp32, log2 domain. s2 = C*log2(e)*tanh(x/C): when |x/C| <= 1/4 over
+// a warp's tile, by the Taylor series of tanh on the FMA pipe (packed f32x2);
+// otherwise as C*log2(e)*(1 - 2/(1 + 2^(2*x*log2(e)/C))) with ex2/rcp. Then a running max
 // per row with lazy rescaling of O (only when the max grows by more than
 // 2^8), p = 2^(s2 - m) rounded to bf16 for the PV product, row sum in fp32.
 // lse = ln2 * (m + log2(l)).
@@ -28,13 +34,23 @@
 
 namespace g2 {
 
-constexpr int PF_THREADS = 192;
+constexpr int PF_THREADS = 320;  // 8 softmax warps, producer, UMMA issuer
+constexpr int PF_WARP_PRODUCER = 8;
+constexpr int PF_WARP_MMA = 9;
+constexpr int PF_SOFTMAX_THREADS = 256;
 constexpr int PF_BM = 128;   // MMA rows per tile (64 positions x 2 heads)
 constexpr int PF_QPOS = 64;  // query positions per tile
 constexpr int PF_BN = 128;   // keys per KV tile
 constexpr int PF_TMEM_COLS = 512;
 constexpr int PF_S_COL0 = 256;  // S buffers at TMEM columns 256 and 384; O at 0
 constexpr float PF_RESCALE_LOG2 = 8.0f;
+// Taylor coefficients of tanh(u) = u (1 + c1 u^2 + c2 u^4 + c3 u^6 + c4 u^8 + ...):
+// -1/3, 2/15, -17/315, 62/2835 (the series of tanh, from its Bernoulli-number form).
+constexpr float kTanhC1 = -1.0f / 3.0f;
+constexpr float kTanhC2 = 2.0f / 15.0f;
+constexpr float kTanhC3 = -17.0f / 315.0f;
+constexpr float kTanhC4 = 62.0f / 2835.0f;
+constexpr float PF_POLY_U_MAX = 0.25f;  // |x / C| bound of the series path
 
 template <int D>
 struct PfCfg {
@@ -47,7 +63,8 @@ struct PfCfg {
     static constexpr int Q_BYTES = PF_BM * D * 2;
     static constexpr int MAX_SEQ_TABLE = 1024;  // varlen: per-sequence unit prefix table
     static constexpr int SMEM_TILES = Q_BYTES + NSLOT * SLOT_BYTES;
-    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + 4 * (MAX_SEQ_TABLE + 1);
+    static constexpr int CTRL_BYTES = 1024 + 2 * 2 * 128 * 4 + 128 * 2 * 2 * 4;
+    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + CTRL_BYTES + 4 * (MAX_SEQ_TABLE + 1);
     static_assert(KCOLS % 64 == 0 && VROWS % 16 == 0, "tile shapes");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -68,7 +85,9 @@ struct PfParams {
     int max_units_per_seq_tiles;  // dense: q tiles per sequence
     float k_exp;    // 2*alpha*log2(e)/C   (cap on)
     float cap_l2;   // C*log2(e)           (cap on)
-    float scale_l2; // alpha*log2(e)       (cap off)
+    float scale_l2; // alpha*log2(e)
+    float u_scale;  // alpha/C             (cap on)
+    float poly_acc_max;  // largest |q.k| for which |alpha q.k / C| <= PF_POLY_U_MAX
     int has_cap;
     unsigned long long timeout_ns;
 };
@@ -161,9 +180,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint64_t* drain = bars + 9;
     uint64_t* slot_full = bars + 10;              // [NSLOT]
     uint64_t* slot_empty = bars + 10 + C::NSLOT;  // [NSLOT]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 10 + 2 * C::NSLOT);
+    // softmax warp pairs: max exchange per tile parity [4][2], sum exchange [4]
+    uint64_t* xbar = bars + 10 + 2 * C::NSLOT;
+    uint64_t* sbar = xbar + 8;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sbar + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    int* pre = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
+    // partial row maxima of the two column halves, by tile parity: [2][2][128]
+    float* xmax = reinterpret_cast<float*>(base + C::SMEM_TILES + 1024);
+    // partial (l, lr) row sums of the two halves at the end of a unit: [2][128][2]
+    float* xsum = xmax + 2 * 2 * 128;
+    int* pre = reinterpret_cast<int*>(base + C::SMEM_TILES + C::CTRL_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -173,10 +199,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         mbar_init(q_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 128);
+            mbar_init(&p_full[i], PF_SOFTMAX_THREADS);
             mbar_init(&o_done[i], 1);
         }
-        mbar_init(o_free, 128);
+        mbar_init(o_free, PF_SOFTMAX_THREADS);
+        for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
+        for (int i = 0; i < 4; ++i) mbar_init(&sbar[i], 64);
         mbar_init(drain, 1);
         for (int i = 0; i < C::NSLOT; ++i) {
             mbar_init(&slot_full[i], 1);
@@ -208,11 +236,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             if (lane == 0) pre[P.num_seqs] = carry;
         }
     }
-    if (warp == 1) {
+    if (warp == PF_WARP_MMA) {
         tmem_alloc(tmem_holder, PF_TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == PF_WARP_PRODUCER && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -226,7 +254,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const int num_units = P.varlen ? min(P.num_units, pre[P.num_seqs]) : P.num_units;
     const uint64_t lim = P.timeout_ns;
 
-    if (warp == 0) {
+    if (warp == PF_WARP_PRODUCER) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t fill = 0;  // slot fills issued so far
@@ -300,7 +328,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             if (q_armed > 0) mbar_wait_drain(q_full, (q_armed - 1) & 1, lim);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == PF_WARP_MMA) {
         // ------------------------------------------------------------ UMMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(PF_BM, PF_BN, false);
@@ -314,11 +342,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
             auto issue_s = [&](uint32_t gt) -> bool {
                 const uint32_t buf = gt & 1;
-                if (gt >= 2) {  // S buffer reuse: P(gt-2) consumed by PV(gt-2)
-                    if (!mbar_wait(&o_done[buf], ((gt - 2) >> 1) & 1, abort_flag, lim,
-                                   SITE_MMA_O_DONE))
-                        return false;
-                }
+                // S(gt) overwrites P(gt-2) in the same TMEM columns. PV(gt-2) was
+                // issued earlier by this thread, and UMMAs issued by one thread
+                // execute in issue order, so no completion wait is needed here.
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + PF_S_COL0 + buf * PF_BN;
 #pragma unroll
@@ -406,10 +432,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int r = ((warp & 3) << 5) | lane;        // MMA row == TMEM lane
-        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        constexpr int HC = PF_BN / 2;                   // key columns per half
+        const int qd = warp & 3;                        // TMEM lane quadrant
+        const int half = warp >> 2;                     // column half of this warp
+        const int r = (qd << 5) | lane;                 // MMA row == TMEM lane
+        const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
         const int hl = r >> 6;                          // head within the pair
         const int pr = r & 63;                          // position within the tile
+        const int col0 = half * HC;                     // first S column of this warp
         uint32_t tile = 0;
         int unit_it = 0;
         bool ok = true;
@@ -420,8 +450,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             pf_unit(P, pre, u, U);
             const int p = U.p_min + pr;  // absolute query position of this row
             float m_ref = -INFINITY;     // log2-domain reference max of the row
-            float l = 0.f;               // sum of the fp32 weights (for lse)
-            float lr = 0.f;              // sum of the bf16-rounded weights (normalises O)
+            float l = 0.f;               // this half's sum of fp32 weights (for lse)
+            float lr = 0.f;              // this half's sum of bf16-rounded weights
             for (int jj = 0; jj < U.nkt; ++jj) {
                 const uint32_t gt = tile + jj;
                 const uint32_t buf = gt & 1;
@@ -430,52 +460,107 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_addr + PF_S_COL0 + buf * PF_BN;
-                float s[PF_BN];
+                float s[HC];
+                {  // two TMEM loads in flight, one wait
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32_async(s_addr + col0, v0);
+                    tmem_ld32_async(s_addr + col0 + 32, v1);
+                    tmem_wait_ld();
+                    tmem_reg_fence(v0);
+                    tmem_reg_fence(v1);
 #pragma unroll
-                for (int c = 0; c < PF_BN / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(s_addr + c * 32, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        s[i] = __uint_as_float(v0[i]);
+                        s[32 + i] = __uint_as_float(v1[i]);
+                    }
                 }
                 // capped logit in log2 units
                 if (P.has_cap) {
+                    float am[8];
 #pragma unroll
-                    for (int i = 0; i < PF_BN; ++i) {
-                        const float e = ex2_approx(s[i] * P.k_exp);
-                        const float rc = rcp_approx(1.0f + e);
-                        s[i] = fmaf(-2.0f * P.cap_l2, rc, P.cap_l2);
+                    for (int k = 0; k < 8; ++k) am[k] = fabsf(s[k]);
+#pragma unroll
+                    for (int i = 8; i < HC; ++i) am[i & 7] = fmaxf(am[i & 7], fabsf(s[i]));
+                    const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
+                                             fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
+                    if (__all_sync(0xffffffffu, amax <= P.poly_acc_max)) {
+                        // |x/C| <= 1/4 over the warp's columns: tanh by its Taylor
+                        // series through u^9 on the FMA pipe (truncation < 2.2e-9 |u|).
+                        const float2 a1 = make_float2(P.u_scale, P.u_scale);
+                        const float2 a2 = make_float2(P.scale_l2, P.scale_l2);
+                        const float2 c4 = make_float2(kTanhC4, kTanhC4);
+                        const float2 c3 = make_float2(kTanhC3, kTanhC3);
+                        const float2 c2 = make_float2(kTanhC2, kTanhC2);
+                        const float2 c1 = make_float2(kTanhC1, kTanhC1);
+                        const float2 one = make_float2(1.0f, 1.0f);
+#pragma unroll
+                        for (int i = 0; i < HC; i += 2) {
+                            const float2 a = make_float2(s[i], s[i + 1]);
+                            const float2 uu = mul2(a, a1);
+                            const float2 u2 = mul2(uu, uu);
+                            float2 q = fma2(u2, c4, c3);
+                            q = fma2(u2, q, c2);
+                            q = fma2(u2, q, c1);
+                            q = fma2(u2, q, one);
+                            const float2 rr2 = mul2(mul2(a, a2), q);
+                            s[i] = rr2.x;
+                            s[i + 1] = rr2.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < HC; ++i) {
+                            const float e = ex2_approx(s[i] * P.k_exp);
+                            const float rc = rcp_approx(1.0f + e);
+                            s[i] = fmaf(-2.0f * P.cap_l2, rc, P.cap_l2);
+                        }
                     }
                 } else {
+                    const float2 a2 = make_float2(P.scale_l2, P.scale_l2);
 #pragma unroll
-                    for (int i = 0; i < PF_BN; ++i) s[i] *= P.scale_l2;
+                    for (int i = 0; i < HC; i += 2) {
+                        const float2 rr2 = mul2(make_float2(s[i], s[i + 1]), a2);
+                        s[i] = rr2.x;
+                        s[i + 1] = rr2.y;
+                    }
                 }
                 const int j0 = (U.kt0 + jj) * PF_BN;  // key position of column 0
                 const bool boundary =
                     (j0 + PF_BN - 1 > U.p_min) || (P.window > 0 && j0 < U.p_max - P.window + 1);
                 if (boundary) {
-                    const int hi = p - j0;  // visible columns: [lo, hi]
-                    const int lo = P.window > 0 ? p - P.window + 1 - j0 : -1;
+                    const int hi = p - j0 - col0;  // visible local columns: [lo, hi]
+                    const int lo = P.window > 0 ? p - P.window + 1 - j0 - col0 : -1;
 #pragma unroll
-                    for (int i = 0; i < PF_BN; ++i)
+                    for (int i = 0; i < HC; ++i)
                         if (i > hi || i < lo) s[i] = -INFINITY;
                 }
-                float mt = s[0];
+                float mx[8];
 #pragma unroll
-                for (int i = 1; i < PF_BN; ++i) mt = fmaxf(mt, s[i]);
+                for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+                for (int i = 8; i < HC; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
+                float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                // row max over both halves
+                xmax[(buf * 2 + half) * 128 + r] = mt;
+                mbar_arrive(&xbar[qd * 2 + buf]);  // release: the partner sees xmax
+                ok = mbar_wait(&xbar[qd * 2 + buf], (gt >> 1) & 1, abort_flag, lim,
+                               SITE_SM_PAIR);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                mt = fmaxf(mt, xmax[(buf * 2 + (half ^ 1)) * 128 + r]);
                 const float m_new = fmaxf(m_ref, mt);
                 const bool need = (m_ref != -INFINITY) && (m_new > m_ref + PF_RESCALE_LOG2);
                 if (__any_sync(0xffffffffu, need)) {
-                    // O holds PV(0..gt-1) relative to m_ref: scale it to m_new.
+                    // O holds PV(0..gt-1) relative to m_ref: scale this half to m_new.
                     ok = mbar_wait(&o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, abort_flag, lim,
                                    SITE_SM_O_DONE);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
                     const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
-                    const uint32_t o_addr = tmem + lane_addr;
+                    const uint32_t o_addr = tmem + lane_addr + half * (D / 2);
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = 0; c < D / 64; ++c) {
                         uint32_t v[32];
                         tmem_ld32(o_addr + c * 32, v);
 #pragma unroll
@@ -493,57 +578,69 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // The PV product sees bf16(p); normalising O by the sum of the
                 // same rounded weights makes them sum to one exactly, so their
                 // rounding errors cancel against the row's mean value.
-                float lsum = 0.f, lrsum = 0.f;
+                const float2 mneg = make_float2(-m_use, -m_use);
+                float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < PF_BN / 64; ++c) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float a = ex2_approx(s[c * 64 + 2 * i] - m_use);
-                        const float b = ex2_approx(s[c * 64 + 2 * i + 1] - m_use);
-                        lsum += a + b;
-                        pk[i] = pack_bf16x2(a, b);
-                        lrsum += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u);
-                    }
-                    tmem_st32(s_addr + c * 32, pk);
+                for (int i = 0; i < 32; ++i) {
+                    const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
+                    const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    ls[i & 1] = add2(ls[i & 1], e);
+                    pk[i] = pack_bf16x2(e.x, e.y);
+                    lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
+                                                              __uint_as_float(pk[i] & 0xFFFF0000u)));
                 }
-                l += lsum;
-                lr += lrsum;
+                tmem_st32(s_addr + half * (HC / 2), pk);  // bf16 pairs: HC/2 columns
+                const float2 lsum = add2(ls[0], ls[1]);
+                const float2 lrsum = add2(lrs[0], lrs[1]);
+                l += lsum.x + lsum.y;
+                lr += lrsum.x + lrsum.y;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[buf]);
             }
             if (!ok) break;
-            // ---- epilogue: O / l -> bf16, lse
+            // ---- epilogue: O / lr -> bf16, lse
             // PV(gl) completing implies every earlier UMMA of this CTA completed.
             const uint32_t gl = tile + U.nkt - 1;
             ok = mbar_wait(&o_done[gl & 1], (gl >> 1) & 1, abort_flag, lim, SITE_SM_O_DONE);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
+            // combine the two halves' sums
+            xsum[(half * 128 + r) * 2 + 0] = l;
+            xsum[(half * 128 + r) * 2 + 1] = lr;
+            mbar_arrive(&sbar[qd]);
+            ok = mbar_wait(&sbar[qd], unit_it & 1, abort_flag, lim, SITE_SM_PAIR);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            l += xsum[((half ^ 1) * 128 + r) * 2 + 0];
+            lr += xsum[((half ^ 1) * 128 + r) * 2 + 1];
             const bool valid = pr < U.tvalid;
             const int h = 2 * U.g + hl;
             const float inv_l = 1.0f / lr;
             const size_t orow = static_cast<size_t>(U.qbase + U.t0 + pr) * P.H + h;
-            __nv_bfloat16* optr = P.out + orow * D;
-            const uint32_t o_addr = tmem + lane_addr;
+            __nv_bfloat16* optr = P.out + orow * D + half * (D / 2);
+            const uint32_t o_addr = tmem + lane_addr + half * (D / 2);
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t v[32];
                 tmem_ld32(o_addr + c * 32, v);
-                uint32_t pk[16];
+                uint32_t pkk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
-                                        __uint_as_float(v[2 * i + 1]) * inv_l);
+                    pkk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
+                                         __uint_as_float(v[2 * i + 1]) * inv_l);
                 if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                        dst[i] = make_uint4(pkk[4 * i], pkk[4 * i + 1], pkk[4 * i + 2],
+                                            pkk[4 * i + 3]);
                 }
             }
-            if (valid && P.lse != nullptr) {
+            if (valid && half == 0 && P.lse != nullptr) {
                 const float lse = (m_ref + log2f(l)) * 0.69314718055994531f;
                 size_t li;
                 if (P.varlen)
@@ -561,7 +658,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == PF_WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, PF_TMEM_COLS);
     }
