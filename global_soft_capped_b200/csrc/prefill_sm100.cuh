@@ -6,16 +6,16 @@
 // window on local layers, softmax over keys, grouped mix of the values);
 // cap formula from the "Gemma 2 Guide", section 1.
 //
-// Design (one persistent CTA per SM, 320 threads, warp-specialised):
-//   warps 0..7  softmax + epilogue: warps w and w+4 share MMA rows 32*(w%4)..+31
-//               (TMEM lanes of their sub-partition); warp w<4 takes key columns
-//               0..63 of every S tile and O columns 0..D/2-1, warp w+4 the rest.
-//               The pair exchanges its partial row maxima through shared memory
-//               once per tile (64-thread named barrier), so both halves use the
-//               same running max.
-//   warp 8      TMA producer: Q tile once per work unit, then K/V tiles into a
+// Design (one persistent CTA per SM, 576 threads, warp-specialised):
+//   warps 0..15 softmax + epilogue: warps w, w+4, w+8, w+12 share MMA rows
+//               32*(w%4)..+31 (the TMEM lanes of their sub-partition); part
+//               w/4 takes key columns 32*part..+31 of every S tile and O columns
+//               part*D/4..+D/4-1. The four parts exchange their partial row
+//               maxima through shared memory once per tile (a bounded mbarrier
+//               wait), so all parts use the same running max.
+//   warp 16     TMA producer: Q tile once per work unit, then K/V tiles into a
 //               ring of shared-memory slots (128-byte swizzle).
-//   warp 9      UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
+//   warp 17     UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
 //               O += P V with P read from TMEM; owns the TMEM allocation.
 // A work unit is (sequence, KV head g, 64 query positions); its 128 MMA rows
 // are the two query heads 2g, 2g+1 that share KV head g (row = head_local*64 +
@@ -23,7 +23,7 @@
 // the causal band (and the window on local layers) are visited, and only
 // tiles that cross a band edge evaluate the mask.
 // Softmax: fp32, log2 domain. s2 = C*log2(e)*tanh(x/C): when |x/C| <= 1/4 over
-// a warp's tile, by the Taylor series of tanh on the FMA pipe (packed f32x2);
+// a warp's tile, by the Taylor series of tanh through x^7 on the FMA pipe;
 // otherwise as C*log2(e)*(1 - 2/(1 + 2^(2*x*log2(e)/C))) with ex2/rcp. Then a running max
 // per row with lazy rescaling of O (only when the max grows by more than
 // 2^8), p = 2^(s2 - m) rounded to bf16 for the PV product, row sum in fp32.
@@ -34,22 +34,23 @@
 
 namespace g2 {
 
-constexpr int PF_THREADS = 320;  // 8 softmax warps, producer, UMMA issuer
-constexpr int PF_WARP_PRODUCER = 8;
-constexpr int PF_WARP_MMA = 9;
-constexpr int PF_SOFTMAX_THREADS = 256;
+constexpr int PF_NSPLIT = 4;     // softmax warps per TMEM lane quadrant
+constexpr int PF_SOFTMAX_THREADS = 128 * PF_NSPLIT;
+constexpr int PF_WARP_PRODUCER = 4 * PF_NSPLIT;
+constexpr int PF_WARP_MMA = PF_WARP_PRODUCER + 1;
+constexpr int PF_THREADS = PF_SOFTMAX_THREADS + 64;  // + producer warp + UMMA warp
 constexpr int PF_BM = 128;   // MMA rows per tile (64 positions x 2 heads)
 constexpr int PF_QPOS = 64;  // query positions per tile
 constexpr int PF_BN = 128;   // keys per KV tile
 constexpr int PF_TMEM_COLS = 512;
 constexpr int PF_S_COL0 = 256;  // S buffers at TMEM columns 256 and 384; O at 0
 constexpr float PF_RESCALE_LOG2 = 8.0f;
-// Taylor coefficients of tanh(u) = u (1 + c1 u^2 + c2 u^4 + c3 u^6 + c4 u^8 + ...):
-// -1/3, 2/15, -17/315, 62/2835 (the series of tanh, from its Bernoulli-number form).
+// Taylor coefficients of tanh(u) = u (1 + c1 u^2 + c2 u^4 + c3 u^6 + ...):
+// -1/3, 2/15, -17/315 (the series of tanh, from its Bernoulli-number form; the
+// next coefficient, 62/2835, bounds the truncation for |u| <= 1/4).
 constexpr float kTanhC1 = -1.0f / 3.0f;
 constexpr float kTanhC2 = 2.0f / 15.0f;
 constexpr float kTanhC3 = -17.0f / 315.0f;
-constexpr float kTanhC4 = 62.0f / 2835.0f;
 constexpr float PF_POLY_U_MAX = 0.25f;  // |x / C| bound of the series path
 
 template <int D>
@@ -63,7 +64,7 @@ struct PfCfg {
     static constexpr int Q_BYTES = PF_BM * D * 2;
     static constexpr int MAX_SEQ_TABLE = 1024;  // varlen: per-sequence unit prefix table
     static constexpr int SMEM_TILES = Q_BYTES + NSLOT * SLOT_BYTES;
-    static constexpr int CTRL_BYTES = 1024 + 2 * 2 * 128 * 4 + 128 * 2 * 2 * 4;
+    static constexpr int CTRL_BYTES = 1024 + 2 * PF_NSPLIT * 128 * 4 + PF_NSPLIT * 128 * 2 * 4;
     static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + CTRL_BYTES + 4 * (MAX_SEQ_TABLE + 1);
     static_assert(KCOLS % 64 == 0 && VROWS % 16 == 0, "tile shapes");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -185,10 +186,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint64_t* sbar = xbar + 8;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sbar + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    // partial row maxima of the two column halves, by tile parity: [2][2][128]
+    // partial row maxima of the column parts, by tile parity: [2][NSPLIT][128]
     float* xmax = reinterpret_cast<float*>(base + C::SMEM_TILES + 1024);
-    // partial (l, lr) row sums of the two halves at the end of a unit: [2][128][2]
-    float* xsum = xmax + 2 * 2 * 128;
+    // partial (l, lr) row sums of the parts at the end of a unit: [NSPLIT][128][2]
+    float* xsum = xmax + 2 * PF_NSPLIT * 128;
     int* pre = reinterpret_cast<int*>(base + C::SMEM_TILES + C::CTRL_BYTES);
 
     const int warp = threadIdx.x >> 5;
@@ -199,12 +200,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         mbar_init(q_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], PF_SOFTMAX_THREADS);
+            mbar_init(&p_full[i], PF_SOFTMAX_THREADS / 32);
             mbar_init(&o_done[i], 1);
         }
-        mbar_init(o_free, PF_SOFTMAX_THREADS);
-        for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
-        for (int i = 0; i < 4; ++i) mbar_init(&sbar[i], 64);
+        // softmax-side barriers take one arrival per warp (elected lane, after
+        // __syncwarp orders the whole warp's prior writes before it)
+        mbar_init(o_free, PF_SOFTMAX_THREADS / 32);
+        for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], PF_NSPLIT);
+        for (int i = 0; i < 4; ++i) mbar_init(&sbar[i], PF_NSPLIT);
         mbar_init(drain, 1);
         for (int i = 0; i < C::NSLOT; ++i) {
             mbar_init(&slot_full[i], 1);
@@ -333,10 +336,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(PF_BM, PF_BN, false);
             constexpr uint32_t IDESC_O = idesc_bf16(PF_BM, D, true);
-            const uint32_t sQ_addr = smem_u32(sQ);
-            const uint32_t slots_addr = smem_u32(sSlots);
-            uint32_t fill = 0;
-            uint32_t tile = 0;  // KV tiles processed by this CTA (S/P/PV index)
+            constexpr uint32_t HI = sdesc_hi(1024);  // SBO 1024 B (8 rows x 128 B)
+            // Q (A of S = Q K^T): K-major, 64-column chunks of 16 KB, k-step = 32 B
+            const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
+            // ring slot s: K-major K (LBO unused) or MN-major V (LBO = VROWS*128 B)
+            const uint32_t slot_lo0 = sdesc_lo(smem_u32(sSlots), 16);
+            const uint32_t slot_lo0_v = sdesc_lo(smem_u32(sSlots), C::VROWS * 128);
+            constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
+            int slot = 0;          // ring position and phase (fills consumed so far)
+            uint32_t phase = 0;
+            uint32_t tile = 0;     // KV tiles processed by this CTA (S/P/PV index)
             int unit_it = 0;
             bool ok = true;
 
@@ -345,28 +354,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // S(gt) overwrites P(gt-2) in the same TMEM columns. PV(gt-2) was
                 // issued earlier by this thread, and UMMAs issued by one thread
                 // execute in issue order, so no completion wait is needed here.
-                tc_fence_after();
                 const uint32_t d_tmem = tmem + PF_S_COL0 + buf * PF_BN;
 #pragma unroll
                 for (int s = 0; s < C::KSL; ++s) {
-                    const int slot = fill % C::NSLOT;
-                    if (!mbar_wait(&slot_full[slot], (fill / C::NSLOT) & 1, abort_flag, lim,
-                                   SITE_MMA_SLOT_FULL))
+                    if (!mbar_wait(&slot_full[slot], phase, abort_flag, lim, SITE_MMA_SLOT_FULL))
                         return false;
                     tc_fence_after();
-                    const uint32_t kb = slots_addr + slot * C::SLOT_BYTES;
+                    const uint32_t k_lo = slot_lo0 + slot * SLOT_STEP;
 #pragma unroll
                     for (int kk = 0; kk < C::KCOLS / 16; ++kk) {
                         const int dcol = s * C::KCOLS + kk * 16;  // Q column of this k-step
-                        const uint64_t a = sdesc_sw128(
-                            sQ_addr + (dcol / 64) * 16384 + ((dcol % 64) / 16) * 32, 16, 1024);
-                        const uint64_t b = sdesc_sw128(
-                            kb + ((kk * 16) / 64) * (PF_BN * 128) + (((kk * 16) % 64) / 16) * 32,
-                            16, 1024);
-                        umma_ss(d_tmem, a, b, IDESC_S, (s | kk) != 0);
+                        const uint32_t a_lo = q_lo + (dcol / 64) * (16384 >> 4) + ((dcol % 64) / 16) * 2;
+                        const uint32_t b_lo = k_lo + (kk / 4) * ((PF_BN * 128) >> 4) + (kk % 4) * 2;
+                        umma_ss_lh(d_tmem, a_lo, b_lo, HI, IDESC_S, (s | kk) != 0);
                     }
                     umma_commit(&slot_empty[slot]);
-                    ++fill;
+                    if (++slot == C::NSLOT) { slot = 0; phase ^= 1u; }
                 }
                 umma_commit(&s_full[buf]);
                 return true;
@@ -376,20 +379,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint32_t p_tmem = tmem + PF_S_COL0 + buf * PF_BN;
 #pragma unroll
                 for (int s = 0; s < C::VSL; ++s) {
-                    const int slot = fill % C::NSLOT;
-                    if (!mbar_wait(&slot_full[slot], (fill / C::NSLOT) & 1, abort_flag, lim,
-                                   SITE_MMA_SLOT_FULL))
+                    if (!mbar_wait(&slot_full[slot], phase, abort_flag, lim, SITE_MMA_SLOT_FULL))
                         return false;
                     tc_fence_after();
-                    const uint32_t vb = slots_addr + slot * C::SLOT_BYTES;
+                    const uint32_t v_lo = slot_lo0_v + slot * SLOT_STEP;
 #pragma unroll
                     for (int kk = 0; kk < C::VROWS / 16; ++kk) {
-                        const uint64_t b = sdesc_sw128(vb + kk * 16 * 128, C::VROWS * 128, 1024);
                         const uint32_t a = p_tmem + (s * C::VROWS + kk * 16) / 2;
-                        umma_ts(tmem, a, b, IDESC_O, (first && s == 0 && kk == 0) ? 0u : 1u);
+                        umma_ts_lh(tmem, a, v_lo + kk * ((16 * 128) >> 4), HI, IDESC_O,
+                                   (first && s == 0 && kk == 0) ? 0u : 1u);
                     }
                     umma_commit(&slot_empty[slot]);
-                    ++fill;
+                    if (++slot == C::NSLOT) { slot = 0; phase ^= 1u; }
                 }
                 umma_commit(&o_done[buf]);
                 return true;
@@ -402,6 +403,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 pf_unit(P, pre, u, U);
                 ok = mbar_wait(q_full, unit_it & 1, abort_flag, lim, SITE_MMA_Q_FULL);
                 if (!ok) break;
+                tc_fence_after();
                 ok = issue_s(tile);
                 for (int jj = 0; ok && jj < U.nkt; ++jj) {
                     const uint32_t gt = tile + jj;
@@ -432,14 +434,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        constexpr int HC = PF_BN / 2;                   // key columns per half
+        constexpr int HC = PF_BN / PF_NSPLIT;           // key columns per part (32)
+        constexpr int OC = D / PF_NSPLIT;               // O columns per part
         const int qd = warp & 3;                        // TMEM lane quadrant
-        const int half = warp >> 2;                     // column half of this warp
+        const int part = warp >> 2;                     // column part of this warp
         const int r = (qd << 5) | lane;                 // MMA row == TMEM lane
         const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
         const int hl = r >> 6;                          // head within the pair
         const int pr = r & 63;                          // position within the tile
-        const int col0 = half * HC;                     // first S column of this warp
+        const int col0 = part * HC;                     // first S column of this warp
+        // s2 = x * (b0 + b1 u^2 + b2 u^4 + b3 u^6) with u = x*alpha/C and
+        // b_k = alpha*log2(e)*c_k: the tanh series through u^7 (|u| <= 1/4:
+        // truncation below 3.3e-7 relative), scaled into log2 units.
+        const float b0 = P.scale_l2, b1 = P.scale_l2 * kTanhC1, b2 = P.scale_l2 * kTanhC2,
+                    b3 = P.scale_l2 * kTanhC3;
+        auto series_s2 = [&](float x) {
+            const float uu = x * P.u_scale, u2 = uu * uu;
+            float q = fmaf(u2, b3, b2);
+            q = fmaf(u2, q, b1);
+            q = fmaf(u2, q, b0);
+            return x * q;
+        };
         uint32_t tile = 0;
         int unit_it = 0;
         bool ok = true;
@@ -450,8 +465,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             pf_unit(P, pre, u, U);
             const int p = U.p_min + pr;  // absolute query position of this row
             float m_ref = -INFINITY;     // log2-domain reference max of the row
-            float l = 0.f;               // this half's sum of fp32 weights (for lse)
-            float lr = 0.f;              // this half's sum of bf16-rounded weights
+            float l = 0.f;               // this part's sum of fp32 weights (for lse)
+            float lr = 0.f;              // this part's sum of bf16-rounded weights
             for (int jj = 0; jj < U.nkt; ++jj) {
                 const uint32_t gt = tile + jj;
                 const uint32_t buf = gt & 1;
@@ -461,112 +476,101 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_addr + PF_S_COL0 + buf * PF_BN;
                 float s[HC];
-                {  // two TMEM loads in flight, one wait
-                    uint32_t v0[32], v1[32];
+                {
+                    uint32_t v0[32];
                     tmem_ld32_async(s_addr + col0, v0);
-                    tmem_ld32_async(s_addr + col0 + 32, v1);
                     tmem_wait_ld();
                     tmem_reg_fence(v0);
-                    tmem_reg_fence(v1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        s[i] = __uint_as_float(v0[i]);
-                        s[32 + i] = __uint_as_float(v1[i]);
-                    }
-                }
-                // capped logit in log2 units
-                if (P.has_cap) {
-                    float am[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) am[k] = fabsf(s[k]);
-#pragma unroll
-                    for (int i = 8; i < HC; ++i) am[i & 7] = fmaxf(am[i & 7], fabsf(s[i]));
-                    const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
-                                             fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
-                    if (__all_sync(0xffffffffu, amax <= P.poly_acc_max)) {
-                        // |x/C| <= 1/4 over the warp's columns: tanh by its Taylor
-                        // series through u^9 on the FMA pipe (truncation < 2.2e-9 |u|).
-                        const float2 a1 = make_float2(P.u_scale, P.u_scale);
-                        const float2 a2 = make_float2(P.scale_l2, P.scale_l2);
-                        const float2 c4 = make_float2(kTanhC4, kTanhC4);
-                        const float2 c3 = make_float2(kTanhC3, kTanhC3);
-                        const float2 c2 = make_float2(kTanhC2, kTanhC2);
-                        const float2 c1 = make_float2(kTanhC1, kTanhC1);
-                        const float2 one = make_float2(1.0f, 1.0f);
-#pragma unroll
-                        for (int i = 0; i < HC; i += 2) {
-                            const float2 a = make_float2(s[i], s[i + 1]);
-                            const float2 uu = mul2(a, a1);
-                            const float2 u2 = mul2(uu, uu);
-                            float2 q = fma2(u2, c4, c3);
-                            q = fma2(u2, q, c2);
-                            q = fma2(u2, q, c1);
-                            q = fma2(u2, q, one);
-                            const float2 rr2 = mul2(mul2(a, a2), q);
-                            s[i] = rr2.x;
-                            s[i + 1] = rr2.y;
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < HC; ++i) {
-                            const float e = ex2_approx(s[i] * P.k_exp);
-                            const float rc = rcp_approx(1.0f + e);
-                            s[i] = fmaf(-2.0f * P.cap_l2, rc, P.cap_l2);
-                        }
-                    }
-                } else {
-                    const float2 a2 = make_float2(P.scale_l2, P.scale_l2);
-#pragma unroll
-                    for (int i = 0; i < HC; i += 2) {
-                        const float2 rr2 = mul2(make_float2(s[i], s[i + 1]), a2);
-                        s[i] = rr2.x;
-                        s[i + 1] = rr2.y;
-                    }
+                    for (int i = 0; i < HC; ++i) s[i] = __uint_as_float(v0[i]);
                 }
                 const int j0 = (U.kt0 + jj) * PF_BN;  // key position of column 0
                 const bool boundary =
                     (j0 + PF_BN - 1 > U.p_min) || (P.window > 0 && j0 < U.p_max - P.window + 1);
-                if (boundary) {
-                    const int hi = p - j0 - col0;  // visible local columns: [lo, hi]
-                    const int lo = P.window > 0 ? p - P.window + 1 - j0 - col0 : -1;
+                // raw accumulator range of this warp's columns
+                float mxa[4], mna[4];
 #pragma unroll
-                    for (int i = 0; i < HC; ++i)
-                        if (i > hi || i < lo) s[i] = -INFINITY;
+                for (int k = 0; k < 4; ++k) mxa[k] = mna[k] = s[k];
+#pragma unroll
+                for (int i = 4; i < HC; ++i) {
+                    mxa[i & 3] = fmaxf(mxa[i & 3], s[i]);
+                    mna[i & 3] = fminf(mna[i & 3], s[i]);
                 }
-                float mx[8];
+                const float amx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+                const float amn = fminf(fminf(mna[0], mna[1]), fminf(mna[2], mna[3]));
+                // Fast path: no mask in this tile, cap on, |x/C| <= 1/4 for the
+                // whole warp. The capped map is monotonic in x, so the tile max
+                // is the map of the extreme accumulators and s2 - m fuses into
+                // one packed FMA below.
+                const bool fast = __all_sync(
+                    0xffffffffu, P.has_cap && !boundary &&
+                                     fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max);
+                float mt;
+                if (fast) {
+                    mt = fmaxf(series_s2(amx), series_s2(amn));
+                } else {
+                    // general path: capped logits in log2 units, then the mask
+                    if (P.has_cap) {
+                        if (__all_sync(0xffffffffu,
+                                       fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max)) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = s[k];
+                            for (int i = 0; i < HC; ++i) s[i] = series_s2(s[i]);
+                        } else {
 #pragma unroll
-                for (int i = 8; i < HC; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-                float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                // row max over both halves
-                xmax[(buf * 2 + half) * 128 + r] = mt;
-                mbar_arrive(&xbar[qd * 2 + buf]);  // release: the partner sees xmax
+                            for (int i = 0; i < HC; ++i) {
+                                const float e = ex2_approx(s[i] * P.k_exp);
+                                const float rc = rcp_approx(1.0f + e);
+                                s[i] = fmaf(-2.0f * P.cap_l2, rc, P.cap_l2);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < HC; ++i) s[i] *= P.scale_l2;
+                    }
+                    if (boundary) {
+                        const int hi = p - j0 - col0;  // visible local columns: [lo, hi]
+                        const int lo = P.window > 0 ? p - P.window + 1 - j0 - col0 : -1;
+#pragma unroll
+                        for (int i = 0; i < HC; ++i)
+                            if (i > hi || i < lo) s[i] = -INFINITY;
+                    }
+                    float mx[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mx[k] = s[k];
+#pragma unroll
+                    for (int i = 4; i < HC; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+                    mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                }
+                // row max over all parts
+                xmax[(buf * PF_NSPLIT + part) * 128 + r] = mt;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xbar[qd * 2 + buf]);  // release for the warp
                 ok = mbar_wait(&xbar[qd * 2 + buf], (gt >> 1) & 1, abort_flag, lim,
                                SITE_SM_PAIR);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                mt = fmaxf(mt, xmax[(buf * 2 + (half ^ 1)) * 128 + r]);
+#pragma unroll
+                for (int k = 0; k < PF_NSPLIT; ++k)
+                    mt = fmaxf(mt, xmax[(buf * PF_NSPLIT + k) * 128 + r]);
                 const float m_new = fmaxf(m_ref, mt);
                 const bool need = (m_ref != -INFINITY) && (m_new > m_ref + PF_RESCALE_LOG2);
                 if (__any_sync(0xffffffffu, need)) {
-                    // O holds PV(0..gt-1) relative to m_ref: scale this half to m_new.
+                    // O holds PV(0..gt-1) relative to m_ref: scale this part to m_new.
                     ok = mbar_wait(&o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, abort_flag, lim,
                                    SITE_SM_O_DONE);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
                     const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
-                    const uint32_t o_addr = tmem + lane_addr + half * (D / 2);
+                    const uint32_t o_addr = tmem + lane_addr + part * OC;
 #pragma unroll 1
-                    for (int c = 0; c < D / 64; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(o_addr + c * 32, v);
+                    for (int c = 0; c < OC / 16; ++c) {
+                        uint32_t v[16];
+                        tmem_ld16(o_addr + c * 16, v);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
+                        for (int i = 0; i < 16; ++i)
                             v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-                        tmem_st32(o_addr + c * 32, v);
+                        tmem_st16(o_addr + c * 16, v);
                     }
                     tmem_wait_st();
                     l *= f;
@@ -581,24 +585,46 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const float2 mneg = make_float2(-m_use, -m_use);
                 float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                uint32_t pk[32];
+                uint32_t pk[HC / 2];
+                if (fast) {
+                    const float2 a1 = make_float2(P.u_scale, P.u_scale);
+                    const float2 B0 = make_float2(b0, b0), B1 = make_float2(b1, b1);
+                    const float2 B2 = make_float2(b2, b2), B3 = make_float2(b3, b3);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
-                    const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                    ls[i & 1] = add2(ls[i & 1], e);
-                    pk[i] = pack_bf16x2(e.x, e.y);
-                    lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
-                                                              __uint_as_float(pk[i] & 0xFFFF0000u)));
+                    for (int i = 0; i < HC / 2; ++i) {
+                        const float2 a = make_float2(s[2 * i], s[2 * i + 1]);
+                        const float2 uu = mul2(a, a1);
+                        const float2 u2 = mul2(uu, uu);
+                        float2 q = fma2(u2, B3, B2);
+                        q = fma2(u2, q, B1);
+                        q = fma2(u2, q, B0);
+                        const float2 x = fma2(a, q, mneg);  // s2 - m
+                        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        ls[i & 1] = add2(ls[i & 1], e);
+                        pk[i] = pack_bf16x2(e.x, e.y);
+                        lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
+                                                                  __uint_as_float(pk[i] & 0xFFFF0000u)));
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < HC / 2; ++i) {
+                        const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
+                        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        ls[i & 1] = add2(ls[i & 1], e);
+                        pk[i] = pack_bf16x2(e.x, e.y);
+                        lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
+                                                                  __uint_as_float(pk[i] & 0xFFFF0000u)));
+                    }
                 }
-                tmem_st32(s_addr + half * (HC / 2), pk);  // bf16 pairs: HC/2 columns
+                tmem_st16(s_addr + part * (HC / 2), pk);  // bf16 pairs: HC/2 columns
                 const float2 lsum = add2(ls[0], ls[1]);
                 const float2 lrsum = add2(lrs[0], lrs[1]);
                 l += lsum.x + lsum.y;
                 lr += lrsum.x + lrsum.y;
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&p_full[buf]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[buf]);
             }
             if (!ok) break;
             // ---- epilogue: O / lr -> bf16, lse
@@ -608,39 +634,43 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            // combine the two halves' sums
-            xsum[(half * 128 + r) * 2 + 0] = l;
-            xsum[(half * 128 + r) * 2 + 1] = lr;
-            mbar_arrive(&sbar[qd]);
+            // combine the parts' sums
+            xsum[(part * 128 + r) * 2 + 0] = l;
+            xsum[(part * 128 + r) * 2 + 1] = lr;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sbar[qd]);
             ok = mbar_wait(&sbar[qd], unit_it & 1, abort_flag, lim, SITE_SM_PAIR);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            l += xsum[((half ^ 1) * 128 + r) * 2 + 0];
-            lr += xsum[((half ^ 1) * 128 + r) * 2 + 1];
+            l = 0.f;
+            lr = 0.f;
+#pragma unroll
+            for (int k = 0; k < PF_NSPLIT; ++k) {
+                l += xsum[(k * 128 + r) * 2 + 0];
+                lr += xsum[(k * 128 + r) * 2 + 1];
+            }
             const bool valid = pr < U.tvalid;
             const int h = 2 * U.g + hl;
             const float inv_l = 1.0f / lr;
             const size_t orow = static_cast<size_t>(U.qbase + U.t0 + pr) * P.H + h;
-            __nv_bfloat16* optr = P.out + orow * D + half * (D / 2);
-            const uint32_t o_addr = tmem + lane_addr + half * (D / 2);
+            __nv_bfloat16* optr = P.out + orow * D + part * OC;
+            const uint32_t o_addr = tmem + lane_addr + part * OC;
 #pragma unroll 1
-            for (int c = 0; c < D / 64; ++c) {
-                uint32_t v[32];
-                tmem_ld32(o_addr + c * 32, v);
-                uint32_t pkk[16];
+            for (int c = 0; c < OC / 16; ++c) {
+                uint32_t v[16];
+                tmem_ld16(o_addr + c * 16, v);
+                uint32_t pkk[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
+                for (int i = 0; i < 8; ++i)
                     pkk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
                                          __uint_as_float(v[2 * i + 1]) * inv_l);
                 if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pkk[4 * i], pkk[4 * i + 1], pkk[4 * i + 2],
-                                            pkk[4 * i + 3]);
+                    uint4* dst = reinterpret_cast<uint4*>(optr + c * 16);
+                    dst[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
+                    dst[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
                 }
             }
-            if (valid && half == 0 && P.lse != nullptr) {
+            if (valid && part == 0 && P.lse != nullptr) {
                 const float lse = (m_ref + log2f(l)) * 0.69314718055994531f;
                 size_t li;
                 if (P.varlen)
@@ -650,7 +680,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 P.lse[li] = lse;
             }
             tc_fence_before();
-            mbar_arrive(o_free);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
             tile += U.nkt;
             ++unit_it;
         }
