@@ -26,12 +26,17 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "g2ref.c")
-_LIB = os.path.join(_HERE, "libg2ref.so")
+_LIB_DEFAULT = os.path.join(_HERE, "libg2ref.so")
+# G2REF_LIB points the oracle at another build of g2ref.c; the mutation tests
+# use it to check that the pins reject deliberately broken copies.
+_LIB = os.environ.get("G2REF_LIB", _LIB_DEFAULT)
 _lib = None
 
 
 def build(force: bool = False) -> str:
     """Compile g2ref.c into libg2ref.so next to it (gcc, OpenMP, -O2)."""
+    if _LIB != _LIB_DEFAULT:
+        return _LIB
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
             os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "g2ref.h"))):
         cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-o",

@@ -1,0 +1,63 @@
+"""The pins reject a broken oracle.
+
+Each case plants one plausible mistake in a copy of oracle/g2ref.c (compiled
+on the CPU into a temporary library), then runs the pin suite against it
+through G2REF_LIB: the suite must fail. The unmodified copy must pass. This
+shows the pins are not tautological: a dropped term, a wrong sign, an
+off-by-one or a wrong index anywhere in the definition is caught.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "g2ref.c")
+
+MUTANTS = {
+    "window keeps W+1 keys": ("p - j >= window", "p - j > window"),
+    "causal mask drops the query's own key": ("if (j > p) return 0;", "if (j >= p) return 0;"),
+    "cap without its outer multiply": ("x = softcap * tanh(x / softcap);", "x = tanh(x / softcap);"),
+    "cap of the raw logit without the inner divide": ("softcap * tanh(x / softcap)", "softcap * tanh(x)"),
+    "softmax exponent with the wrong sign": ("exp(s[j] - m)", "exp(m - s[j])"),
+    "query scale dropped": ("qs[c] = query_scale * widen(qrow[c]);", "qs[c] = widen(qrow[c]);"),
+    "wrong GQA head mapping": ("const int64_t g = h / group;", "const int64_t g = h % Hkv;"),
+    "lse without the max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "values mixed from the mirrored key": ("const uint16_t* vrow = v + ((b * S + j) * Hkv + g) * d;",
+                                           "const uint16_t* vrow = v + ((b * S + (S - 1 - j)) * Hkv + g) * d;"),
+    "mask before cap (a masked key gets -cap, not -inf)": (
+        "s[j] = visible(p, j, window) ? sj : -INFINITY;",
+        "s[j] = visible(p, j, window) ? sj : (softcap > 0.0 ? -softcap : -INFINITY);"),
+}
+
+
+def _build(tmp_path, name, old=None, new=None):
+    src = open(SRC).read()
+    if old is not None:
+        assert src.count(old) == 1, old
+        src = src.replace(old, new)
+    c = tmp_path / f"{name}.c"
+    c.write_text(src)
+    lib = tmp_path / f"{name}.so"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-I",
+                    os.path.join(ROOT, "oracle"), "-o", str(lib), str(c), "-lm"], check=True)
+    return str(lib)
+
+
+def _pins_pass(lib):
+    env = dict(os.environ, G2REF_LIB=lib, OMP_NUM_THREADS="4")
+    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return res.returncode == 0
+
+
+def test_unmodified_copy_passes_the_pins(tmp_path):
+    assert _pins_pass(_build(tmp_path, "control"))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_the_pins(tmp_path, name):
+    old, new = MUTANTS[name]
+    assert not _pins_pass(_build(tmp_path, "mutant", old, new)), name
