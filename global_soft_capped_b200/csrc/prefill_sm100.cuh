@@ -6,16 +6,16 @@
 // window on local layers, softmax over keys, grouped mix of the values);
 // cap formula from the "Gemma 2 Guide", section 1.
 //
-// Design (one persistent CTA per SM, 576 threads, warp-specialised):
-//   warps 0..15 softmax + epilogue: warps w, w+4, w+8, w+12 share MMA rows
-//               32*(w%4)..+31 (the TMEM lanes of their sub-partition); part
-//               w/4 takes key columns 32*part..+31 of every S tile and O columns
-//               part*D/4..+D/4-1. The four parts exchange their partial row
-//               maxima through shared memory once per tile (a bounded mbarrier
-//               wait), so all parts use the same running max.
-//   warp 16     TMA producer: Q tile once per work unit, then K/V tiles into a
+// Design (one persistent CTA per SM, 320 threads, warp-specialised):
+//   warps 0..7  softmax + epilogue: warps w and w+4 share MMA rows 32*(w%4)..+31
+//               (the TMEM lanes of their sub-partition); part w/4 takes key
+//               columns 64*part..+63 of every S tile and O columns
+//               part*D/2..+D/2-1. The parts exchange their partial row maxima
+//               through shared memory once per tile (a bounded mbarrier wait),
+//               so both use the same running max.
+//   warp 8      TMA producer: Q tile once per work unit, then K/V tiles into a
 //               ring of shared-memory slots (128-byte swizzle).
-//   warp 17     UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
+//   warp 9      UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
 //               O += P V with P read from TMEM; owns the TMEM allocation.
 // A work unit is (sequence, KV head g, 64 query positions); its 128 MMA rows
 // are the two query heads 2g, 2g+1 that share KV head g (row = head_local*64 +
@@ -34,7 +34,7 @@
 
 namespace g2 {
 
-constexpr int PF_NSPLIT = 4;     // softmax warps per TMEM lane quadrant
+constexpr int PF_NSPLIT = 2;     // softmax warps per TMEM lane quadrant
 constexpr int PF_SOFTMAX_THREADS = 128 * PF_NSPLIT;
 constexpr int PF_WARP_PRODUCER = 4 * PF_NSPLIT;
 constexpr int PF_WARP_MMA = PF_WARP_PRODUCER + 1;
@@ -434,7 +434,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        constexpr int HC = PF_BN / PF_NSPLIT;           // key columns per part (32)
+        constexpr int HC = PF_BN / PF_NSPLIT;           // key columns per part
+        static_assert(HC % 32 == 0 && (D / PF_NSPLIT) % 16 == 0, "softmax split");
         constexpr int OC = D / PF_NSPLIT;               // O columns per part
         const int qd = warp & 3;                        // TMEM lane quadrant
         const int part = warp >> 2;                     // column part of this warp
@@ -476,13 +477,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_addr + PF_S_COL0 + buf * PF_BN;
                 float s[HC];
-                {
-                    uint32_t v0[32];
-                    tmem_ld32_async(s_addr + col0, v0);
-                    tmem_wait_ld();
-                    tmem_reg_fence(v0);
+                {  // HC/32 TMEM loads in flight, one wait
+                    uint32_t v[HC / 32][32];
 #pragma unroll
-                    for (int i = 0; i < HC; ++i) s[i] = __uint_as_float(v0[i]);
+                    for (int c = 0; c < HC / 32; ++c) tmem_ld32_async(s_addr + col0 + 32 * c, v[c]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < HC / 32; ++c) tmem_reg_fence(v[c]);
+#pragma unroll
+                    for (int i = 0; i < HC; ++i) s[i] = __uint_as_float(v[i / 32][i % 32]);
                 }
                 const int j0 = (U.kt0 + jj) * PF_BN;  // key position of column 0
                 const bool boundary =
@@ -616,7 +619,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                                                                   __uint_as_float(pk[i] & 0xFFFF0000u)));
                     }
                 }
-                tmem_st16(s_addr + part * (HC / 2), pk);  // bf16 pairs: HC/2 columns
+#pragma unroll
+                for (int c = 0; c < HC / 32; ++c) {  // bf16 pairs: HC/2 columns
+                    uint32_t pc[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pc[i] = pk[16 * c + i];
+                    tmem_st16(s_addr + part * (HC / 2) + 16 * c, pc);
+                }
                 const float2 lsum = add2(ls[0], ls[1]);
                 const float2 lrsum = add2(lrs[0], lrs[1]);
                 l += lsum.x + lsum.y;
