@@ -62,10 +62,11 @@ struct PfCfg {
     static constexpr int VSL = PF_BN / VROWS;               // V slots per KV tile
     static constexpr int NSLOT = (D == 64) ? 8 : (D == 128 ? 5 : 4);
     static constexpr int Q_BYTES = PF_BM * D * 2;
-    static constexpr int MAX_SEQ_TABLE = 1024;  // varlen: per-sequence unit prefix table
+    static constexpr int MAX_SEQ_TABLE = 1024;  // varlen: sequences per launch
+    static constexpr int VL_BYTES = 4 * (3 * MAX_SEQ_TABLE + 1);
     static constexpr int SMEM_TILES = Q_BYTES + NSLOT * SLOT_BYTES;
     static constexpr int CTRL_BYTES = 1024 + 2 * PF_NSPLIT * 128 * 4 + PF_NSPLIT * 128 * 2 * 4;
-    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + CTRL_BYTES + 4 * (MAX_SEQ_TABLE + 1);
+    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + CTRL_BYTES + VL_BYTES;
     static_assert(KCOLS % 64 == 0 && VROWS % 16 == 0, "tile shapes");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -106,11 +107,31 @@ struct PfUnit {
     int p_min, p_max;
 };
 
+// Per-launch varlen schedule in shared memory: sequences ranked by their work
+// (KV tiles over all their query tiles), heaviest first, so the light units
+// land at the end of the static schedule; within a sequence, query tiles run
+// longest first. Consecutive units stay within one sequence, which keeps that
+// sequence's K/V resident in L2 while all SMs work on it.
+struct VlTables {
+    int* work;   // [num_seqs] KV tiles of the sequence (one KV head)
+    int* order;  // [num_seqs] sequences ranked by work, descending
+    int* cum;    // [num_seqs + 1] units before each ranked sequence; cum[num_seqs] = total
+};
+
+// KV tiles visited by query tile t0 of a sequence (T queries at the end of S keys).
+__device__ __forceinline__ int pf_tiles(int t0, int T, int S, int window) {
+    const int tvalid = min(PF_QPOS, T - t0);
+    const int p_min = t0 + (S - T), p_max = p_min + tvalid - 1;
+    const int j_lo = window > 0 ? max(0, p_min - window + 1) : 0;
+    const int j_hi = min(p_max, S - 1);
+    return j_hi / PF_BN - j_lo / PF_BN + 1;
+}
+
 // Work unit u of the launch. Dense: query tiles in descending order (longest
-// rows first), then batch, then KV head. Varlen: sequences in order, each with
-// its query tiles descending; `pre` holds the unit prefix per sequence.
-__device__ __forceinline__ void pf_unit(const PfParams& P, const int* pre, int u, PfUnit& U) {
-    int seq, lu, Tq, Sk, qbase, kbase;
+// rows first), then batch, then KV head. Varlen: sequences in rank order, each
+// with its query tiles descending, then KV head.
+__device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, int u, PfUnit& U) {
+    int seq, Tq, Sk, qbase, kbase;
     if (!P.varlen) {
         const int BG = P.num_seqs * P.Hkv;
         const int nq = P.max_units_per_seq_tiles;
@@ -125,21 +146,20 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const int* pre, int u
         U.t0 = qt * PF_QPOS;
         U.qoff = P.q_offset;
     } else {
-        int lo = 0, hi = P.num_seqs - 1;  // largest s with pre[s] <= u
+        int lo = 0, hi = P.num_seqs - 1;  // largest rank with cum[rank] <= u
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (pre[mid] <= u) lo = mid; else hi = mid - 1;
+            if (V.cum[mid] <= u) lo = mid; else hi = mid - 1;
         }
-        seq = lo;
-        lu = u - pre[seq];
+        seq = V.order[lo];
+        const int lu = u - V.cum[lo];
         qbase = P.cu_q[seq];
         kbase = P.cu_k[seq];
         Tq = P.cu_q[seq + 1] - qbase;
         Sk = P.cu_k[seq + 1] - kbase;
         const int nq = (Tq + PF_QPOS - 1) / PF_QPOS;
-        const int qt = nq - 1 - lu / P.Hkv;
         U.g = lu % P.Hkv;
-        U.t0 = qt * PF_QPOS;
+        U.t0 = (nq - 1 - lu / P.Hkv) * PF_QPOS;
         U.qoff = Sk - Tq;
     }
     U.seq = seq;
@@ -190,7 +210,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     float* xmax = reinterpret_cast<float*>(base + C::SMEM_TILES + 1024);
     // partial (l, lr) row sums of the parts at the end of a unit: [NSPLIT][128][2]
     float* xsum = xmax + 2 * PF_NSPLIT * 128;
-    int* pre = reinterpret_cast<int*>(base + C::SMEM_TILES + C::CTRL_BYTES);
+    VlTables vt;
+    vt.work = reinterpret_cast<int*>(base + C::SMEM_TILES + C::CTRL_BYTES);
+    vt.order = vt.work + C::MAX_SEQ_TABLE;
+    vt.cum = vt.order + C::MAX_SEQ_TABLE;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -216,27 +239,47 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (P.varlen) {  // unit prefix per sequence: Hkv * q-tiles of each sequence
-        for (int s = threadIdx.x; s < P.num_seqs; s += blockDim.x) {
+    if (P.varlen) {  // per-launch schedule (see VlTables)
+        const int ns = P.num_seqs;
+        for (int s = threadIdx.x; s < ns; s += blockDim.x) {
             const int t = max(0, P.cu_q[s + 1] - P.cu_q[s]);
-            pre[s] = P.Hkv * ((t + PF_QPOS - 1) / PF_QPOS);
+            const int sk = max(t, P.cu_k[s + 1] - P.cu_k[s]);
+            int w = 0;
+            for (int t0 = 0; t0 < t; t0 += PF_QPOS) w += pf_tiles(t0, t, sk, P.window);
+            vt.work[s] = w;
+        }
+        __syncthreads();
+        for (int s = threadIdx.x; s < ns; s += blockDim.x) {
+            const int ws = vt.work[s];
+            int rank = 0;
+            for (int s2 = 0; s2 < ns; ++s2) {
+                const int w2 = vt.work[s2];
+                rank += (w2 > ws) || (w2 == ws && s2 < s);
+            }
+            vt.order[rank] = s;
+        }
+        __syncthreads();
+        for (int r = threadIdx.x; r < ns; r += blockDim.x) {
+            const int s = vt.order[r];
+            const int t = max(0, P.cu_q[s + 1] - P.cu_q[s]);
+            vt.cum[r] = P.Hkv * ((t + PF_QPOS - 1) / PF_QPOS);
         }
         __syncthreads();
         if (warp == 0) {  // exclusive scan, 32 entries at a time
             int carry = 0;
-            for (int s0 = 0; s0 < P.num_seqs; s0 += 32) {
+            for (int s0 = 0; s0 < ns; s0 += 32) {
                 const int s = s0 + lane;
-                const int x = (s < P.num_seqs) ? pre[s] : 0;
+                const int x = (s < ns) ? vt.cum[s] : 0;
                 int incl = x;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
                     const int y = __shfl_up_sync(0xffffffffu, incl, off);
                     if (lane >= off) incl += y;
                 }
-                if (s < P.num_seqs) pre[s] = carry + incl - x;
+                if (s < ns) vt.cum[s] = carry + incl - x;
                 carry += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (lane == 0) pre[P.num_seqs] = carry;
+            if (lane == 0) vt.cum[ns] = carry;
         }
     }
     if (warp == PF_WARP_MMA) {
@@ -254,7 +297,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const uint32_t tmem = *tmem_holder;
     const int G = gridDim.x;
     const int cta = blockIdx.x;
-    const int num_units = P.varlen ? min(P.num_units, pre[P.num_seqs]) : P.num_units;
+    const int num_units = P.varlen ? min(P.num_units, vt.cum[P.num_seqs]) : P.num_units;
     const uint64_t lim = P.timeout_ns;
 
     if (warp == PF_WARP_PRODUCER) {
@@ -268,7 +311,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int u = pf_sched(r, cta, G);
                 if (u >= num_units) continue;
                 PfUnit U;
-                pf_unit(P, pre, u, U);
+                pf_unit(P, vt, u, U);
                 if (unit_it > 0) {
                     ok = mbar_wait(q_empty, (unit_it - 1) & 1, abort_flag, lim, SITE_PROD_Q_EMPTY);
                     if (!ok) break;
@@ -400,7 +443,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int u = pf_sched(r, cta, G);
                 if (u >= num_units) continue;
                 PfUnit U;
-                pf_unit(P, pre, u, U);
+                pf_unit(P, vt, u, U);
                 ok = mbar_wait(q_full, unit_it & 1, abort_flag, lim, SITE_MMA_Q_FULL);
                 if (!ok) break;
                 tc_fence_after();
@@ -463,7 +506,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const int u = pf_sched(rr, cta, G);
             if (u >= num_units) continue;
             PfUnit U;
-            pf_unit(P, pre, u, U);
+            pf_unit(P, vt, u, U);
             const int p = U.p_min + pr;  // absolute query position of this row
             float m_ref = -INFINITY;     // log2-domain reference max of the row
             float l = 0.f;               // this part's sum of fp32 weights (for lse)

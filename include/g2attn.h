@@ -86,7 +86,10 @@ G2ATTN_API int g2attn_prefill(const void* q, const void* k, const void* v, void*
  *   cannot check these; a violation gives undefined results, never an
  *   out-of-bounds access of q/k/v/out/lse, which are bounded by total_q/k).
  * total_q and total_k are the packed extents (the host does not read the
- * device arrays). Source: as g2attn_prefill; the packing is this library's.
+ * device arrays). Limit: num_seqs <= 1024 (the kernel ranks the sequences by
+ * their work in a per-launch table in shared memory); more sequences return
+ * G2ATTN_ERR_UNSUPPORTED.
+ * Source: as g2attn_prefill; the packing is this library's.
  */
 G2ATTN_API int g2attn_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                           const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
