@@ -15,7 +15,8 @@ Printed (rank 0, one JSON line): the contract keys, plus
   clocks        nvidia-smi samples taken during the timed region
   layers        per-layer times of the step
   extra         9B pair (local/global separately), 27B decode (KV GB/s,
-                tokens/s) and the 9B ragged varlen prefill
+                tokens/s), the 9B ragged varlen prefill and the Gemma 3-shaped
+                variant of the 2B pair (window 1024, no cap)
 
 `--impl reference` times the fp64 oracle (the reference arm of this build)
 on the host cores on bounded samples of the same workload.
@@ -313,6 +314,22 @@ def extra_workloads(g2, dev, stream, flush):
         r9[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
                    "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
     res["9b_prefill"] = r9
+    del q, k, v, out, lse
+
+    # Gemma 3-shaped variant of the 2B pair: window 1024, no soft-cap
+    w = WORKLOADS["gemma3_2b"]
+    q, k, v = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+    rg = {}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        f = prefill_flops(w.B, w.T, w.S, w.H, w.d, 0, win)
+        med, best = time_launches(lambda: g2.prefill(q, k, v, query_scale=w.query_scale,
+                                                     softcap=w.softcap, window=win, out=out,
+                                                     lse=lse, stream=stream), flush, stream)
+        rg[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                   "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+    res["gemma3_2b_prefill"] = rg
     del q, k, v, out, lse
 
     # 27B decode

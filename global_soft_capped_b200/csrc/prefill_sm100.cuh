@@ -548,12 +548,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // whole warp. The capped map is monotonic in x, so the tile max
                 // is the map of the extreme accumulators and s2 - m fuses into
                 // one packed FMA below.
+                // Without the cap the map is the plain scale: the same fused path.
                 const bool fast = __all_sync(
-                    0xffffffffu, P.has_cap && !boundary &&
-                                     fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max);
+                    0xffffffffu, !boundary && (!P.has_cap ||
+                                               fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max));
                 float mt;
                 if (fast) {
-                    mt = fmaxf(series_s2(amx), series_s2(amn));
+                    mt = P.has_cap ? fmaxf(series_s2(amx), series_s2(amn))
+                                   : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
                 } else {
                     // general path: capped logits in log2 units, then the mask
                     if (P.has_cap) {
@@ -632,7 +634,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 uint32_t pk[HC / 2];
-                if (fast) {
+                if (fast && !P.has_cap) {
+                    const float2 B0 = make_float2(b0, b0);
+#pragma unroll
+                    for (int i = 0; i < HC / 2; ++i) {
+                        const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), B0, mneg);
+                        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        ls[i & 1] = add2(ls[i & 1], e);
+                        pk[i] = pack_bf16x2(e.x, e.y);
+                        lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
+                                                                  __uint_as_float(pk[i] & 0xFFFF0000u)));
+                    }
+                } else if (fast) {
                     const float2 a1 = make_float2(P.u_scale, P.u_scale);
                     const float2 B0 = make_float2(b0, b0), B1 = make_float2(b1, b1);
                     const float2 B2 = make_float2(b2, b2), B3 = make_float2(b3, b3);

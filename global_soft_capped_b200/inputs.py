@@ -71,6 +71,13 @@ WORKLOADS = {
         softcap=50.0, std=1.0, seed=4, num_seqs=16, len_lo=512, len_hi=8192,
         tail_T=1024, tail_S=8192,
         note="9B-shaped ragged packed prefill plus a chunked-prefill tail"),
+    # Gemma 3-shaped parameter variant of the same layer pair (the research-hub
+    # page: window 1024, soft-capping replaced by QK-norm, which acts on the
+    # inputs upstream of this kernel, so the cap is off here).
+    "gemma3_2b": Workload(
+        "gemma3_2b", "prefill", H=8, Hkv=4, d=256, window_local=1024, query_scale=1.0 / 16,
+        softcap=0.0, std=1.0, seed=5, B=1, T=8192, S=8192,
+        note="Gemma 3-shaped prefill layer pair: window 1024, no soft-cap"),
 }
 
 
