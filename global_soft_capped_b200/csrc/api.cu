@@ -95,6 +95,14 @@ void fill_poly(float query_scale, float softcap, g2::PfParams& P) {
     P.u_scale = softcap > 0.f ? query_scale / softcap : 0.f;
     const float a = fabsf(query_scale);
     P.poly_acc_max = (softcap > 0.f && a > 0.f) ? g2::PF_POLY_U_MAX * softcap / a : INFINITY;
+    // The series path runs in powers of the raw accumulator with the factors
+    // (alpha/C)^(2k) folded into its coefficients; use it only while the
+    // smallest folded coefficient is a comfortably normal float.
+    if (softcap > 0.f && a > 0.f) {
+        const float us2 = P.u_scale * P.u_scale;
+        const float b3 = fabsf(query_scale * kLog2e * (17.0f / 315.0f) * us2 * us2 * us2);
+        if (!(b3 > 1e-30f) || !isfinite(b3) || !isfinite(P.poly_acc_max)) P.poly_acc_max = 0.f;
+    }
 }
 
 template <int D>

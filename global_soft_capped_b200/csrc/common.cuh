@@ -358,6 +358,19 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
+// Three-input min / max (sm_100 forms of max.f32 / min.f32).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float fmin3f(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Packed fp32 pairs (sm_100 .f32x2 forms: one instruction, two lanes of work).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     float2 d;

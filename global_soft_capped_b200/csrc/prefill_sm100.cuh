@@ -487,16 +487,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int hl = r >> 6;                          // head within the pair
         const int pr = r & 63;                          // position within the tile
         const int col0 = part * HC;                     // first S column of this warp
-        // s2 = x * (b0 + b1 u^2 + b2 u^4 + b3 u^6) with u = x*alpha/C and
-        // b_k = alpha*log2(e)*c_k: the tanh series through u^7 (|u| <= 1/4:
-        // truncation below 3.3e-7 relative), scaled into log2 units.
-        const float b0 = P.scale_l2, b1 = P.scale_l2 * kTanhC1, b2 = P.scale_l2 * kTanhC2,
-                    b3 = P.scale_l2 * kTanhC3;
+        // s2 = x * (b0 + b1 x^2 + b2 x^4 + b3 x^6) with b_k = alpha*log2(e)*c_k*(alpha/C)^(2k):
+        // the tanh series through u^7 in u = x*alpha/C (|u| <= 1/4: truncation
+        // below 3.3e-7 relative), in powers of the raw accumulator x and scaled
+        // into log2 units.
+        const float us2 = P.u_scale * P.u_scale;
+        const float b0 = P.scale_l2, b1 = P.scale_l2 * kTanhC1 * us2,
+                    b2 = P.scale_l2 * kTanhC2 * us2 * us2, b3 = P.scale_l2 * kTanhC3 * us2 * us2 * us2;
         auto series_s2 = [&](float x) {
-            const float uu = x * P.u_scale, u2 = uu * uu;
-            float q = fmaf(u2, b3, b2);
-            q = fmaf(u2, q, b1);
-            q = fmaf(u2, q, b0);
+            const float x2 = x * x;
+            float q = fmaf(x2, b3, b2);
+            q = fmaf(x2, q, b1);
+            q = fmaf(x2, q, b0);
             return x * q;
         };
         uint32_t tile = 0;
@@ -538,9 +540,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) mxa[k] = mna[k] = s[k];
 #pragma unroll
-                for (int i = 4; i < HC; ++i) {
-                    mxa[i & 3] = fmaxf(mxa[i & 3], s[i]);
-                    mna[i & 3] = fminf(mna[i & 3], s[i]);
+                for (int i = 4; i < HC; i += 2) {
+                    mxa[(i >> 1) & 3] = fmax3f(mxa[(i >> 1) & 3], s[i], s[i + 1]);
+                    mna[(i >> 1) & 3] = fmin3f(mna[(i >> 1) & 3], s[i], s[i + 1]);
                 }
                 const float amx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
                 const float amn = fminf(fminf(mna[0], mna[1]), fminf(mna[2], mna[3]));
@@ -586,7 +588,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) mx[k] = s[k];
 #pragma unroll
-                    for (int i = 4; i < HC; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+                    for (int i = 4; i < HC; i += 2)
+                        mx[(i >> 1) & 3] = fmax3f(mx[(i >> 1) & 3], s[i], s[i + 1]);
                     mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                 }
                 // row max over all parts
@@ -646,17 +649,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                                                                   __uint_as_float(pk[i] & 0xFFFF0000u)));
                     }
                 } else if (fast) {
-                    const float2 a1 = make_float2(P.u_scale, P.u_scale);
                     const float2 B0 = make_float2(b0, b0), B1 = make_float2(b1, b1);
                     const float2 B2 = make_float2(b2, b2), B3 = make_float2(b3, b3);
 #pragma unroll
                     for (int i = 0; i < HC / 2; ++i) {
                         const float2 a = make_float2(s[2 * i], s[2 * i + 1]);
-                        const float2 uu = mul2(a, a1);
-                        const float2 u2 = mul2(uu, uu);
-                        float2 q = fma2(u2, B3, B2);
-                        q = fma2(u2, q, B1);
-                        q = fma2(u2, q, B0);
+                        const float2 x2 = mul2(a, a);
+                        float2 q = fma2(x2, B3, B2);
+                        q = fma2(x2, q, B1);
+                        q = fma2(x2, q, B0);
                         const float2 x = fma2(a, q, mneg);  // s2 - m
                         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         ls[i & 1] = add2(ls[i & 1], e);
