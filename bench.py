@@ -352,7 +352,55 @@ def extra_workloads(g2, dev, stream, flush):
                    "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
                    "tokens_per_s": round(len(lengths) / (med * 1e-3), 1), "kv_bytes": nbytes}
     res["27b_decode"] = rd
-    del q, k, v, out, lse, ws
+
+    # the same decode from a ring cache (local layer, 4096 slots per sequence)
+    # and from a paged cache (global layer, 64-row blocks in shuffled order)
+    n, R, bs = len(lengths), w.window_local, 64
+    Ls = torch.tensor(lengths, device=dev, dtype=torch.long)
+    cul = cu.long()
+    seq_of = torch.repeat_interleave(torch.arange(n, device=dev), Ls)
+    pos = torch.arange(int(Ls.sum()), device=dev) - cul[:-1][seq_of]
+    keep = pos >= (Ls[seq_of] - R)
+    kr = torch.zeros((n * R,) + tuple(k.shape[1:]), dtype=k.dtype, device=dev)
+    vr = torch.zeros_like(kr)
+    kr[(seq_of * R + pos % R)[keep]] = k[keep]
+    vr[(seq_of * R + pos % R)[keep]] = v[keep]
+    kr, vr = kr.view(n, R, *k.shape[1:]), vr.view(n, R, *k.shape[1:])
+    sl = Ls.to(torch.int32)
+    nblk = (Ls + bs - 1) // bs
+    total_blocks = int(nblk.sum())
+    perm = torch.randperm(total_blocks, generator=torch.Generator().manual_seed(7)).to(dev)
+    blk_start = torch.cumsum(nblk, 0) - nblk
+    blk_of_row = perm[blk_start[seq_of] + pos // bs]
+    kp = torch.zeros((total_blocks * bs,) + tuple(k.shape[1:]), dtype=k.dtype, device=dev)
+    vp = torch.zeros_like(kp)
+    kp[blk_of_row * bs + pos % bs] = k
+    vp[blk_of_row * bs + pos % bs] = v
+    kp, vp = kp.view(total_blocks, bs, *k.shape[1:]), vp.view(total_blocks, bs, *k.shape[1:])
+    table = torch.full((n, int(nblk.max())), -1, dtype=torch.int32, device=dev)
+    for s_ in range(n):
+        table[s_, :int(nblk[s_])] = perm[int(blk_start[s_]):int(blk_start[s_] + nblk[s_])].int()
+    del k, v
+    rl = {}
+    nbytes = decode_kv_bytes(lengths, w.Hkv, w.d, w.window_local)
+    med, best = time_launches(lambda: g2.decode_ring(q, kr, vr, sl, w.window_local,
+                                                     query_scale=w.query_scale,
+                                                     softcap=w.softcap, out=out, lse=lse,
+                                                     workspace=ws, stream=stream), flush, stream)
+    gbs = nbytes / (med * 1e-3) / 1e9
+    rl["ring_local"] = {"ms": round(med, 4), "kv_GBps": round(gbs, 1),
+                        "frac_hbm": round(gbs / pk["hbm_gbs"], 4), "ring_slots": R}
+    nbytes = decode_kv_bytes(lengths, w.Hkv, w.d, 0)
+    med, best = time_launches(lambda: g2.decode_paged(q, kp, vp, table, sl, max(lengths),
+                                                      query_scale=w.query_scale,
+                                                      softcap=w.softcap, window=0, out=out,
+                                                      lse=lse, workspace=ws, stream=stream),
+                              flush, stream)
+    gbs = nbytes / (med * 1e-3) / 1e9
+    rl["paged_global"] = {"ms": round(med, 4), "kv_GBps": round(gbs, 1),
+                          "frac_hbm": round(gbs / pk["hbm_gbs"], 4), "block_size": bs}
+    res["27b_decode_cache_layouts"] = rl
+    del q, kr, vr, kp, vp, out, lse, ws
 
     # 9B ragged packed prefill (16 sequences + chunked-prefill tail)
     w = WORKLOADS["9b_varlen"]

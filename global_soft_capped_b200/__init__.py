@@ -4,7 +4,8 @@ Two layers:
 
 * The C entry points under their own names (``g2attn_prefill``,
   ``g2attn_prefill_varlen``, ``g2attn_decode_workspace_size``,
-  ``g2attn_decode``, ``g2attn_decode_noalloc``, ``g2attn_status_string``,
+  ``g2attn_decode``, ``g2attn_decode_ring``, ``g2attn_decode_paged``,
+  ``g2attn_decode_noalloc``, ``g2attn_status_string``,
   ``g2attn_get_device_error``,
   ``g2attn_selftest_wait_timeout``): plain argument marshalling of integers,
   floats and raw pointers through ctypes, returning the status code.
@@ -37,6 +38,8 @@ EXPORTS = (
     "g2attn_prefill_varlen",
     "g2attn_decode_workspace_size",
     "g2attn_decode",
+    "g2attn_decode_ring",
+    "g2attn_decode_paged",
     "g2attn_decode_noalloc",
     "g2attn_status_string",
     "g2attn_get_device_error",
@@ -72,6 +75,10 @@ def load_library():
     lib.g2attn_decode_workspace_size.restype = SZ
     lib.g2attn_decode.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P, SZ, P]
     lib.g2attn_decode.restype = I
+    lib.g2attn_decode_ring.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P, SZ, P]
+    lib.g2attn_decode_ring.restype = I
+    lib.g2attn_decode_paged.argtypes = [P, P, P, P, P, P, P] + [I] * 8 + [F, F, I, P, SZ, P]
+    lib.g2attn_decode_paged.restype = I
     lib.g2attn_decode_noalloc.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P]
     lib.g2attn_decode_noalloc.restype = I
     lib.g2attn_status_string.argtypes = [I]
@@ -109,6 +116,24 @@ def g2attn_decode(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs, total_k
     return load_library().g2attn_decode(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs,
                                         total_k, max_cache_len, H, Hkv, d, query_scale, softcap,
                                         window, workspace, workspace_bytes, stream)
+
+
+def g2attn_decode_ring(q, k_ring, v_ring, seq_lens, out, lse, num_seqs, ring_size, max_cache_len,
+                       H, Hkv, d, query_scale, softcap, window, workspace, workspace_bytes,
+                       stream):
+    return load_library().g2attn_decode_ring(q, k_ring, v_ring, seq_lens, out, lse, num_seqs,
+                                             ring_size, max_cache_len, H, Hkv, d, query_scale,
+                                             softcap, window, workspace, workspace_bytes, stream)
+
+
+def g2attn_decode_paged(q, k_blocks, v_blocks, block_table, seq_lens, out, lse, num_seqs,
+                        num_blocks, block_size, max_blocks_per_seq, max_cache_len, H, Hkv, d,
+                        query_scale, softcap, window, workspace, workspace_bytes, stream):
+    return load_library().g2attn_decode_paged(q, k_blocks, v_blocks, block_table, seq_lens, out,
+                                              lse, num_seqs, num_blocks, block_size,
+                                              max_blocks_per_seq, max_cache_len, H, Hkv, d,
+                                              query_scale, softcap, window, workspace,
+                                              workspace_bytes, stream)
 
 
 def g2attn_decode_noalloc(q, k_cache, v_cache, cu_seqlens_k, out, lse, num_seqs, total_k,
@@ -225,4 +250,51 @@ def decode(q, k_cache, v_cache, cu_seqlens_k, max_cache_len, *, query_scale=1.0,
                        _stream(stream))
     if st != G2ATTN_OK:
         raise G2AttnError(st, "g2attn_decode")
+    return out, lse
+
+
+def decode_ring(q, k_ring, v_ring, seq_lens, window, max_cache_len=None, *, query_scale=1.0,
+                softcap=50.0, out=None, lse=None, workspace=None, want_lse=True, stream=None):
+    """Decode over ring caches (n, R, Hkv, d); seq_lens int32 CUDA (n,)."""
+    import torch
+    _check_bf16(q, k_ring, v_ring)
+    n, H, d = q.shape
+    R, Hkv = k_ring.shape[1], k_ring.shape[2]
+    max_cache_len = int(window if max_cache_len is None else max_cache_len)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((n, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(n, H, d, max_cache_len, q.device)
+    st = g2attn_decode_ring(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(seq_lens), _ptr(out),
+                            _ptr(lse), n, R, max_cache_len, H, Hkv, d, float(query_scale),
+                            float(softcap), int(window), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    if st != G2ATTN_OK:
+        raise G2AttnError(st, "g2attn_decode_ring")
+    return out, lse
+
+
+def decode_paged(q, k_blocks, v_blocks, block_table, seq_lens, max_cache_len, *,
+                 query_scale=1.0, softcap=50.0, window=0, out=None, lse=None, workspace=None,
+                 want_lse=True, stream=None):
+    """Decode over paged caches (num_blocks, bs, Hkv, d); block_table int32 (n, max_blocks)."""
+    import torch
+    _check_bf16(q, k_blocks, v_blocks)
+    n, H, d = q.shape
+    nb, bs, Hkv = k_blocks.shape[0], k_blocks.shape[1], k_blocks.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((n, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(n, H, d, max_cache_len, q.device)
+    st = g2attn_decode_paged(_ptr(q), _ptr(k_blocks), _ptr(v_blocks), _ptr(block_table),
+                             _ptr(seq_lens), _ptr(out), _ptr(lse), n, nb, bs,
+                             block_table.shape[1], int(max_cache_len), H, Hkv, d,
+                             float(query_scale), float(softcap), int(window), _ptr(workspace),
+                             workspace.numel(), _stream(stream))
+    if st != G2ATTN_OK:
+        raise G2AttnError(st, "g2attn_decode_paged")
     return out, lse

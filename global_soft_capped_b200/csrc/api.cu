@@ -161,14 +161,67 @@ size_t decode_ws_bytes(int num_seqs, int H, int d, int max_len, int chunk) {
     return ml + slots * static_cast<size_t>(d) * sizeof(float);
 }
 
-template <int D>
-int launch_decode(g2::DecParams& P, cudaStream_t stream) {
+template <int D, int LAYOUT>
+int launch_decode(g2::DecParams& P, const g2::DecLayoutParams& LP, cudaStream_t stream) {
     dim3 grid(P.max_splits, P.Hkv, P.num_seqs);
-    g2::decode_split<D><<<grid, g2::DEC_THREADS, 0, stream>>>(P);
+    // ring / paged layouts: per-CTA table of the chunk's cache rows
+    const size_t dyn = (LAYOUT == g2::DEC_LINEAR) ? 0 : static_cast<size_t>(P.chunk) * sizeof(int);
+    g2::decode_split<D, LAYOUT><<<grid, g2::DEC_THREADS, dyn, stream>>>(P, LP);
     if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
     const int warps = P.num_seqs * P.H;
-    g2::decode_merge<D><<<(warps + 3) / 4, 128, 0, stream>>>(P);
+    g2::decode_merge<D, LAYOUT><<<(warps + 3) / 4, 128, 0, stream>>>(P, LP);
     return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+}
+
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int log2i(int x) {
+    int r = 0;
+    while ((1 << r) < x) ++r;
+    return r;
+}
+
+// Checks shared by every decode layout, then the split plan and workspace
+// carving; launches the layout's kernels on success.
+template <int LAYOUT>
+int decode_common(g2::DecParams& P, const g2::DecLayoutParams& LP, const void* q, const void* k_cache, const void* v_cache,
+                  void* out, float* lse, int num_seqs, int max_cache_len, int H, int Hkv, int d,
+                  float query_scale, float softcap, int window, void* workspace,
+                  size_t workspace_bytes, g2attn_stream_t stream) {
+    if (!q || !k_cache || !v_cache || !out) return G2ATTN_ERR_INVALID_ARG;
+    if (num_seqs <= 0 || max_cache_len <= 0) return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (lse && !aligned16(lse)) || (workspace && !aligned16(workspace)))
+        return G2ATTN_ERR_MISALIGNED;
+    const int chunk = decode_chunk(num_seqs, H, max_cache_len);
+    const size_t need = decode_ws_bytes(num_seqs, H, d, max_cache_len, chunk);
+    if (!workspace || workspace_bytes < need) return G2ATTN_ERR_WORKSPACE;
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.k = static_cast<const __nv_bfloat16*>(k_cache);
+    P.v = static_cast<const __nv_bfloat16*>(v_cache);
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    const int splits = (max_cache_len + chunk - 1) / chunk;
+    size_t ml = static_cast<size_t>(num_seqs) * H * splits * 2 * sizeof(float);
+    ml = (ml + 255) & ~static_cast<size_t>(255);
+    P.ws_ml = static_cast<float*>(workspace);
+    P.ws_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + ml);
+    P.num_seqs = num_seqs;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.window = window;
+    P.chunk = chunk;
+    P.max_splits = splits;
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (d) {
+        case 64: return launch_decode<64, LAYOUT>(P, LP, st);
+        case 128: return launch_decode<128, LAYOUT>(P, LP, st);
+        case 256: return launch_decode<256, LAYOUT>(P, LP, st);
+        default: return G2ATTN_ERR_UNSUPPORTED;
+    }
 }
 
 __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
@@ -303,44 +356,61 @@ int g2attn_decode(const void* q, const void* k_cache, const void* v_cache,
                   const int* cu_seqlens_k, void* out, float* lse, int num_seqs, int total_k,
                   int max_cache_len, int H, int Hkv, int d, float query_scale, float softcap,
                   int window, void* workspace, size_t workspace_bytes, g2attn_stream_t stream) {
-    if (!q || !k_cache || !v_cache || !cu_seqlens_k || !out) return G2ATTN_ERR_INVALID_ARG;
-    if (num_seqs <= 0 || total_k <= 0 || max_cache_len <= 0) return G2ATTN_ERR_INVALID_ARG;
-    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
-    if (rc) return rc;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-        (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
-        (workspace && !aligned16(workspace)))
-        return G2ATTN_ERR_MISALIGNED;
-    const int chunk = decode_chunk(num_seqs, H, max_cache_len);
-    const size_t need = decode_ws_bytes(num_seqs, H, d, max_cache_len, chunk);
-    if (!workspace || workspace_bytes < need) return G2ATTN_ERR_WORKSPACE;
+    if (!cu_seqlens_k || total_k <= 0) return G2ATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) return G2ATTN_ERR_MISALIGNED;
     g2::DecParams P{};
-    P.q = static_cast<const __nv_bfloat16*>(q);
-    P.k = static_cast<const __nv_bfloat16*>(k_cache);
-    P.v = static_cast<const __nv_bfloat16*>(v_cache);
     P.cu_k = cu_seqlens_k;
-    P.out = static_cast<__nv_bfloat16*>(out);
-    P.lse = lse;
-    const int splits = (max_cache_len + chunk - 1) / chunk;
-    size_t ml = static_cast<size_t>(num_seqs) * H * splits * 2 * sizeof(float);
-    ml = (ml + 255) & ~static_cast<size_t>(255);
-    P.ws_ml = static_cast<float*>(workspace);
-    P.ws_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + ml);
-    P.num_seqs = num_seqs;
     P.total_k = total_k;
-    P.H = H;
-    P.Hkv = Hkv;
-    P.window = window;
-    P.chunk = chunk;
-    P.max_splits = splits;
-    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    switch (d) {
-        case 64: return launch_decode<64>(P, st);
-        case 128: return launch_decode<128>(P, st);
-        case 256: return launch_decode<256>(P, st);
-        default: return G2ATTN_ERR_UNSUPPORTED;
-    }
+    const g2::DecLayoutParams LP{};
+    return decode_common<g2::DEC_LINEAR>(P, LP, q, k_cache, v_cache, out, lse, num_seqs,
+                                         max_cache_len, H, Hkv, d, query_scale, softcap, window,
+                                         workspace, workspace_bytes, stream);
+}
+
+int g2attn_decode_ring(const void* q, const void* k_ring, const void* v_ring,
+                       const int* seq_lens, void* out, float* lse, int num_seqs, int ring_size,
+                       int max_cache_len, int H, int Hkv, int d, float query_scale,
+                       float softcap, int window, void* workspace, size_t workspace_bytes,
+                       g2attn_stream_t stream) {
+    if (!seq_lens) return G2ATTN_ERR_INVALID_ARG;
+    if (!pow2(ring_size) || window <= 0 || window > ring_size) return G2ATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(num_seqs) * ring_size > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(seq_lens) & 3u) return G2ATTN_ERR_MISALIGNED;
+    g2::DecParams P{};
+    g2::DecLayoutParams LP{};
+    LP.seq_lens = seq_lens;
+    LP.ring_mask = ring_size - 1;
+    LP.ring_shift = log2i(ring_size);
+    return decode_common<g2::DEC_RING>(P, LP, q, k_ring, v_ring, out, lse, num_seqs, max_cache_len,
+                                       H, Hkv, d, query_scale, softcap, window, workspace,
+                                       workspace_bytes, stream);
+}
+
+int g2attn_decode_paged(const void* q, const void* k_blocks, const void* v_blocks,
+                        const int* block_table, const int* seq_lens, void* out, float* lse,
+                        int num_seqs, int num_blocks, int block_size, int max_blocks_per_seq,
+                        int max_cache_len, int H, int Hkv, int d, float query_scale,
+                        float softcap, int window, void* workspace, size_t workspace_bytes,
+                        g2attn_stream_t stream) {
+    if (!block_table || !seq_lens) return G2ATTN_ERR_INVALID_ARG;
+    if (!pow2(block_size) || num_blocks <= 0 || max_blocks_per_seq <= 0)
+        return G2ATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(num_blocks) * block_size > INT32_MAX ||
+        static_cast<long long>(max_blocks_per_seq) * block_size > INT32_MAX)
+        return G2ATTN_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return G2ATTN_ERR_MISALIGNED;
+    g2::DecParams P{};
+    g2::DecLayoutParams LP{};
+    LP.seq_lens = seq_lens;
+    LP.block_table = block_table;
+    LP.block_shift = log2i(block_size);
+    LP.max_blocks = max_blocks_per_seq;
+    LP.num_blocks = num_blocks;
+    return decode_common<g2::DEC_PAGED>(P, LP, q, k_blocks, v_blocks, out, lse, num_seqs,
+                                        max_cache_len, H, Hkv, d, query_scale, softcap, window,
+                                        workspace, workspace_bytes, stream);
 }
 
 int g2attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

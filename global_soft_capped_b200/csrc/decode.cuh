@@ -24,11 +24,19 @@ namespace g2 {
 constexpr int DEC_THREADS = 128;
 constexpr int DEC_MAX_CHUNK = 512;
 
+// KV cache layouts of the decode path. Every layout stores rows of
+// (Hkv, d) bf16; they differ in where position p of sequence s lives.
+//   DEC_LINEAR  packed by cu_seqlens_k:      row = cu_k[s] + p
+//   DEC_RING    ring of R slots per sequence: row = s*R + p mod R (R a power of
+//               two; holds the last R positions, enough for a window <= R)
+//   DEC_PAGED   blocks of bs rows:           row = block_table[s][p / bs]*bs + p mod bs
+enum DecLayout : int { DEC_LINEAR = 0, DEC_RING = 1, DEC_PAGED = 2 };
+
 struct DecParams {
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
-    const int* cu_k;
+    const int* cu_k;         // DEC_LINEAR
     __nv_bfloat16* out;
     float* lse;
     float* ws_ml;   // [n][H][max_splits][2]  (m, l) log2 domain
@@ -38,15 +46,58 @@ struct DecParams {
     int has_cap;
 };
 
-__device__ __forceinline__ void dec_range(const DecParams& P, int s, int& lo, int& hi,
-                                          int& nsplit) {
-    int k0 = P.cu_k[s], k1 = P.cu_k[s + 1];
-    k0 = max(0, min(k0, P.total_k));  // never read outside the cache
-    k1 = max(k0, min(k1, P.total_k));
-    const int L = k1 - k0;
+// Layout-specific parameters, a separate kernel argument (kept out of
+// DecParams: a larger DecParams raised the linear kernel's registers and cost
+// occupancy).
+struct DecLayoutParams {
+    const int* seq_lens;     // DEC_RING, DEC_PAGED: tokens seen per sequence
+    const int* block_table;  // DEC_PAGED: [num_seqs][max_blocks]
+    int ring_mask;           // DEC_RING: R - 1
+    int ring_shift;          // DEC_RING: log2 R
+    int block_shift;         // DEC_PAGED: log2 bs
+    int max_blocks;          // DEC_PAGED: blocks per sequence in the table
+    int num_blocks;          // DEC_PAGED: blocks in the cache
+};
+
+// Tokens seen by sequence s (the query sits at position L - 1).
+template <int LAYOUT>
+__device__ __forceinline__ int dec_len(const DecParams& P, const DecLayoutParams& LP, int s) {
+    if (LAYOUT == DEC_LINEAR) {
+        const int k0 = max(0, min(P.cu_k[s], P.total_k));  // never read outside the cache
+        const int k1 = max(k0, min(P.cu_k[s + 1], P.total_k));
+        return k1 - k0;
+    } else if (LAYOUT == DEC_PAGED) {
+        return max(0, min(LP.seq_lens[s], LP.max_blocks << LP.block_shift));
+    } else {
+        return max(0, LP.seq_lens[s]);
+    }
+}
+
+// Cache row of position p of sequence s for the ring and paged layouts
+// (always inside the cache arrays).
+template <int LAYOUT>
+__device__ __forceinline__ int dec_row(const DecLayoutParams& LP, int s, int p) {
+    if constexpr (LAYOUT == DEC_RING) {
+        return (s << LP.ring_shift) + (p & LP.ring_mask);
+    } else {
+        int b = LP.block_table[static_cast<size_t>(s) * LP.max_blocks + (p >> LP.block_shift)];
+        b = max(0, min(b, LP.num_blocks - 1));
+        return (b << LP.block_shift) + (p & ((1 << LP.block_shift) - 1));
+    }
+}
+
+// Visible key range [lo, hi) of sequence s and its number of splits. A ring
+// holds only its last R positions: the range is clipped to them.
+template <int LAYOUT>
+__device__ __forceinline__ void dec_range(const DecParams& P, const DecLayoutParams& LP, int s,
+                                          int& lo, int& hi, int& nsplit) {
+    const int L = dec_len<LAYOUT>(P, LP, s);
     lo = (P.window > 0) ? max(0, L - P.window) : 0;
+    if (LAYOUT == DEC_RING) lo = max(lo, L - (LP.ring_mask + 1));
     hi = L;
-    nsplit = (hi - lo + P.chunk - 1) / P.chunk;
+    // more splits than planned only when the caller's max_cache_len undercounts:
+    // drop the excess (wrong result, but never a read past the workspace)
+    nsplit = min((hi - lo + P.chunk - 1) / P.chunk, P.max_splits);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
@@ -66,24 +117,28 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     return r;
 }
 
-template <int D>
-__global__ void __launch_bounds__(DEC_THREADS) decode_split(const DecParams P) {
+template <int D, int LAYOUT>
+__global__ void __launch_bounds__(DEC_THREADS) decode_split(const DecParams P, const DecLayoutParams LP) {
     constexpr int TPR = D / 8;               // threads per key row (8 bf16 each)
     constexpr int RPW = 32 / TPR;            // rows per warp per load
     constexpr int RPC = RPW * (DEC_THREADS / 32);  // rows per CTA per load
-    constexpr int UNR = 4;                   // loads in flight per thread
+    // loads in flight per thread: the linear layout steps one pointer by a
+    // constant stride (offsets fold into the loads); the others read each
+    // key's cache row from a per-CTA table and keep more loads in flight
+    constexpr int UNR = (LAYOUT == DEC_LINEAR) ? 4 : 8;
     __shared__ float sc[2][DEC_MAX_CHUNK];
     __shared__ float red[RPC][2][D];
     __shared__ float wred[2][DEC_THREADS / 32];
 
     const int s = blockIdx.z, g = blockIdx.y, sp = blockIdx.x;
     int lo, hi, nsplit;
-    dec_range(P, s, lo, hi, nsplit);
+    dec_range<LAYOUT>(P, LP, s, lo, hi, nsplit);
     if (sp >= nsplit) return;
     const int kb = lo + sp * P.chunk;
     const int ke = min(hi, kb + P.chunk);
     const int n = ke - kb;
-    const size_t row0 = static_cast<size_t>(max(0, min(P.cu_k[s], P.total_k)));
+    size_t row0 = 0;  // linear layout: first cache row of the sequence
+    if constexpr (LAYOUT == DEC_LINEAR) row0 = static_cast<size_t>(max(0, min(P.cu_k[s], P.total_k)));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rw = lane / TPR, cg = lane % TPR;
@@ -97,8 +152,17 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split(const DecParams P) {
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(qp + D), q1);
     }
     const size_t kstride = static_cast<size_t>(P.Hkv) * D;
-    const __nv_bfloat16* kbase = P.k + (row0 + kb) * kstride + static_cast<size_t>(g) * D + cg * 8;
-    const __nv_bfloat16* vbase = P.v + (row0 + kb) * kstride + static_cast<size_t>(g) * D + cg * 8;
+    // linear layout: base pointers of this chunk, stepped by j rows below
+    const __nv_bfloat16* klin = P.k + (row0 + kb) * kstride + static_cast<size_t>(g) * D + cg * 8;
+    const __nv_bfloat16* vlin = P.v + (row0 + kb) * kstride + static_cast<size_t>(g) * D + cg * 8;
+    const size_t gofs = static_cast<size_t>(g) * D + cg * 8;  // this thread's columns
+    // other layouts: cache row of every key of the chunk (dynamic shared memory,
+    // n <= chunk entries, sized at launch)
+    extern __shared__ int rows_dyn[];
+    if constexpr (LAYOUT != DEC_LINEAR) {
+        for (int j = tid; j < n; j += DEC_THREADS) rows_dyn[j] = dec_row<LAYOUT>(LP, s, kb + j);
+        __syncthreads();
+    }
 
     // ---- phase 1: scores (log2 domain, capped)
     for (int base = 0; base < n; base += RPC * UNR) {
@@ -106,7 +170,12 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split(const DecParams P) {
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
             const int j = base + u * RPC + rslot;
-            kv[u] = (j < n) ? ldg_stream(kbase + static_cast<size_t>(j) * kstride)
+            const __nv_bfloat16* kp;
+            if constexpr (LAYOUT == DEC_LINEAR)
+                kp = klin + static_cast<size_t>(j) * kstride;
+            else
+                kp = P.k + static_cast<size_t>(rows_dyn[j < n ? j : 0]) * kstride + gofs;
+            kv[u] = (j < n) ? ldg_stream(kp)
                             : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
@@ -203,7 +272,12 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split(const DecParams P) {
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
             const int j = base + u * RPC + rslot;
-            vv[u] = (j < n) ? ldg_stream(vbase + static_cast<size_t>(j) * kstride)
+            const __nv_bfloat16* vp;
+            if constexpr (LAYOUT == DEC_LINEAR)
+                vp = vlin + static_cast<size_t>(j) * kstride;
+            else
+                vp = P.v + static_cast<size_t>(rows_dyn[j < n ? j : 0]) * kstride + gofs;
+            vv[u] = (j < n) ? ldg_stream(vp)
                             : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
@@ -260,14 +334,14 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split(const DecParams P) {
     }
 }
 
-template <int D>
-__global__ void __launch_bounds__(128) decode_merge(const DecParams P) {
+template <int D, int LAYOUT>
+__global__ void __launch_bounds__(128) decode_merge(const DecParams P, const DecLayoutParams LP) {
     const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (wid >= P.num_seqs * P.H) return;
     const int s = wid / P.H, h = wid % P.H;
     int lo, hi, nsplit;
-    dec_range(P, s, lo, hi, nsplit);
+    dec_range<LAYOUT>(P, LP, s, lo, hi, nsplit);
     if (nsplit <= 1) return;  // written by decode_split
     const size_t slot0 = (static_cast<size_t>(s) * P.H + h) * P.max_splits;
     float M = -INFINITY;

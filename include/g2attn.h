@@ -124,6 +124,46 @@ G2ATTN_API int g2attn_decode(const void* q, const void* k_cache, const void* v_c
                   void* workspace, size_t workspace_bytes, g2attn_stream_t stream);
 
 /*
+ * Decode over a ring-buffer KV cache, for local layers: each sequence keeps only
+ * its last ring_size cached tokens (the Guide's serving note: local layers
+ * only store 4,096 tokens; the Hub page: the local layer's cache is bounded by
+ * its window).
+ *   q (num_seqs, H, d); k_ring, v_ring (num_seqs, ring_size, Hkv, d): position
+ *   p of sequence s is in slot p mod ring_size of that sequence.
+ *   seq_lens: device int32 [num_seqs], L_s >= 1 tokens seen so far; the query
+ *   sits at position L_s - 1 and sees positions max(0, L_s - window) .. L_s - 1.
+ *   Requires ring_size a power of two and 0 < window <= ring_size.
+ *   max_cache_len: at least the keys any query sees (min(L_s, window)); it
+ *   sizes the split plan and the workspace (g2attn_decode_workspace_size).
+ *   out, lse, workspace and errors as g2attn_decode.
+ */
+G2ATTN_API int g2attn_decode_ring(const void* q, const void* k_ring, const void* v_ring,
+                       const int* seq_lens, void* out, float* lse, int num_seqs, int ring_size,
+                       int max_cache_len, int H, int Hkv, int d, float query_scale,
+                       float softcap, int window, void* workspace, size_t workspace_bytes,
+                       g2attn_stream_t stream);
+
+/*
+ * Decode over a paged KV cache: fixed blocks of block_size token rows, located
+ * through a per-sequence block table (the block-managed caches of the serving
+ * runtimes the Guide names, "Deep Dive" item 2).
+ *   k_blocks, v_blocks (num_blocks, block_size, Hkv, d); block_table: device
+ *   int32 [num_seqs][max_blocks_per_seq], entry b = cache block of positions
+ *   b*block_size .. b*block_size + block_size - 1; seq_lens: device int32
+ *   [num_seqs], L_s >= 1, L_s <= max_blocks_per_seq * block_size.
+ *   Requires block_size a power of two. Table entries outside [0, num_blocks)
+ *   are clamped (undefined results, never an out-of-bounds read).
+ *   max_cache_len: at least the keys any query sees. Global (window 0) and
+ *   local layers; out, lse, workspace and errors as g2attn_decode.
+ */
+G2ATTN_API int g2attn_decode_paged(const void* q, const void* k_blocks, const void* v_blocks,
+                        const int* block_table, const int* seq_lens, void* out, float* lse,
+                        int num_seqs, int num_blocks, int block_size, int max_blocks_per_seq,
+                        int max_cache_len, int H, int Hkv, int d, float query_scale,
+                        float softcap, int window, void* workspace, size_t workspace_bytes,
+                        g2attn_stream_t stream);
+
+/*
  * Decode without allocating: the same operation and arguments as
  * g2attn_decode, minus the workspace. For callers that cannot allocate device
  * memory at call time -- a serving loop whose device memory is planned up

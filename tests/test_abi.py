@@ -109,3 +109,26 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(g2, "_lib", None)
     with pytest.raises(RuntimeError, match="libg2attn.so is missing"):
         g2.load_library()
+
+
+def test_ring_and_paged_reject_before_launch(lib):
+    cu = ctypes.c_void_p(1 << 21)
+    ring = [FAKE, FAKE, FAKE, cu, FAKE, None, 4, 4096, 4096, 32, 16, 128, 0.083, 50.0, 4096,
+            FAKE, 1 << 30, None]
+    bad = list(ring); bad[7] = 3000          # ring size not a power of two
+    assert g2.g2attn_decode_ring(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(ring); bad[14] = 0            # a ring serves local layers only
+    assert g2.g2attn_decode_ring(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(ring); bad[14] = 8192         # window larger than the ring
+    assert g2.g2attn_decode_ring(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(ring); bad[3] = None
+    assert g2.g2attn_decode_ring(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    paged = [FAKE, FAKE, FAKE, cu, cu, FAKE, None, 4, 100, 48, 10, 4096, 32, 16, 128, 0.083,
+             50.0, 0, FAKE, 1 << 30, None]
+    bad = list(paged); bad[9] = 48           # block size not a power of two
+    assert g2.g2attn_decode_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    paged[9] = 64
+    bad = list(paged); bad[3] = None         # no block table
+    assert g2.g2attn_decode_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(paged); bad[18] = None        # no workspace
+    assert g2.g2attn_decode_paged(*bad) == g2.G2ATTN_ERR_WORKSPACE
