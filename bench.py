@@ -420,6 +420,39 @@ def extra_workloads(g2, dev, stream, flush):
         rv[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
                    "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
     res["9b_varlen"] = rv
+
+    # the same packed queries with K/V in a paged cache (256-row blocks, shuffled)
+    bs = 256
+    Sl = torch.tensor(Ss, device=dev, dtype=torch.long)
+    nblk = (Sl + bs - 1) // bs
+    total_blocks = int(nblk.sum())
+    perm = torch.randperm(total_blocks, generator=torch.Generator().manual_seed(9)).to(dev)
+    seq_of = torch.repeat_interleave(torch.arange(len(Ss), device=dev), Sl)
+    pos = torch.arange(int(Sl.sum()), device=dev) - ck.long()[:-1][seq_of]
+    bstart = torch.cumsum(nblk, 0) - nblk
+    dst = perm[bstart[seq_of] + pos // bs] * bs + pos % bs
+    kp = torch.zeros((total_blocks * bs,) + tuple(k.shape[1:]), dtype=k.dtype, device=dev)
+    vp = torch.zeros_like(kp)
+    kp[dst] = k
+    vp[dst] = v
+    kp, vp = kp.view(total_blocks, bs, *k.shape[1:]), vp.view(total_blocks, bs, *k.shape[1:])
+    table = torch.full((len(Ss), int(nblk.max())), -1, dtype=torch.int32, device=dev)
+    for s_ in range(len(Ss)):
+        table[s_, :int(nblk[s_])] = perm[int(bstart[s_]):int(bstart[s_] + nblk[s_])].int()
+    sl = Sl.to(torch.int32)
+    del k, v
+    rp = {}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        f = varlen_flops(Ts, Ss, w.H, w.d, win)
+        med, best = time_launches(lambda: g2.prefill_paged(q, kp, vp, cq, table, sl, max(Ts),
+                                                           max(Ss), query_scale=w.query_scale,
+                                                           softcap=w.softcap, window=win,
+                                                           out=out, lse=lse, stream=stream),
+                                  flush, stream)
+        rp[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                   "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+                   "block_size": bs}
+    res["9b_varlen_paged_kv"] = rp
     return res
 
 

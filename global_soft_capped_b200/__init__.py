@@ -3,7 +3,7 @@
 Two layers:
 
 * The C entry points under their own names (``g2attn_prefill``,
-  ``g2attn_prefill_varlen``, ``g2attn_decode_workspace_size``,
+  ``g2attn_prefill_varlen``, ``g2attn_prefill_paged``, ``g2attn_decode_workspace_size``,
   ``g2attn_decode``, ``g2attn_decode_ring``, ``g2attn_decode_paged``,
   ``g2attn_decode_noalloc``, ``g2attn_status_string``,
   ``g2attn_get_device_error``,
@@ -36,6 +36,7 @@ G2ATTN_ERR_WORKSPACE = 6
 EXPORTS = (
     "g2attn_prefill",
     "g2attn_prefill_varlen",
+    "g2attn_prefill_paged",
     "g2attn_decode_workspace_size",
     "g2attn_decode",
     "g2attn_decode_ring",
@@ -71,6 +72,8 @@ def load_library():
     lib.g2attn_prefill.restype = I
     lib.g2attn_prefill_varlen.argtypes = [P, P, P, P, P, P, P] + [I] * 8 + [F, F, I, P]
     lib.g2attn_prefill_varlen.restype = I
+    lib.g2attn_prefill_paged.argtypes = [P, P, P, P, P, P, P, P] + [I] * 10 + [F, F, I, P]
+    lib.g2attn_prefill_paged.restype = I
     lib.g2attn_decode_workspace_size.argtypes = [I, I, I, I]
     lib.g2attn_decode_workspace_size.restype = SZ
     lib.g2attn_decode.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P, SZ, P]
@@ -105,6 +108,16 @@ def g2attn_prefill_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, num_seq
     return load_library().g2attn_prefill_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k,
                                                 num_seqs, total_q, total_k, max_T, max_S, H, Hkv,
                                                 d, query_scale, softcap, window, stream)
+
+
+def g2attn_prefill_paged(q, k_blocks, v_blocks, out, lse, cu_seqlens_q, block_table, seq_lens_k,
+                         num_seqs, total_q, num_blocks, block_size, max_blocks_per_seq, max_T,
+                         max_S, H, Hkv, d, query_scale, softcap, window, stream):
+    return load_library().g2attn_prefill_paged(q, k_blocks, v_blocks, out, lse, cu_seqlens_q,
+                                               block_table, seq_lens_k, num_seqs, total_q,
+                                               num_blocks, block_size, max_blocks_per_seq, max_T,
+                                               max_S, H, Hkv, d, query_scale, softcap, window,
+                                               stream)
 
 
 def g2attn_decode_workspace_size(num_seqs, H, d, max_cache_len):
@@ -297,4 +310,27 @@ def decode_paged(q, k_blocks, v_blocks, block_table, seq_lens, max_cache_len, *,
                              workspace.numel(), _stream(stream))
     if st != G2ATTN_OK:
         raise G2AttnError(st, "g2attn_decode_paged")
+    return out, lse
+
+
+def prefill_paged(q, k_blocks, v_blocks, cu_seqlens_q, block_table, seq_lens_k, max_T, max_S, *,
+                  query_scale=1.0, softcap=50.0, window=0, out=None, lse=None, want_lse=True,
+                  stream=None):
+    """Chunked prefill: packed q (sum T,H,d) over paged K/V (num_blocks, bs, Hkv, d)."""
+    import torch
+    _check_bf16(q, k_blocks, v_blocks)
+    total_q, H, d = q.shape
+    nb, bs, Hkv = k_blocks.shape[0], k_blocks.shape[1], k_blocks.shape[2]
+    num_seqs = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    st = g2attn_prefill_paged(_ptr(q), _ptr(k_blocks), _ptr(v_blocks), _ptr(out), _ptr(lse),
+                              _ptr(cu_seqlens_q), _ptr(block_table), _ptr(seq_lens_k), num_seqs,
+                              total_q, nb, bs, block_table.shape[1], int(max_T), int(max_S), H,
+                              Hkv, d, float(query_scale), float(softcap), int(window),
+                              _stream(stream))
+    if st != G2ATTN_OK:
+        raise G2AttnError(st, "g2attn_prefill_paged")
     return out, lse

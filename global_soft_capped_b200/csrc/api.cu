@@ -347,6 +347,60 @@ int g2attn_prefill_varlen(const void* q, const void* k, const void* v, void* out
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+int g2attn_prefill_paged(const void* q, const void* k_blocks, const void* v_blocks, void* out,
+                         float* lse, const int* cu_seqlens_q, const int* block_table,
+                         const int* seq_lens_k, int num_seqs, int total_q, int num_blocks,
+                         int block_size, int max_blocks_per_seq, int max_T, int max_S, int H,
+                         int Hkv, int d, float query_scale, float softcap, int window,
+                         g2attn_stream_t stream) {
+    if (!q || !k_blocks || !v_blocks || !out || !cu_seqlens_q || !block_table || !seq_lens_k)
+        return G2ATTN_ERR_INVALID_ARG;
+    if (num_seqs <= 0 || total_q <= 0 || max_T <= 0 || max_S <= 0 || max_T > max_S ||
+        max_T > total_q || num_blocks <= 0 || max_blocks_per_seq <= 0)
+        return G2ATTN_ERR_INVALID_ARG;
+    if (!pow2(block_size) || block_size < g2::PF_BN) return G2ATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(max_blocks_per_seq) * block_size < max_S)
+        return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (num_seqs > g2::PfCfg<64>::MAX_SEQ_TABLE) return G2ATTN_ERR_UNSUPPORTED;
+    const long long rows = static_cast<long long>(num_blocks) * block_size;
+    if (rows > INT32_MAX || static_cast<long long>(max_blocks_per_seq) * block_size > INT32_MAX)
+        return G2ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_blocks) || !aligned16(v_blocks) || !aligned16(out) ||
+        (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens_k) & 3u))
+        return G2ATTN_ERR_MISALIGNED;
+    g2::PfParams P{};
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    P.cu_q = cu_seqlens_q;
+    P.num_seqs = num_seqs;
+    P.T = max_T;
+    P.S = max_S;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.window = window;
+    P.varlen = 1;
+    P.paged = 1;
+    P.kv_table = block_table;
+    P.kv_lens = seq_lens_k;
+    P.kv_block_shift = log2i(block_size);
+    P.kv_max_blocks = max_blocks_per_seq;
+    P.kv_num_blocks = num_blocks;
+    P.total_q = total_q;
+    const long long ub = (static_cast<long long>(total_q) / g2::PF_QPOS + num_seqs) * Hkv;
+    if (ub > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    P.num_units = static_cast<int>(ub);
+    P.max_units_per_seq_tiles = (max_T + g2::PF_QPOS - 1) / g2::PF_QPOS;
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
+    fill_poly(query_scale, softcap, P);
+    P.timeout_ns = wait_limit_ns();
+    return dispatch_prefill(d, q, k_blocks, v_blocks, total_q, rows, P,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t g2attn_decode_workspace_size(int num_seqs, int H, int d, int max_cache_len) {
     if (num_seqs <= 0 || H <= 0 || d <= 0 || max_cache_len <= 0) return 0;
     return decode_ws_bytes(num_seqs, H, d, max_cache_len, decode_chunk(num_seqs, H, max_cache_len));

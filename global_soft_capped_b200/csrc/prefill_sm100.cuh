@@ -82,6 +82,12 @@ struct PfParams {
     int q_offset;     // dense only
     int window;
     int varlen;
+    // paged K/V (varlen queries only): blocks of 2^kv_block_shift >= 128 rows
+    // located through kv_table[seq][block]; S_s = kv_lens[seq]
+    const int* kv_table;
+    const int* kv_lens;
+    int kv_block_shift, kv_max_blocks, kv_num_blocks;
+    int paged;
     int total_q;      // packed query rows (dense: B*T); lse head stride for varlen
     int num_units;
     int max_units_per_seq_tiles;  // dense: q tiles per sequence
@@ -154,9 +160,14 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, in
         seq = V.order[lo];
         const int lu = u - V.cum[lo];
         qbase = P.cu_q[seq];
-        kbase = P.cu_k[seq];
         Tq = P.cu_q[seq + 1] - qbase;
-        Sk = P.cu_k[seq + 1] - kbase;
+        if (P.paged) {
+            kbase = 0;
+            Sk = max(Tq, min(P.kv_lens[seq], P.kv_max_blocks << P.kv_block_shift));
+        } else {
+            kbase = P.cu_k[seq];
+            Sk = P.cu_k[seq + 1] - kbase;
+        }
         const int nq = (Tq + PF_QPOS - 1) / PF_QPOS;
         U.g = lu % P.Hkv;
         U.t0 = (nq - 1 - lu / P.Hkv) * PF_QPOS;
@@ -172,6 +183,15 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, in
     const int j_hi = min(U.p_max, Sk - 1);
     U.kt0 = j_lo / PF_BN;
     U.nkt = j_hi / PF_BN - U.kt0 + 1;
+}
+
+// Row of key `key` (relative to the sequence start) in the K/V tensor maps. A
+// paged cache keeps every 128-key tile inside one block (blocks >= 128 rows).
+__device__ __forceinline__ int pf_key_row(const PfParams& P, const PfUnit& U, int key) {
+    if (!P.paged) return U.kbase + key;
+    int b = P.kv_table[static_cast<size_t>(U.seq) * P.kv_max_blocks + (key >> P.kv_block_shift)];
+    b = max(0, min(b, P.kv_num_blocks - 1));
+    return (b << P.kv_block_shift) + (key & ((1 << P.kv_block_shift) - 1));
 }
 
 // Static persistent schedule: round r gives CTA c unit r*G + c (even rounds)
@@ -243,7 +263,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int ns = P.num_seqs;
         for (int s = threadIdx.x; s < ns; s += blockDim.x) {
             const int t = max(0, P.cu_q[s + 1] - P.cu_q[s]);
-            const int sk = max(t, P.cu_k[s + 1] - P.cu_k[s]);
+            const int sk = max(t, P.paged ? min(P.kv_lens[s], P.kv_max_blocks << P.kv_block_shift)
+                                          : P.cu_k[s + 1] - P.cu_k[s]);
             int w = 0;
             for (int t0 = 0; t0 < t; t0 += PF_QPOS) w += pf_tiles(t0, t, sk, P.window);
             vt.work[s] = w;
@@ -322,8 +343,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sQ + c * 16384, &tmQ, q_full, c * 64, U.qbase + U.t0, 2 * U.g);
                 // Consumption order of the MMA warp: K0, K1, V0, K2, V1, ..., V(n-1).
-                auto load_k = [&](int jj) -> bool {
-                    const int key0 = U.kbase + (U.kt0 + jj) * PF_BN;
+                auto load_k = [&](int key0) -> bool {
 #pragma unroll
                     for (int s = 0; s < C::KSL; ++s) {
                         const int slot = fill % C::NSLOT;
@@ -340,8 +360,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     }
                     return true;
                 };
-                auto load_v = [&](int jj) -> bool {
-                    const int key0 = U.kbase + (U.kt0 + jj) * PF_BN;
+                auto load_v = [&](int key0) -> bool {
 #pragma unroll
                     for (int s = 0; s < C::VSL; ++s) {
                         const int slot = fill % C::NSLOT;
@@ -358,10 +377,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     }
                     return true;
                 };
-                ok = load_k(0);
+                // Tile rows are looked up two tiles ahead (a paged cache reads
+                // the block table), so the lookup overlaps the slot waits.
+                int row0 = pf_key_row(P, U, U.kt0 * PF_BN);
+                int row1 = (U.nkt > 1) ? pf_key_row(P, U, (U.kt0 + 1) * PF_BN) : 0;
+                ok = load_k(row0);
                 for (int jj = 0; ok && jj < U.nkt; ++jj) {
-                    if (jj + 1 < U.nkt) ok = load_k(jj + 1);
-                    if (ok) ok = load_v(jj);
+                    const int row2 =
+                        (jj + 2 < U.nkt) ? pf_key_row(P, U, (U.kt0 + jj + 2) * PF_BN) : 0;
+                    if (jj + 1 < U.nkt) ok = load_k(row1);
+                    if (ok) ok = load_v(row0);
+                    row0 = row1;
+                    row1 = row2;
                 }
                 ++unit_it;
             }

@@ -98,6 +98,30 @@ G2ATTN_API int g2attn_prefill_varlen(const void* q, const void* k, const void* v
                           g2attn_stream_t stream);
 
 /*
+ * Chunked prefill over a paged KV cache: queries packed as in
+ * g2attn_prefill_varlen (cu_seqlens_q), keys and values read from fixed blocks
+ * of block_size token rows through a per-sequence block table (the
+ * block-managed caches of the serving runtimes the Guide names, "Deep Dive"
+ * item 2). Sequence s has S_s = seq_lens_k[s] keys and T_s queries at its last
+ * positions (q_offset_s = S_s - T_s).
+ *   k_blocks, v_blocks (num_blocks, block_size, Hkv, d); block_table: device
+ *   int32 [num_seqs][max_blocks_per_seq], entry b = cache block of key rows
+ *   b*block_size .. b*block_size + block_size - 1; seq_lens_k: device int32
+ *   [num_seqs] with T_s <= S_s <= max_S.
+ *   Requires block_size a power of two >= 128 (every 128-key tile then lies in
+ *   one block) and max_blocks_per_seq * block_size >= max_S. Rows of a sequence's
+ *   last block beyond S_s must hold finite values (they meet zero weights).
+ *   Table entries outside [0, num_blocks) are clamped. out, lse, limits and
+ *   errors as g2attn_prefill_varlen.
+ */
+G2ATTN_API int g2attn_prefill_paged(const void* q, const void* k_blocks, const void* v_blocks,
+                         void* out, float* lse, const int* cu_seqlens_q,
+                         const int* block_table, const int* seq_lens_k, int num_seqs,
+                         int total_q, int num_blocks, int block_size, int max_blocks_per_seq,
+                         int max_T, int max_S, int H, int Hkv, int d, float query_scale,
+                         float softcap, int window, g2attn_stream_t stream);
+
+/*
  * Bytes of device workspace g2attn_decode needs for these sizes (split-KV
  * partial results: per sequence, query head and split, a running max, a sum
  * and d accumulators, fp32). Depends only on the arguments.

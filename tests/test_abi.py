@@ -132,3 +132,17 @@ def test_ring_and_paged_reject_before_launch(lib):
     assert g2.g2attn_decode_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
     bad = list(paged); bad[18] = None        # no workspace
     assert g2.g2attn_decode_paged(*bad) == g2.G2ATTN_ERR_WORKSPACE
+
+
+def test_paged_prefill_rejects_before_launch(lib):
+    cu = ctypes.c_void_p(1 << 21)
+    base = [FAKE, FAKE, FAKE, FAKE, None, cu, cu, cu, 2, 256, 16, 256, 8, 128, 2048, 8, 4, 256,
+            0.0625, 50.0, 0, None]
+    bad = list(base); bad[11] = 64           # blocks smaller than a 128-key tile
+    assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(base); bad[11] = 384          # not a power of two
+    assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(base); bad[12] = 4            # table cannot hold max_S keys
+    assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+    bad = list(base); bad[6] = None          # no block table
+    assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
