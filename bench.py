@@ -8,7 +8,8 @@ count 4*d per visible (query, key, head) triple only. Inputs live in HBM; the
 L2 is flushed (a 512 MiB write) between timed steps, outside the timed events.
 
 Printed (rank 0, one JSON line): the contract keys, plus
-  roofline      dominant kernel (prefill_fwd_sm100<256>) vs measured bf16 peak
+  roofline      dominant kernel (prefill_fwd_sm100<256,2>, the CTA-pair kernel
+                that d = 256 runs on) vs measured bf16 peak
   cpu_baseline  the fp64 oracle on the host cores on a bounded row sample
   e2e           the same metric with pinned-host inputs and outputs copied
                 inside the timed region
@@ -78,6 +79,11 @@ def peaks():
         p = json.load(open(path))
         return p, "measured"
     return PEAKS_FALLBACK, "fallback"
+
+
+# CTA-group size of the d = 256 prefill kernel the library launches (pairs
+# unless G2ATTN_PREFILL_PAIR=0 selects the single-CTA kernel).
+KERNEL_CG = 1 if os.environ.get("G2ATTN_PREFILL_PAIR", "1").startswith("0") else 2
 
 
 def kernel_source_hash():
@@ -215,10 +221,10 @@ def run_ours(args, rank, world, dev):
     pk, pk_kind = peaks()
     avg_loc, avg_glo = sum(loc) / nsteps, sum(glo) / nsteps
     ach = (flops["local"] + flops["global"]) / ((avg_loc + avg_glo) * 1e-3) / 1e12
-    roof = {"kernel": "prefill_fwd_sm100<256>", "bound": "tensor", "achieved": round(ach, 2),
+    roof = {"kernel": f"prefill_fwd_sm100<256,{KERNEL_CG}>", "bound": "tensor", "achieved": round(ach, 2),
             "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
             "peak_kind": f"{pk_kind} bf16 dense (burst; kernel timed alone)",
-            "traffic": ncu_traffic("prefill_fwd_sm100<256>/2b_pair", 1.0),
+            "traffic": ncu_traffic(f"prefill_fwd_sm100<256,{KERNEL_CG}>/2b_pair", 1.0),
             "traffic_unit": "bytes per launch (mean of the local and global launch)",
             "algorithmic": "4*d*H*B per visible (query,key) pair; 0.4811 TFLOP per step "
                            "(two launches); compulsory bytes Q+K+V+O = 100663296 per launch"}

@@ -105,32 +105,79 @@ void fill_poly(float query_scale, float softcap, g2::PfParams& P) {
     }
 }
 
-template <int D>
+// CG = 2 launches clusters of two CTAs (one unit of 128 query positions per
+// pair); the grid holds as many pairs as can be resident at once.
+template <int D, int CG>
 int launch_prefill(const void* q, const void* k, const void* v, long long total_q,
                    long long total_k, g2::PfParams& P, cudaStream_t stream) {
-    using C = g2::PfCfg<D>;
+    using C = g2::PfCfg<D, CG>;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, D, total_q, P.H, g2::PF_QPOS, 2) ||
-        !make_map(&mk, k, D, total_k, P.Hkv, g2::PF_BN, 1) ||
+        !make_map(&mk, k, D, total_k, P.Hkv, C::KROWS, 1) ||
         !make_map(&mv, v, D, total_k, P.Hkv, C::VROWS, 1))
         return G2ATTN_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return G2ATTN_ERR_CUDA;
-    auto kern = g2::prefill_fwd_sm100<D>;
+    auto kern = g2::prefill_fwd_sm100<D, CG>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return G2ATTN_ERR_CUDA;
-    const int grid = P.num_units < sms ? P.num_units : sms;
-    kern<<<grid, g2::PF_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, P);
+    if (CG == 1) {
+        const int grid = P.num_units < sms ? P.num_units : sms;
+        kern<<<grid, g2::PF_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, P);
+        return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(g2::PF_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static int pairs_resident = -1;  // per process: one device type
+    if (pairs_resident < 0) {
+        cfg.gridDim = dim3(CG * (sms / CG), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0)
+            return G2ATTN_ERR_CUDA;
+        pairs_resident = n;
+    }
+    const int pairs = P.num_units < pairs_resident ? P.num_units : pairs_resident;
+    cfg.gridDim = dim3(CG * pairs, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, P) != cudaSuccess) return G2ATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+}
+
+// d = 256 runs on CTA pairs unless G2ATTN_PREFILL_PAIR=0 selects the
+// single-CTA kernel (read once per process).
+bool use_pairs() {
+    static bool v = [] {
+        const char* e = getenv("G2ATTN_PREFILL_PAIR");
+        return !(e != nullptr && e[0] == '0');
+    }();
+    return v;
 }
 
 int dispatch_prefill(int d, const void* q, const void* k, const void* v, long long tq,
                      long long tk, g2::PfParams& P, cudaStream_t st) {
     switch (d) {
-        case 64: return launch_prefill<64>(q, k, v, tq, tk, P, st);
-        case 128: return launch_prefill<128>(q, k, v, tq, tk, P, st);
-        case 256: return launch_prefill<256>(q, k, v, tq, tk, P, st);
+        case 64: return launch_prefill<64, 1>(q, k, v, tq, tk, P, st);
+        case 128: return launch_prefill<128, 1>(q, k, v, tq, tk, P, st);
+        case 256:
+            if (use_pairs()) {
+                // units of 128 query positions (varlen: the kernel counts them
+                // itself; the single-CTA count stays a valid upper bound)
+                if (!P.varlen) {
+                    P.max_units_per_seq_tiles = (P.T + 2 * g2::PF_QPOS - 1) / (2 * g2::PF_QPOS);
+                    P.num_units = P.max_units_per_seq_tiles * P.num_seqs * P.Hkv;
+                }
+                return launch_prefill<256, 2>(q, k, v, tq, tk, P, st);
+            }
+            return launch_prefill<256, 1>(q, k, v, tq, tk, P, st);
         default: return G2ATTN_ERR_UNSUPPORTED;
     }
 }

@@ -53,12 +53,19 @@ constexpr float kTanhC2 = 2.0f / 15.0f;
 constexpr float kTanhC3 = -17.0f / 315.0f;
 constexpr float PF_POLY_U_MAX = 0.25f;  // |x / C| bound of the series path
 
-template <int D>
+// CG = 1: one CTA per unit of 64 query positions. CG = 2 (d = 256 only): a CTA
+// pair per unit of 128 positions, 64 per CTA; each CTA stages half of every
+// K tile (64 of its 128 keys) and half of every V tile (128 of its 256
+// d-columns), and the even CTA issues M = 256 UMMAs over both halves.
+template <int D, int CG = 1>
 struct PfCfg {
+    static_assert(CG == 1 || (CG == 2 && D == 256), "CTA pairs are built for d = 256");
     static constexpr int SLOT_BYTES = (D == 64) ? 16384 : 32768;
-    static constexpr int KCOLS = SLOT_BYTES / (PF_BN * 2);  // d-columns per K slot (64 or 128)
+    static constexpr int KROWS = PF_BN / CG;                // keys of a K tile staged by this CTA
+    static constexpr int KCOLS = SLOT_BYTES / (KROWS * 2);  // d-columns per K slot
     static constexpr int KSL = D / KCOLS;                   // K slots per KV tile
-    static constexpr int VROWS = SLOT_BYTES / (D * 2);      // keys per V slot
+    static constexpr int VCOLS = D / CG;                    // d-columns of V staged by this CTA
+    static constexpr int VROWS = SLOT_BYTES / (VCOLS * 2);  // keys per V slot
     static constexpr int VSL = PF_BN / VROWS;               // V slots per KV tile
     static constexpr int NSLOT = (D == 64) ? 8 : (D == 128 ? 5 : 4);
     static constexpr int Q_BYTES = PF_BM * D * 2;
@@ -67,7 +74,8 @@ struct PfCfg {
     static constexpr int SMEM_TILES = Q_BYTES + NSLOT * SLOT_BYTES;
     static constexpr int CTRL_BYTES = 1024 + 2 * PF_NSPLIT * 128 * 4 + PF_NSPLIT * 128 * 2 * 4;
     static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + CTRL_BYTES + VL_BYTES;
-    static_assert(KCOLS % 64 == 0 && VROWS % 16 == 0, "tile shapes");
+    static_assert(KCOLS % 64 == 0 && KCOLS <= D && VROWS % 16 == 0 && VROWS <= PF_BN,
+                  "tile shapes");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -135,8 +143,14 @@ __device__ __forceinline__ int pf_tiles(int t0, int T, int S, int window) {
 
 // Work unit u of the launch. Dense: query tiles in descending order (longest
 // rows first), then batch, then KV head. Varlen: sequences in rank order, each
-// with its query tiles descending, then KV head.
-__device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, int u, PfUnit& U) {
+// with its query tiles descending, then KV head. A unit covers 64 * CG query
+// positions; the KV tile range is that of the whole unit, and CTA `rank` of a
+// pair takes the rows of positions t0 + 64*rank .. + 63 (tvalid may be <= 0
+// for the odd CTA at the end of a sequence: it then stores nothing).
+template <int CG = 1>
+__device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, int u, PfUnit& U,
+                                        int rank = 0) {
+    constexpr int QT = PF_QPOS * CG;
     int seq, Tq, Sk, qbase, kbase;
     if (!P.varlen) {
         const int BG = P.num_seqs * P.Hkv;
@@ -149,7 +163,7 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, in
         Sk = P.S;
         qbase = seq * P.T;
         kbase = seq * P.S;
-        U.t0 = qt * PF_QPOS;
+        U.t0 = qt * QT;
         U.qoff = P.q_offset;
     } else {
         int lo = 0, hi = P.num_seqs - 1;  // largest rank with cum[rank] <= u
@@ -168,21 +182,26 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, in
             kbase = P.cu_k[seq];
             Sk = P.cu_k[seq + 1] - kbase;
         }
-        const int nq = (Tq + PF_QPOS - 1) / PF_QPOS;
+        const int nq = (Tq + QT - 1) / QT;
         U.g = lu % P.Hkv;
-        U.t0 = (nq - 1 - lu / P.Hkv) * PF_QPOS;
+        U.t0 = (nq - 1 - lu / P.Hkv) * QT;
         U.qoff = Sk - Tq;
     }
     U.seq = seq;
     U.qbase = qbase;
     U.kbase = kbase;
+    {  // KV tiles of the whole unit
+        const int tv = min(QT, Tq - U.t0);
+        const int p_lo = U.t0 + U.qoff, p_hi = U.t0 + tv - 1 + U.qoff;
+        const int j_lo = P.window > 0 ? max(0, p_lo - P.window + 1) : 0;
+        const int j_hi = min(p_hi, Sk - 1);
+        U.kt0 = j_lo / PF_BN;
+        U.nkt = j_hi / PF_BN - U.kt0 + 1;
+    }
+    U.t0 += PF_QPOS * rank;  // this CTA's rows
     U.tvalid = min(PF_QPOS, Tq - U.t0);
     U.p_min = U.t0 + U.qoff;
-    U.p_max = U.t0 + U.tvalid - 1 + U.qoff;
-    const int j_lo = P.window > 0 ? max(0, U.p_min - P.window + 1) : 0;
-    const int j_hi = min(U.p_max, Sk - 1);
-    U.kt0 = j_lo / PF_BN;
-    U.nkt = j_hi / PF_BN - U.kt0 + 1;
+    U.p_max = U.p_min + max(U.tvalid, 1) - 1;
 }
 
 // Row of key `key` (relative to the sequence start) in the K/V tensor maps. A
@@ -200,12 +219,13 @@ __device__ __forceinline__ int pf_sched(int r, int c, int G) {
     return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-template <int D>
+template <int D, int CG = 1>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PfParams P) {
-    using C = PfCfg<D>;
+    using C = PfCfg<D, CG>;
+    constexpr bool PAIR = CG == 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -243,12 +263,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         mbar_init(q_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], PF_SOFTMAX_THREADS / 32);
+            mbar_init(&p_full[i], CG * PF_SOFTMAX_THREADS / 32);
             mbar_init(&o_done[i], 1);
         }
         // softmax-side barriers take one arrival per warp (elected lane, after
-        // __syncwarp orders the whole warp's prior writes before it)
-        mbar_init(o_free, PF_SOFTMAX_THREADS / 32);
+        // __syncwarp orders the whole warp's prior writes before it); a pair
+        // counts the warps of both CTAs on the even CTA's p_full and o_free
+        mbar_init(o_free, CG * PF_SOFTMAX_THREADS / 32);
         for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], PF_NSPLIT);
         for (int i = 0; i < 4; ++i) mbar_init(&sbar[i], PF_NSPLIT);
         mbar_init(drain, 1);
@@ -283,7 +304,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         for (int r = threadIdx.x; r < ns; r += blockDim.x) {
             const int s = vt.order[r];
             const int t = max(0, P.cu_q[s + 1] - P.cu_q[s]);
-            vt.cum[r] = P.Hkv * ((t + PF_QPOS - 1) / PF_QPOS);
+            vt.cum[r] = P.Hkv * ((t + CG * PF_QPOS - 1) / (CG * PF_QPOS));
         }
         __syncthreads();
         if (warp == 0) {  // exclusive scan, 32 entries at a time
@@ -304,8 +325,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
     }
     if (warp == PF_WARP_MMA) {
-        tmem_alloc(tmem_holder, PF_TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(tmem_holder, PF_TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_holder, PF_TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     if (warp == PF_WARP_PRODUCER && lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -313,16 +339,34 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         tma_prefetch_desc(&tmV);
     }
     tc_fence_before();
-    __syncthreads();
+    // A pair: both CTAs' barriers are initialised before either CTA's copies,
+    // arrivals or commits can reach the other.
+    if constexpr (PAIR) {
+        __syncwarp();
+        cluster_sync_all();
+    } else {
+        __syncthreads();
+    }
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int G = gridDim.x;
-    const int cta = blockIdx.x;
+    // G units run in parallel (CTAs, or CTA pairs); this CTA (pair) is `cta`.
+    const int G = PAIR ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+    const int cta = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+    const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+    const bool leader = rank == 0;  // issues the UMMAs and owns the pair's shared barriers
     const int num_units = P.varlen ? min(P.num_units, vt.cum[P.num_seqs]) : P.num_units;
     const uint64_t lim = P.timeout_ns;
+    // Cluster-window addresses of the even CTA's barriers that both CTAs of a
+    // pair signal (data arrival, P ready, O read).
+    const uint32_t l_q_full = PAIR ? mapa_shared(smem_u32(q_full), 0) : 0u;
+    const uint32_t l_o_free = PAIR ? mapa_shared(smem_u32(o_free), 0) : 0u;
 
     if (warp == PF_WARP_PRODUCER) {
         // ------------------------------------------------------------ producer
+        // A pair: each CTA copies its own share into its own shared memory and
+        // counts the bytes on the even CTA's barrier, which the even CTA's
+        // producer arms for both shares. Empty barriers are local (the even
+        // CTA's commits reach both CTAs).
         if (lane == 0) {
             uint32_t fill = 0;  // slot fills issued so far
             int unit_it = 0;
@@ -332,49 +376,62 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int u = pf_sched(r, cta, G);
                 if (u >= num_units) continue;
                 PfUnit U;
-                pf_unit(P, vt, u, U);
+                pf_unit<CG>(P, vt, u, U, rank);
                 if (unit_it > 0) {
-                    ok = mbar_wait(q_empty, (unit_it - 1) & 1, abort_flag, lim, SITE_PROD_Q_EMPTY);
+                    ok = mbar_wait(q_empty, (unit_it - 1) & 1, abort_flag, lim,
+                                         SITE_PROD_Q_EMPTY);
                     if (!ok) break;
                 }
-                mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+                if (leader) mbar_arrive_expect_tx(q_full, CG * C::Q_BYTES);
                 ++q_armed;
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_3d(sQ + c * 16384, &tmQ, q_full, c * 64, U.qbase + U.t0, 2 * U.g);
+                for (int c = 0; c < D / 64; ++c) {
+                    if constexpr (PAIR)
+                        tma_load_3d_pair(sQ + c * 16384, &tmQ, l_q_full, c * 64, U.qbase + U.t0,
+                                         2 * U.g);
+                    else
+                        tma_load_3d(sQ + c * 16384, &tmQ, q_full, c * 64, U.qbase + U.t0, 2 * U.g);
+                }
                 // Consumption order of the MMA warp: K0, K1, V0, K2, V1, ..., V(n-1).
-                auto load_k = [&](int key0) -> bool {
+                // Slot `slot` of a fill: wait until it is free, arm its barrier,
+                // then copy `nbox` boxes of 64 d-columns.
+                auto fill_slot = [&](const CUtensorMap* map, int nbox, int box_bytes, int col0,
+                                     int row) -> bool {
+                    const int slot = fill % C::NSLOT;
+                    if (!mbar_wait(&slot_empty[slot], ((fill / C::NSLOT) & 1) ^ 1, abort_flag,
+                                         lim, SITE_PROD_SLOT_EMPTY))
+                        return false;
+                    if (leader) mbar_arrive_expect_tx(&slot_full[slot], CG * C::SLOT_BYTES);
+                    uint8_t* dst = sSlots + slot * C::SLOT_BYTES;
 #pragma unroll
-                    for (int s = 0; s < C::KSL; ++s) {
-                        const int slot = fill % C::NSLOT;
-                        if (!mbar_wait(&slot_empty[slot], ((fill / C::NSLOT) & 1) ^ 1, abort_flag,
-                                       lim, SITE_PROD_SLOT_EMPTY))
-                            return false;
-                        mbar_arrive_expect_tx(&slot_full[slot], C::SLOT_BYTES);
-                        uint8_t* dst = sSlots + slot * C::SLOT_BYTES;
-#pragma unroll
-                        for (int b = 0; b < C::KCOLS / 64; ++b)
-                            tma_load_3d(dst + b * (PF_BN * 128), &tmK, &slot_full[slot],
-                                        s * C::KCOLS + b * 64, key0, U.g);
-                        ++fill;
+                    for (int b = 0; b < nbox; ++b) {
+                        if constexpr (PAIR)
+                            tma_load_3d_pair(dst + b * box_bytes, map,
+                                             mapa_shared(smem_u32(&slot_full[slot]), 0),
+                                             col0 + b * 64, row, U.g);
+                        else
+                            tma_load_3d(dst + b * box_bytes, map, &slot_full[slot], col0 + b * 64,
+                                        row, U.g);
                     }
+                    ++fill;
                     return true;
                 };
+                // K: this CTA's KROWS keys of the tile, KCOLS d-columns per slot
+                auto load_k = [&](int key0) -> bool {
+#pragma unroll
+                    for (int s = 0; s < C::KSL; ++s)
+                        if (!fill_slot(&tmK, C::KCOLS / 64, C::KROWS * 128, s * C::KCOLS,
+                                       key0 + rank * C::KROWS))
+                            return false;
+                    return true;
+                };
+                // V: VROWS keys per slot, this CTA's VCOLS d-columns
                 auto load_v = [&](int key0) -> bool {
 #pragma unroll
-                    for (int s = 0; s < C::VSL; ++s) {
-                        const int slot = fill % C::NSLOT;
-                        if (!mbar_wait(&slot_empty[slot], ((fill / C::NSLOT) & 1) ^ 1, abort_flag,
-                                       lim, SITE_PROD_SLOT_EMPTY))
+                    for (int s = 0; s < C::VSL; ++s)
+                        if (!fill_slot(&tmV, C::VCOLS / 64, C::VROWS * 128, rank * C::VCOLS,
+                                       key0 + s * C::VROWS))
                             return false;
-                        mbar_arrive_expect_tx(&slot_full[slot], C::SLOT_BYTES);
-                        uint8_t* dst = sSlots + slot * C::SLOT_BYTES;
-#pragma unroll
-                        for (int b = 0; b < D / 64; ++b)
-                            tma_load_3d(dst + b * (C::VROWS * 128), &tmV, &slot_full[slot], b * 64,
-                                        key0 + s * C::VROWS, U.g);
-                        ++fill;
-                    }
                     return true;
                 };
                 // Tile rows are looked up two tiles ahead (a paged cache reads
@@ -392,24 +449,42 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
                 ++unit_it;
             }
-            // Drain: every copy this thread issued lands before the CTA exits.
-            const uint32_t last = fill < (uint32_t)C::NSLOT ? fill : (uint32_t)C::NSLOT;
-            for (uint32_t i = 0; i < last; ++i) {
-                const uint32_t f = fill - 1 - i;
-                mbar_wait_drain(&slot_full[f % C::NSLOT], (f / C::NSLOT) & 1, lim);
+            // Drain: every copy issued lands before the CTA exits. The full
+            // barriers of a pair live in the even CTA and count both CTAs'
+            // copies; the odd CTA's copies are drained there, before the
+            // cluster barrier at the end of the kernel.
+            if (leader) {
+                const uint32_t last = fill < (uint32_t)C::NSLOT ? fill : (uint32_t)C::NSLOT;
+                for (uint32_t i = 0; i < last; ++i) {
+                    const uint32_t f = fill - 1 - i;
+                    mbar_wait_drain(&slot_full[f % C::NSLOT], (f / C::NSLOT) & 1, lim);
+                }
+                if (q_armed > 0) mbar_wait_drain(q_full, (q_armed - 1) & 1, lim);
             }
-            if (q_armed > 0) mbar_wait_drain(q_full, (q_armed - 1) & 1, lim);
+            if constexpr (PAIR) {
+                // The even CTA's commits reach this CTA's empty barriers: wait
+                // for the last of them so none lands after the pair has left.
+                const uint32_t last = fill < (uint32_t)C::NSLOT ? fill : (uint32_t)C::NSLOT;
+                for (uint32_t i = 0; i < last; ++i) {
+                    const uint32_t f = fill - 1 - i;
+                    mbar_wait_drain(&slot_empty[f % C::NSLOT], (f / C::NSLOT) & 1, lim);
+                }
+                if (q_armed > 0) mbar_wait_drain(q_empty, (q_armed - 1) & 1, lim);
+            }
         }
         __syncwarp();
     } else if (warp == PF_WARP_MMA) {
         // ------------------------------------------------------------ UMMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16(PF_BM, PF_BN, false);
-            constexpr uint32_t IDESC_O = idesc_bf16(PF_BM, D, true);
+        // In a pair the even CTA issues for both (M = 256: its 128 rows, then
+        // the odd CTA's); the odd CTA's issuer warp only holds the allocation.
+        if (lane == 0 && leader) {
+            constexpr uint32_t IDESC_S = idesc_bf16(PF_BM * CG, PF_BN, false);
+            constexpr uint32_t IDESC_O = idesc_bf16(PF_BM * CG, D, true);
             constexpr uint32_t HI = sdesc_hi(1024);  // SBO 1024 B (8 rows x 128 B)
             // Q (A of S = Q K^T): K-major, 64-column chunks of 16 KB, k-step = 32 B
             const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
-            // ring slot s: K-major K (LBO unused) or MN-major V (LBO = VROWS*128 B)
+            // ring slot s: K-major K (LBO unused) or MN-major V (LBO = VROWS*128 B);
+            // a pair's descriptors address the same offsets in both CTAs
             const uint32_t slot_lo0 = sdesc_lo(smem_u32(sSlots), 16);
             const uint32_t slot_lo0_v = sdesc_lo(smem_u32(sSlots), C::VROWS * 128);
             constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
@@ -419,6 +494,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             int unit_it = 0;
             bool ok = true;
 
+            // completion of the UMMAs issued so far (both CTAs' barriers for a pair)
+            auto commit = [&](uint64_t* bar) {
+                if constexpr (PAIR) umma_commit_pair(bar); else umma_commit(bar);
+            };
             auto issue_s = [&](uint32_t gt) -> bool {
                 const uint32_t buf = gt & 1;
                 // S(gt) overwrites P(gt-2) in the same TMEM columns. PV(gt-2) was
@@ -427,7 +506,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint32_t d_tmem = tmem + PF_S_COL0 + buf * PF_BN;
 #pragma unroll
                 for (int s = 0; s < C::KSL; ++s) {
-                    if (!mbar_wait(&slot_full[slot], phase, abort_flag, lim, SITE_MMA_SLOT_FULL))
+                    if (!mbar_wait(&slot_full[slot], phase, abort_flag, lim,
+                                         SITE_MMA_SLOT_FULL))
                         return false;
                     tc_fence_after();
                     const uint32_t k_lo = slot_lo0 + slot * SLOT_STEP;
@@ -435,13 +515,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     for (int kk = 0; kk < C::KCOLS / 16; ++kk) {
                         const int dcol = s * C::KCOLS + kk * 16;  // Q column of this k-step
                         const uint32_t a_lo = q_lo + (dcol / 64) * (16384 >> 4) + ((dcol % 64) / 16) * 2;
-                        const uint32_t b_lo = k_lo + (kk / 4) * ((PF_BN * 128) >> 4) + (kk % 4) * 2;
-                        umma_ss_lh(d_tmem, a_lo, b_lo, HI, IDESC_S, (s | kk) != 0);
+                        const uint32_t b_lo = k_lo + (kk / 4) * ((C::KROWS * 128) >> 4) + (kk % 4) * 2;
+                        if constexpr (PAIR)
+                            umma_ss_lh_pair(d_tmem, a_lo, b_lo, HI, IDESC_S, (s | kk) != 0);
+                        else
+                            umma_ss_lh(d_tmem, a_lo, b_lo, HI, IDESC_S, (s | kk) != 0);
                     }
-                    umma_commit(&slot_empty[slot]);
+                    commit(&slot_empty[slot]);
                     if (++slot == C::NSLOT) { slot = 0; phase ^= 1u; }
                 }
-                umma_commit(&s_full[buf]);
+                commit(&s_full[buf]);
                 return true;
             };
             auto issue_pv = [&](uint32_t gt, bool first) -> bool {
@@ -449,20 +532,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint32_t p_tmem = tmem + PF_S_COL0 + buf * PF_BN;
 #pragma unroll
                 for (int s = 0; s < C::VSL; ++s) {
-                    if (!mbar_wait(&slot_full[slot], phase, abort_flag, lim, SITE_MMA_SLOT_FULL))
+                    if (!mbar_wait(&slot_full[slot], phase, abort_flag, lim,
+                                         SITE_MMA_SLOT_FULL))
                         return false;
                     tc_fence_after();
                     const uint32_t v_lo = slot_lo0_v + slot * SLOT_STEP;
 #pragma unroll
                     for (int kk = 0; kk < C::VROWS / 16; ++kk) {
                         const uint32_t a = p_tmem + (s * C::VROWS + kk * 16) / 2;
-                        umma_ts_lh(tmem, a, v_lo + kk * ((16 * 128) >> 4), HI, IDESC_O,
-                                   (first && s == 0 && kk == 0) ? 0u : 1u);
+                        const uint32_t acc = (first && s == 0 && kk == 0) ? 0u : 1u;
+                        if constexpr (PAIR)
+                            umma_ts_lh_pair(tmem, a, v_lo + kk * ((16 * 128) >> 4), HI, IDESC_O, acc);
+                        else
+                            umma_ts_lh(tmem, a, v_lo + kk * ((16 * 128) >> 4), HI, IDESC_O, acc);
                     }
-                    umma_commit(&slot_empty[slot]);
+                    commit(&slot_empty[slot]);
                     if (++slot == C::NSLOT) { slot = 0; phase ^= 1u; }
                 }
-                umma_commit(&o_done[buf]);
+                commit(&o_done[buf]);
                 return true;
             };
 
@@ -470,7 +557,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int u = pf_sched(r, cta, G);
                 if (u >= num_units) continue;
                 PfUnit U;
-                pf_unit(P, vt, u, U);
+                pf_unit<CG>(P, vt, u, U, rank);
                 ok = mbar_wait(q_full, unit_it & 1, abort_flag, lim, SITE_MMA_Q_FULL);
                 if (!ok) break;
                 tc_fence_after();
@@ -481,14 +568,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         ok = issue_s(gt + 1);
                         if (!ok) break;
                     } else {
-                        umma_commit(q_empty);  // last S of the unit issued: Q reusable
+                        commit(q_empty);  // last S of the unit issued: Q reusable
                     }
                     ok = mbar_wait(&p_full[gt & 1], (gt >> 1) & 1, abort_flag, lim,
-                                   SITE_MMA_P_FULL);
+                                         SITE_MMA_P_FULL);
                     if (!ok) break;
                     if (jj == 0 && unit_it > 0) {
                         ok = mbar_wait(o_free, (unit_it - 1) & 1, abort_flag, lim,
-                                       SITE_MMA_O_FREE);
+                                             SITE_MMA_O_FREE);
                         if (!ok) break;
                     }
                     tc_fence_after();
@@ -497,8 +584,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 tile += U.nkt;
                 ++unit_it;
             }
-            // Drain: all issued UMMAs complete before TMEM is released.
-            umma_commit(drain);
+            // Drain: all issued UMMAs complete before TMEM is released (a
+            // pair: signalled in this CTA only, never into the other CTA
+            // after it may have left).
+            if constexpr (PAIR) umma_commit_pair_local(drain); else umma_commit(drain);
             mbar_wait_drain(drain, 0, lim);
         }
         __syncwarp();
@@ -535,7 +624,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const int u = pf_sched(rr, cta, G);
             if (u >= num_units) continue;
             PfUnit U;
-            pf_unit(P, vt, u, U);
+            pf_unit<CG>(P, vt, u, U, rank);
             const int p = U.p_min + pr;  // absolute query position of this row
             float m_ref = -INFINITY;     // log2-domain reference max of the row
             float l = 0.f;               // this part's sum of fp32 weights (for lse)
@@ -634,8 +723,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const bool need = (m_ref != -INFINITY) && (m_new > m_ref + PF_RESCALE_LOG2);
                 if (__any_sync(0xffffffffu, need)) {
                     // O holds PV(0..gt-1) relative to m_ref: scale this part to m_new.
-                    ok = mbar_wait(&o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, abort_flag, lim,
-                                   SITE_SM_O_DONE);
+                    ok = mbar_wait(&o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, abort_flag,
+                                         lim, SITE_SM_O_DONE);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
@@ -717,7 +806,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[buf]);
+                if (lane == 0) {
+                    if constexpr (PAIR)
+                        mbar_arrive_cluster(mapa_shared(smem_u32(&p_full[buf]), 0));
+                    else
+                        mbar_arrive(&p_full[buf]);
+                }
             }
             if (!ok) break;
             // ---- epilogue: O / lr -> bf16, lse
@@ -774,17 +868,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(o_free);
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(l_o_free); else mbar_arrive(o_free);
+            }
             tile += U.nkt;
             ++unit_it;
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    // A pair leaves together: no copy, arrival or UMMA of one CTA may still
+    // reach the other's shared or tensor memory after this barrier.
+    if constexpr (PAIR) {
+        __syncwarp();
+        cluster_sync_all();
+    } else {
+        __syncthreads();
+    }
     if (warp == PF_WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem, PF_TMEM_COLS);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, PF_TMEM_COLS);
+        else tmem_dealloc(tmem, PF_TMEM_COLS);
     }
 }
 

@@ -65,6 +65,11 @@ typedef enum {
  *   lse (B, H, T)         fp32 natural-log log-sum-exp of the capped logits
  * Requires B, T, S >= 1, 0 <= q_offset, q_offset + T <= S, window >= 0,
  * finite query_scale, finite softcap >= 0.
+ * Kernel choice (all three prefill calls): d = 256 launches clusters of two
+ * CTAs sharing each K/V tile (tcgen05 .cta_group::2); the environment variable
+ * G2ATTN_PREFILL_PAIR=0, read once per process, selects the single-CTA kernel
+ * instead. d = 64 and 128 always use the single-CTA kernel. Both kernels
+ * compute the same result.
  * Source: Gemma 2 card, "Method" (attention_layer pseudo-code: queries
  * (B,T,H,d), keys/values (B,S,K,d), K = H/2, cap 50, causal and 4096 window).
  */
