@@ -13,8 +13,10 @@ Functions (each follows the Gemma 2 card's per-layer attention pseudo-code,
 * :func:`row_detail`  one row's masked capped logits and softmax weights
 * :func:`decode`      one query per sequence at position L-1 of its cache
 * :func:`varlen`      packed sequences, each a dense layer with q_offset = S_i - T_i
+* :func:`attn_bwd`    gradients of the dense layer (dq, dk, dv) for an upstream dout
 
-Parity of every function is pinned by ``tests/test_oracle_pins.py``.
+Parity of every function is pinned by ``tests/test_oracle_pins.py`` (the
+gradients by ``tests/test_oracle_backward_pins.py``).
 """
 from __future__ import annotations
 
@@ -58,6 +60,8 @@ def _load():
         lib.g2ref_attn_rows.restype = ctypes.c_int
         lib.g2ref_row_detail.argtypes = [P, P, P, P, I64, I64, I64] + [I64] * 7 + [D, D, I64]
         lib.g2ref_row_detail.restype = ctypes.c_int
+        lib.g2ref_attn_bwd.argtypes = [P] * 7 + [I64] * 7 + [D, D, I64]
+        lib.g2ref_attn_bwd.restype = ctypes.c_int
         lib.g2ref_set_threads.argtypes = [ctypes.c_int]
         lib.g2ref_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -132,6 +136,28 @@ def row_detail(q, k, b, i, h, q_offset=0, query_scale=1.0, softcap=50.0, window=
     if rc != 0:
         raise ValueError("g2ref_row_detail rejected its arguments")
     return s, w
+
+
+def attn_bwd(q, k, v, dout, q_offset=0, query_scale=1.0, softcap=50.0, window=0):
+    """Gradients of :func:`attn` for the upstream gradient dout (B,T,H,d).
+
+    Returns (dq (B,T,H,d), dk (B,S,Hkv,d), dv (B,S,Hkv,d)) as float64: the
+    chain rule through the mix, the softmax, the soft-cap (derivative
+    1 - tanh^2, "Gemma 2 Guide", Deep Dive item 1) and the scaled dot product.
+    """
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, T, H, d = qb.shape
+    S, Hkv = kb.shape[1], kb.shape[2]
+    assert kb.shape == (B, S, Hkv, d) and vb.shape == kb.shape and gb.shape == qb.shape
+    dq = np.empty((B, T, H, d), np.float64)
+    dk = np.empty((B, S, Hkv, d), np.float64)
+    dv = np.empty((B, S, Hkv, d), np.float64)
+    rc = _load().g2ref_attn_bwd(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, T, S, H, Hkv, d, int(q_offset), float(query_scale),
+                                float(softcap), int(window))
+    if rc != 0:
+        raise ValueError("g2ref_attn_bwd rejected its arguments")
+    return dq, dk, dv
 
 
 def decode(q, k_cache, v_cache, cu_seqlens_k, query_scale=1.0, softcap=50.0, window=0,

@@ -1,5 +1,6 @@
 /*
- * g2ref.c -- fp64 CPU oracle for the Gemma 2 per-layer attention forward.
+ * g2ref.c -- fp64 CPU oracle for the Gemma 2 per-layer attention forward
+ * and its gradients.
  *
  * TEST INFRASTRUCTURE (see g2ref.h): loaded only by the tests, the smoke
  * check and the benchmark's CPU-baseline leg. Plain loops, no blocking, no
@@ -177,6 +178,84 @@ int g2ref_row_detail(const uint16_t* q, const uint16_t* k,
             s, w, NULL, NULL);
     free(qs);
     return 0;
+}
+
+/* Gradients (see g2ref.h). Each (b, g) owns dk[b,:,g,:] and dv[b,:,g,:] and
+ * the dq rows of its heads, so the parallel loop runs over (b, g). */
+int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint16_t* dout, double* dq, double* dk, double* dv,
+                   int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                   int64_t q_offset, double query_scale, double softcap, int64_t window) {
+    if (check_args(B, T, S, H, Hkv, d, q_offset, softcap, window)) return -1;
+    const int64_t group = H / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)(B * T * H * d));
+    memset(dk, 0, sizeof(double) * (size_t)(B * S * Hkv * d));
+    memset(dv, 0, sizeof(double) * (size_t)(B * S * Hkv * d));
+    int err = 0;
+#pragma omp parallel
+    {
+        double* qs = (double*)malloc(sizeof(double) * (size_t)d);
+        double* s = (double*)malloc(sizeof(double) * (size_t)S);
+        double* w = (double*)malloc(sizeof(double) * (size_t)S);
+        double* x = (double*)malloc(sizeof(double) * (size_t)S);
+        double* out_row = (double*)malloc(sizeof(double) * (size_t)d);
+        if (!qs || !s || !w || !x || !out_row) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bg = 0; bg < B * Hkv; ++bg) {
+                const int64_t b = bg / Hkv, g = bg % Hkv;
+                for (int64_t h = g * group; h < (g + 1) * group; ++h) {
+                    for (int64_t i = 0; i < T; ++i) {
+                        /* forward of this row: s, w (and qs = query_scale * q) */
+                        one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale,
+                                softcap, window, qs, s, w, out_row, NULL);
+                        const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
+                        /* dw_j = dout . v_j, and D = sum_j w_j dw_j */
+                        double D = 0.0;
+                        for (int64_t j = 0; j < S; ++j) {
+                            x[j] = 0.0;
+                            if (w[j] == 0.0) continue;
+                            const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
+                            double dw = 0.0;
+                            for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
+                            x[j] = dw; /* holds dw_j until ds_j is formed */
+                            D += w[j] * dw;
+                        }
+                        double* dqrow = dq + ((b * T + i) * H + h) * d;
+                        for (int64_t j = 0; j < S; ++j) {
+                            if (w[j] == 0.0) continue;
+                            const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
+                            /* softmax: ds_j = w_j (dw_j - D) */
+                            double dx = w[j] * (x[j] - D);
+                            /* cap: d(C tanh(x/C))/dx = 1 - tanh^2(x/C), with x the scaled logit */
+                            if (softcap > 0.0) {
+                                double xl = 0.0;
+                                for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
+                                const double t = tanh(xl / softcap);
+                                dx *= 1.0 - t * t;
+                            }
+                            /* x = (query_scale q) . k */
+                            double* dkrow = dk + ((b * S + j) * Hkv + g) * d;
+                            double* dvrow = dv + ((b * S + j) * Hkv + g) * d;
+                            for (int64_t c = 0; c < d; ++c) {
+                                dqrow[c] += query_scale * dx * widen(krow[c]);
+                                dkrow[c] += dx * qs[c];
+                                dvrow[c] += w[j] * widen(dorow[c]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(qs);
+        free(s);
+        free(w);
+        free(x);
+        free(out_row);
+    }
+    return err ? -1 : 0;
 }
 
 void g2ref_set_threads(int n) {

@@ -1,5 +1,6 @@
 /*
- * g2ref.h -- fp64 CPU oracle for the Gemma 2 per-layer attention forward.
+ * g2ref.h -- fp64 CPU oracle for the Gemma 2 per-layer attention forward
+ * and its gradients.
  *
  * TEST INFRASTRUCTURE. This is the slow, plain reference that the CUDA
  * library is checked against. Only the test suite, the package smoke check
@@ -51,6 +52,22 @@ int g2ref_row_detail(const uint16_t* q, const uint16_t* k,
                      double* s, double* w, int64_t b, int64_t i, int64_t h,
                      int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
                      int64_t q_offset, double query_scale, double softcap, int64_t window);
+
+/* Gradients of the dense layer above for an upstream gradient dout (B,T,H,d),
+ * the chain rule applied to the same definition step by step:
+ *   dw_j  = dout[b,i,h,:] . v[b,j,g,:]          (out = sum_j w_j v_j)
+ *   ds_j  = w_j (dw_j - sum_k w_k dw_k)          (softmax)
+ *   dx_j  = ds_j (1 - tanh^2(x_j / softcap))     (cap; "Gemma 2 Guide", Deep Dive
+ *                                                  item 1; dx_j = ds_j without cap)
+ *   dq[b,i,h,:] += query_scale sum_j dx_j k[b,j,g,:]
+ *   dk[b,j,g,:] += dx_j query_scale q[b,i,h,:]    (summed over the heads of g)
+ *   dv[b,j,g,:] += w_j dout[b,i,h,:]              (summed over the heads of g)
+ * Masked keys have w_j = 0 and contribute nothing. dout is bf16 bits; dq
+ * (B,T,H,d), dk and dv (B,S,Hkv,d) are double and fully overwritten. */
+int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint16_t* dout, double* dq, double* dk, double* dv,
+                   int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                   int64_t q_offset, double query_scale, double softcap, int64_t window);
 
 /* Threads used by the OpenMP loops (0 leaves the runtime default). */
 void g2ref_set_threads(int n);

@@ -4,7 +4,8 @@ Each case plants one plausible mistake in a copy of oracle/g2ref.c (compiled
 on the CPU into a temporary library), then runs the pin suite against it
 through G2REF_LIB: the suite must fail. The unmodified copy must pass. This
 shows the pins are not tautological: a dropped term, a wrong sign, an
-off-by-one or a wrong index anywhere in the definition is caught.
+off-by-one or a wrong index anywhere in the definition or in its gradients is
+caught.
 """
 import os
 import subprocess
@@ -29,6 +30,16 @@ MUTANTS = {
     "mask before cap (a masked key gets -cap, not -inf)": (
         "s[j] = visible(p, j, window) ? sj : -INFINITY;",
         "s[j] = visible(p, j, window) ? sj : (softcap > 0.0 ? -softcap : -INFINITY);"),
+    # gradients
+    "backward: cap derivative dropped": ("dx *= 1.0 - t * t;", "dx *= 1.0;"),
+    "backward: cap derivative at the capped logit": (
+        "const double t = tanh(xl / softcap);", "const double t = tanh(tanh(xl / softcap));"),
+    "backward: softmax gradient without the row term": (
+        "double dx = w[j] * (x[j] - D);", "double dx = w[j] * x[j];"),
+    "backward: dq without the query scale": (
+        "dqrow[c] += query_scale * dx * widen(krow[c]);", "dqrow[c] += dx * widen(krow[c]);"),
+    "backward: dv without the weight": (
+        "dvrow[c] += w[j] * widen(dorow[c]);", "dvrow[c] += widen(dorow[c]);"),
 }
 
 
@@ -48,7 +59,8 @@ def _build(tmp_path, name, old=None, new=None):
 def _pins_pass(lib):
     env = dict(os.environ, G2REF_LIB=lib, OMP_NUM_THREADS="4")
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                          os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     return res.returncode == 0
 
