@@ -16,8 +16,9 @@ Printed (rank 0, one JSON line): the contract keys, plus
   clocks        nvidia-smi samples taken during the timed region
   layers        per-layer times of the step
   extra         9B pair (local/global separately), 27B decode (KV GB/s,
-                tokens/s), the 9B ragged varlen prefill and the Gemma 3-shaped
-                variant of the 2B pair (window 1024, no cap)
+                tokens/s), the 9B ragged varlen prefill, the Gemma 3-shaped
+                variant of the 2B pair (window 1024, no cap) and the gradients
+                of the 27B-shaped pair (useful backward TFLOP/s)
 
 `--impl reference` times the fp64 oracle (the reference arm of this build)
 on the host cores on bounded samples of the same workload.
@@ -42,7 +43,8 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from global_soft_capped_b200.inputs import WORKLOADS, decode_inputs, prefill_inputs, varlen_inputs  # noqa: E402
+from global_soft_capped_b200.inputs import (  # noqa: E402
+    WORKLOADS, backward_inputs, decode_inputs, prefill_inputs, varlen_inputs)
 
 METRIC = "useful attention TFLOP/s (prefill) and KV GB/s (decode) vs B200 roofline"
 WORKLOAD = "2b"
@@ -62,6 +64,12 @@ def visible_pairs(T, S, q_offset, window):
 
 def prefill_flops(B, T, S, H, d, q_offset, window):
     return 4.0 * d * H * B * visible_pairs(T, S, q_offset, window)
+
+
+def backward_flops(B, T, S, H, d, q_offset, window):
+    """Useful FLOPs of the gradients: the five products S, dP, dV, dK, dQ,
+    2d each, per visible (query, key, head) triple (2.5 x the forward)."""
+    return 2.5 * prefill_flops(B, T, S, H, d, q_offset, window)
 
 
 def varlen_flops(Ts, Ss, H, d, window):
@@ -459,6 +467,26 @@ def extra_workloads(g2, dev, stream, flush):
                    "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
                    "block_size": bs}
     res["9b_varlen_paged_kv"] = rp
+    del q, kp, vp, out, lse
+
+    # gradients of the 27B-shaped layer pair (dq, dk, dv; three launches per call)
+    w = WORKLOADS["27b_backward"]
+    q, k, v, dout = (t.to(dev) for t in backward_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std,
+                                                         w.seed))
+    ws = g2.backward_workspace(w.B, w.T, w.H, dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rb = {}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        out, lse = g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap, window=win,
+                              stream=stream)
+        f = backward_flops(w.B, w.T, w.S, w.H, w.d, 0, win)
+        med, best = time_launches(
+            lambda: g2.prefill_backward(q, k, v, out, lse, dout, query_scale=w.query_scale,
+                                        softcap=w.softcap, window=win, workspace=ws, dq=dq, dk=dk,
+                                        dv=dv, stream=stream), flush, stream)
+        rb[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                   "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+    res["27b_backward"] = rb
     return res
 
 
@@ -532,7 +560,16 @@ def run_single(args, dev):
     w = WORKLOADS[name]
     win = w.window_local if lay == "local" else 0
     stream = torch.cuda.current_stream()
-    if w.kind == "prefill":
+    if name == "27b_backward":
+        q, k, v, dout = (t.to(dev) for t in backward_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d,
+                                                             w.std, w.seed))
+        out, lse = g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap, window=win,
+                              stream=stream)
+        ws = g2.backward_workspace(w.B, w.T, w.H, dev)
+        fn = lambda: g2.prefill_backward(q, k, v, out, lse, dout, query_scale=w.query_scale,
+                                         softcap=w.softcap, window=win, workspace=ws,
+                                         stream=stream)
+    elif w.kind == "prefill":
         q, k, v = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std,
                                                       w.seed))
         fn = lambda: g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap,

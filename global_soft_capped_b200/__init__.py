@@ -5,11 +5,13 @@ Two layers:
 * The C entry points under their own names (``g2attn_prefill``,
   ``g2attn_prefill_varlen``, ``g2attn_prefill_paged``, ``g2attn_decode_workspace_size``,
   ``g2attn_decode``, ``g2attn_decode_ring``, ``g2attn_decode_paged``,
-  ``g2attn_decode_noalloc``, ``g2attn_status_string``,
+  ``g2attn_decode_noalloc``, ``g2attn_backward_workspace_size``,
+  ``g2attn_prefill_backward``, ``g2attn_status_string``,
   ``g2attn_get_device_error``,
   ``g2attn_selftest_wait_timeout``): plain argument marshalling of integers,
   floats and raw pointers through ctypes, returning the status code.
-* Tensor helpers (:func:`prefill`, :func:`prefill_varlen`, :func:`decode`)
+* Tensor helpers (:func:`prefill`, :func:`prefill_varlen`, :func:`decode`,
+  :func:`prefill_backward` and the others below)
   that take torch CUDA tensors, allocate the outputs with torch (memory
   plumbing only) and raise :class:`G2AttnError` on a nonzero status.
 
@@ -42,6 +44,8 @@ EXPORTS = (
     "g2attn_decode_ring",
     "g2attn_decode_paged",
     "g2attn_decode_noalloc",
+    "g2attn_backward_workspace_size",
+    "g2attn_prefill_backward",
     "g2attn_status_string",
     "g2attn_get_device_error",
     "g2attn_selftest_wait_timeout",
@@ -84,6 +88,10 @@ def load_library():
     lib.g2attn_decode_paged.restype = I
     lib.g2attn_decode_noalloc.argtypes = [P, P, P, P, P, P] + [I] * 6 + [F, F, I, P]
     lib.g2attn_decode_noalloc.restype = I
+    lib.g2attn_backward_workspace_size.argtypes = [I, I, I]
+    lib.g2attn_backward_workspace_size.restype = SZ
+    lib.g2attn_prefill_backward.argtypes = [P] * 9 + [I] * 7 + [F, F, I, P, SZ, P]
+    lib.g2attn_prefill_backward.restype = I
     lib.g2attn_status_string.argtypes = [I]
     lib.g2attn_status_string.restype = ctypes.c_char_p
     lib.g2attn_get_device_error.argtypes = []
@@ -118,6 +126,17 @@ def g2attn_prefill_paged(q, k_blocks, v_blocks, out, lse, cu_seqlens_q, block_ta
                                                num_blocks, block_size, max_blocks_per_seq, max_T,
                                                max_S, H, Hkv, d, query_scale, softcap, window,
                                                stream)
+
+
+def g2attn_backward_workspace_size(B, T, H):
+    return load_library().g2attn_backward_workspace_size(B, T, H)
+
+
+def g2attn_prefill_backward(q, k, v, out, lse, dout, dq, dk, dv, B, T, S, H, Hkv, d, q_offset,
+                            query_scale, softcap, window, workspace, workspace_bytes, stream):
+    return load_library().g2attn_prefill_backward(q, k, v, out, lse, dout, dq, dk, dv, B, T, S,
+                                                  H, Hkv, d, q_offset, query_scale, softcap,
+                                                  window, workspace, workspace_bytes, stream)
 
 
 def g2attn_decode_workspace_size(num_seqs, H, d, max_cache_len):
@@ -236,6 +255,34 @@ def prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_T, max_S, *, query_s
     if st != G2ATTN_OK:
         raise G2AttnError(st, "g2attn_prefill_varlen")
     return out, lse
+
+
+def backward_workspace(B, T, H, device="cuda"):
+    """A device buffer of g2attn_backward_workspace_size(B, T, H) bytes."""
+    import torch
+    n = g2attn_backward_workspace_size(B, T, H)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def prefill_backward(q, k, v, out, lse, dout, *, q_offset=0, query_scale=1.0, softcap=50.0,
+                     window=0, workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """Gradients of :func:`prefill`: returns (dq, dk, dv) like q, k, v (bf16)."""
+    import torch
+    _check_bf16(q, k, v, out, dout)
+    B, T, H, d = q.shape
+    S, Hkv = k.shape[1], k.shape[2]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = backward_workspace(B, T, H, q.device)
+    st = g2attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, T, S, H, Hkv, d, int(q_offset),
+                                 float(query_scale), float(softcap), int(window), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != G2ATTN_OK:
+        raise G2AttnError(st, "g2attn_prefill_backward")
+    return dq, dk, dv
 
 
 def decode_workspace(num_seqs, H, d, max_cache_len, device="cuda"):

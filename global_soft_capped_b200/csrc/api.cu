@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_sm100.cuh"
+#include "backward_sm100.cuh"
 
 // Scratch of g2attn_decode_noalloc (see there): 24 MiB, reserved on every GPU
 // that loads the library until the process exits.
@@ -313,9 +314,119 @@ int noalloc_scratch(void** out) {
     return G2ATTN_OK;
 }
 
+// Backward: query-side positions padded to whole 64-position tiles in the
+// workspace (lse2 and D, fp32 each).
+long long bwd_tp(int T) { return (static_cast<long long>(T) + 63) / 64 * 64; }
+
+size_t bwd_ws_bytes(int B, int T, int H) {
+    return 2ull * static_cast<size_t>(B) * static_cast<size_t>(H) * bwd_tp(T) * sizeof(float);
+}
+
+template <int D, int MODE>
+int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mo, const CUtensorMap& mk,
+               const CUtensorMap& mv, g2::BwParams P, int units, int sms, cudaStream_t st) {
+    using C = g2::BwCfg<D>;
+    auto kern = g2::bwd_sm100<D, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+        return G2ATTN_ERR_CUDA;
+    P.num_units = units;
+    const int grid = units < sms ? units : sms;
+    kern<<<grid, g2::BW_THREADS, C::SMEM_BYTES, st>>>(mq, mo, mk, mv, P);
+    return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+}
+
+template <int D>
+int launch_backward(const void* q, const void* k, const void* v, const void* out,
+                    const float* lse, const void* dout, g2::BwParams& P, cudaStream_t st) {
+    CUtensorMap mq, mo, mk, mv;
+    const long long tq = static_cast<long long>(P.B) * P.T, tk = static_cast<long long>(P.B) * P.S;
+    if (!make_map(&mq, q, D, tq, P.H, g2::BW_QPOS, 2) ||
+        !make_map(&mo, dout, D, tq, P.H, g2::BW_QPOS, 2) ||
+        !make_map(&mk, k, D, tk, P.Hkv, g2::BW_KEYS, 1) ||
+        !make_map(&mv, v, D, tk, P.Hkv, g2::BW_KEYS, 1))
+        return G2ATTN_ERR_CUDA;
+    const int sms = num_sms();
+    if (sms <= 0) return G2ATTN_ERR_CUDA;
+    // D = dout . out and lse * log2(e) per (b, h, position)
+    const long long rows = static_cast<long long>(P.B) * P.H * P.Tp;
+    const long long threads = rows * (D / 8);
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    g2::bwd_prep<D><<<static_cast<int>(blocks), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse,
+        const_cast<float*>(P.nlse2), const_cast<float*>(P.ndvec), P.B, P.T, P.H, P.Tp);
+    if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
+    const int BG = P.B * P.Hkv;
+    const int key_tiles = (P.S + g2::BW_KEYS - 1) / g2::BW_KEYS;
+    const int q_tiles = (P.T + g2::BW_QPOS - 1) / g2::BW_QPOS;
+    P.row_tiles = key_tiles;
+    int rc = launch_bwd<D, g2::BW_KV>(mq, mo, mk, mv, P, key_tiles * BG, sms, st);
+    if (rc) return rc;
+    P.row_tiles = q_tiles;
+    return launch_bwd<D, g2::BW_Q>(mq, mo, mk, mv, P, q_tiles * BG, sms, st);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t g2attn_backward_workspace_size(int B, int T, int H) {
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    return bwd_ws_bytes(B, T, H);
+}
+
+int g2attn_prefill_backward(const void* q, const void* k, const void* v, const void* out,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                            int B, int T, int S, int H, int Hkv, int d, int q_offset,
+                            float query_scale, float softcap, int window, void* workspace,
+                            size_t workspace_bytes, g2attn_stream_t stream) {
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)
+        return G2ATTN_ERR_INVALID_ARG;
+    if (B <= 0 || T <= 0 || S <= 0 || q_offset < 0 ||
+        static_cast<long long>(q_offset) + T > S)
+        return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (d != 64 && d != 128) return G2ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return G2ATTN_ERR_MISALIGNED;
+    const long long tq = static_cast<long long>(B) * T, tk = static_cast<long long>(B) * S;
+    if (tq > INT32_MAX || tk > INT32_MAX || static_cast<long long>(B) * H * bwd_tp(T) > INT32_MAX)
+        return G2ATTN_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < bwd_ws_bytes(B, T, H)) return G2ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return G2ATTN_ERR_MISALIGNED;
+    g2::BwParams P{};
+    P.dq = static_cast<__nv_bfloat16*>(dq);
+    P.dk = static_cast<__nv_bfloat16*>(dk);
+    P.dv = static_cast<__nv_bfloat16*>(dv);
+    P.B = B;
+    P.T = T;
+    P.S = S;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.Tp = static_cast<int>(bwd_tp(T));
+    P.q_offset = q_offset;
+    P.window = window;
+    float* ws = static_cast<float*>(workspace);
+    P.nlse2 = ws;
+    P.ndvec = ws + static_cast<size_t>(B) * H * P.Tp;
+    int has_cap = 0;
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, has_cap);
+    P.has_cap = has_cap;
+    P.query_scale = query_scale;
+    {  // the same series window as the forward's fast path
+        g2::PfParams F{};
+        fill_poly(query_scale, softcap, F);
+        P.u_scale = F.u_scale;
+        P.poly_acc_max = F.poly_acc_max;
+    }
+    P.timeout_ns = wait_limit_ns();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 64) return launch_backward<64>(q, k, v, out, lse, dout, P, st);
+    return launch_backward<128>(q, k, v, out, lse, dout, P, st);
+}
 
 int g2attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                    int T, int S, int H, int Hkv, int d, int q_offset, float query_scale,

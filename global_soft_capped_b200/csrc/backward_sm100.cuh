@@ -1,0 +1,678 @@
+// backward_sm100.cuh -- gradients of the soft-capped local/global attention
+// layer on sm_100a (tcgen05 UMMA + TMA), for head sizes d = 64 and 128.
+//
+// Chain rule through the layer (Gemma 2 card, "Method", per-layer attention
+// pseudo-code; derivative of the soft-cap from the "Gemma 2 Guide", Deep Dive
+// item 1: d/dx C tanh(x/C) = 1 - tanh^2(x/C)). With x the scaled logit
+// (query_scale q.k), s = C tanh(x/C) its capped value, P the softmax weights
+// recomputed from the forward's log-sum-exp, and D_i = dout_i . out_i:
+//   dP_ij = dout_i . v_j
+//   dS_ij = P_ij (dP_ij - D_i) (1 - (s_ij / C)^2)         (no cap: the last factor is 1)
+//   dv_j  = sum_i P_ij dout_i,  dk_j = query_scale sum_i dS_ij q_i,
+//   dq_i  = query_scale sum_j dS_ij k_j
+// summing dk, dv over the two query heads that share a KV head.
+//
+// Three launches:
+//   bwd_prep      D_i and lse_i * log2(e), per (b, h, position), into the
+//                 caller's workspace (positions padded to a multiple of 64)
+//   bwd_sm100<D, BW_KV>  one unit = 128 keys of one KV head: K and V stay in
+//                 shared memory, the 64-position query tiles (both heads of
+//                 the group: 128 rows) stream through. X = K Q^T (S^T) and
+//                 Y = V dout^T (dP^T) land in TMEM with one key per lane, so
+//                 P^T and dS^T are written back as bf16 and used directly as
+//                 the A operand of dv += P^T dout and dk += dS^T q.
+//   bwd_sm100<D, BW_Q>   one unit = 64 query positions x 2 heads: q and dout
+//                 stay, the 128-key tiles stream; X = q K^T, Y = dout V^T,
+//                 dq += dS K.
+// TMEM (512 columns): accumulators at 0.., X at 256, Y at 384. KV mode needs
+// 2d + 256 columns, which is why d = 256 is not built here.
+#pragma once
+
+#include "common.cuh"
+
+namespace g2 {
+
+constexpr int BW_KV = 0;
+constexpr int BW_Q = 1;
+constexpr int BW_THREADS = 320;          // 8 elementwise warps, producer, UMMA issuer
+constexpr int BW_EW_THREADS = 256;
+constexpr int BW_WARP_PRODUCER = 8;
+constexpr int BW_WARP_MMA = 9;
+constexpr int BW_QPOS = 64;              // query positions per column/row tile (x 2 heads)
+constexpr int BW_KEYS = 128;             // keys per tile
+constexpr int BW_X_COL = 256;
+constexpr int BW_Y_COL = 384;
+constexpr uint32_t BW_TMEM_COLS = 512;
+
+template <int D>
+struct BwCfg {
+    static_assert(D == 64 || D == 128, "backward kernels are built for d = 64 and 128");
+    static constexpr int TILE_BYTES = 128 * D * 2;         // one 128-row operand tile
+    static constexpr int VEC_BYTES = 2 * 128 * 4;          // lse2 and D of 128 query rows
+    static constexpr int SLOT_BYTES = 2 * TILE_BYTES + VEC_BYTES;
+    static constexpr int SMEM_TILES = 2 * TILE_BYTES + 2 * SLOT_BYTES;  // R1, R2, 2 column slots
+    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct BwParams {
+    __nv_bfloat16* dq;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    const float* nlse2;  // (B, H, Tp): -lse * log2(e); -inf at positions >= T
+    const float* ndvec;  // (B, H, Tp): -D = -(dout . out); 0 at positions >= T
+    int B, T, S, H, Hkv, Tp;
+    int q_offset, window;
+    int num_units;
+    int row_tiles;      // KV: key tiles per (b, g); Q: query tiles per (b, g)
+    float k_exp;        // 2 alpha log2(e) / C   (cap on)
+    float cap_l2;       // C log2(e)             (cap on)
+    float scale_l2;     // alpha log2(e)
+    float query_scale;
+    float u_scale;       // alpha / C              (cap on)
+    float poly_acc_max;  // largest |q.k| with |alpha q.k / C| <= 1/4 (0: series off)
+    int has_cap;
+    unsigned long long timeout_ns;
+};
+
+// tanh(u) for |u| <= 1/4: Taylor series through u^7 (coefficients -1/3, 2/15,
+// -17/315; truncation below 3.3e-7 relative), on the FMA pipe.
+__device__ __forceinline__ float bw_tanh_series(float u) {
+    const float u2 = u * u;
+    float q = fmaf(u2, -17.0f / 315.0f, 2.0f / 15.0f);
+    q = fmaf(u2, q, -1.0f / 3.0f);
+    q = fmaf(u2, q, 1.0f);
+    return u * q;
+}
+
+struct BwUnit {
+    int b, g;
+    int row0;     // KV: first key; Q: first query position (row index t within the sequence)
+    int rvalid;   // KV: keys in the tile (<= 128); Q: positions in the tile (<= 64)
+    int col0;     // first column tile index (KV: 64-position tiles; Q: 128-key tiles)
+    int ncols;    // column tiles (0: no visible pair; KV units then store zeros)
+};
+
+// KV units: key tiles ascending (the earliest keys see the most queries), then
+// batch, then KV head. Q units: query tiles descending, then batch, then head.
+template <int MODE>
+__device__ __forceinline__ void bw_unit(const BwParams& P, int u, BwUnit& U) {
+    const int BG = P.B * P.Hkv;
+    const int rt = u / BG, rem = u % BG;
+    U.b = rem / P.Hkv;
+    U.g = rem % P.Hkv;
+    if (MODE == BW_KV) {
+        U.row0 = rt * BW_KEYS;
+        U.rvalid = min(BW_KEYS, P.S - U.row0);
+        // query rows t whose position t + q_offset sees a key of the tile
+        const int t_lo = max(0, U.row0 - P.q_offset);
+        const int t_hi = P.window > 0
+                             ? min(P.T - 1, U.row0 + BW_KEYS - 1 + P.window - 1 - P.q_offset)
+                             : P.T - 1;
+        U.col0 = t_lo / BW_QPOS;
+        U.ncols = (t_lo <= t_hi) ? t_hi / BW_QPOS - U.col0 + 1 : 0;
+    } else {
+        const int qt = P.row_tiles - 1 - rt;
+        U.row0 = qt * BW_QPOS;
+        U.rvalid = min(BW_QPOS, P.T - U.row0);
+        const int p_min = U.row0 + P.q_offset, p_max = p_min + U.rvalid - 1;
+        const int j_lo = P.window > 0 ? max(0, p_min - P.window + 1) : 0;
+        const int j_hi = min(p_max, P.S - 1);
+        U.col0 = j_lo / BW_KEYS;
+        U.ncols = j_hi / BW_KEYS - U.col0 + 1;
+    }
+}
+
+// -D_i = -(dout_i . out_i) (fp32 sum of bf16 products) and -lse_i * log2(e),
+// D/8 lanes of 16 bytes per (b, h, t); padding positions t in [T, Tp) get
+// -lse2 = -inf (zero weight) and -D = 0. Both are stored negated so that the
+// kernels add them with one packed FMA / ADD.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict__ out,
+                                                const __nv_bfloat16* __restrict__ dout,
+                                                const float* __restrict__ lse, float* nlse2,
+                                                float* ndvec, int B, int T, int H, int Tp) {
+    constexpr int LPR = D / 8;  // lanes per row
+    const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / LPR;
+    const int sub = threadIdx.x % LPR;
+    const long long nrows = static_cast<long long>(B) * H * Tp;
+    const bool in_range = row < nrows;  // no early return: the whole warp shuffles below
+    const int t = static_cast<int>(row % Tp);
+    const long long bh = row / Tp;  // b * H + h
+    const int h = static_cast<int>(bh % H);
+    const long long b = bh / H;
+    float acc = 0.f;
+    if (in_range && t < T) {
+        const size_t off = ((static_cast<size_t>(b) * T + t) * H + h) * D + sub * 8;
+        const uint4 o = *reinterpret_cast<const uint4*>(out + off);
+        const uint4 g = *reinterpret_cast<const uint4*>(dout + off);
+        const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc = fmaf(__uint_as_float(ow[i] << 16), __uint_as_float(gw[i] << 16), acc);
+            acc = fmaf(__uint_as_float(ow[i] & 0xFFFF0000u), __uint_as_float(gw[i] & 0xFFFF0000u),
+                       acc);
+        }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (in_range && sub == 0) {
+        ndvec[row] = -acc;
+        nlse2[row] = (t < T) ? lse[bh * T + t] * -1.4426950408889634f : -INFINITY;
+    }
+}
+
+// Static persistent schedule (as the forward): round r gives CTA c unit
+// r*G + c on even rounds and r*G + G-1-c on odd rounds.
+__device__ __forceinline__ int bw_sched(int r, int c, int G) {
+    return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
+
+// 128-row tile of a (rows, heads, d) tensor into shared memory: D/64 boxes of
+// 64 d-columns (128-byte swizzle). `two_heads`: 64 positions x heads 2g, 2g+1
+// (query-side tensors); else 128 rows of head g (key-side tensors).
+template <int D>
+__device__ __forceinline__ void bw_load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                             int row, int head) {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * 16384, map, bar, c * 64, row, head);
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(BW_THREADS, 1)
+    bwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+              const BwParams P) {
+    using C = BwCfg<D>;
+    constexpr bool KV = MODE == BW_KV;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* sR1 = base;                    // KV: K tile;  Q: q tile
+    uint8_t* sR2 = base + C::TILE_BYTES;    // KV: V tile;  Q: dout tile
+    uint8_t* sSlot = base + 2 * C::TILE_BYTES;  // [2] x (C1 tile, C2 tile, lse2[128], D[128])
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::SMEM_TILES);
+    uint64_t* r_full = bars + 0;
+    uint64_t* r_empty = bars + 1;
+    uint64_t* c_full = bars + 2;    // [2]
+    uint64_t* c_empty = bars + 4;   // [2]
+    uint64_t* xy_full = bars + 6;   // X and Y of the current column tile are in TMEM
+    uint64_t* z_full = bars + 7;    // P / dS written back (8 warp arrivals)
+    uint64_t* acc_done = bars + 8;  // last accumulation of the unit completed
+    uint64_t* acc_free = bars + 9;  // epilogue read the accumulators (8 warp arrivals)
+    uint64_t* drain = bars + 10;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 11);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(r_full, 1);
+        mbar_init(r_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&c_full[i], 1);
+            mbar_init(&c_empty[i], 1);
+        }
+        mbar_init(xy_full, 1);
+        mbar_init(z_full, BW_EW_THREADS / 32);
+        mbar_init(acc_done, 1);
+        mbar_init(acc_free, BW_EW_THREADS / 32);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == BW_WARP_MMA) {
+        tmem_alloc(tmem_holder, BW_TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == BW_WARP_PRODUCER && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmO);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int G = gridDim.x;
+    const int cta = blockIdx.x;
+    const uint64_t lim = P.timeout_ns;
+
+    if (warp == BW_WARP_PRODUCER) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t ct = 0;  // column tiles loaded so far
+            int uw = 0;       // units with work so far
+            bool ok = true;
+            for (int r = 0; ok && r * G < P.num_units; ++r) {
+                const int u = bw_sched(r, cta, G);
+                if (u >= P.num_units) continue;
+                BwUnit U;
+                bw_unit<MODE>(P, u, U);
+                if (U.ncols == 0) continue;
+                if (uw > 0) {
+                    ok = mbar_wait(r_empty, (uw - 1) & 1, abort_flag, lim, SITE_BW_PROD);
+                    if (!ok) break;
+                }
+                mbar_arrive_expect_tx(r_full, 2 * C::TILE_BYTES);
+                if (KV) {
+                    bw_load_tile<D>(sR1, &tmK, r_full, U.b * P.S + U.row0, U.g);
+                    bw_load_tile<D>(sR2, &tmV, r_full, U.b * P.S + U.row0, U.g);
+                } else {
+                    bw_load_tile<D>(sR1, &tmQ, r_full, U.b * P.T + U.row0, 2 * U.g);
+                    bw_load_tile<D>(sR2, &tmO, r_full, U.b * P.T + U.row0, 2 * U.g);
+                }
+                for (int c = 0; c < U.ncols; ++c) {
+                    const int sl = ct & 1;
+                    ok = mbar_wait(&c_empty[sl], ((ct >> 1) & 1) ^ 1, abort_flag, lim,
+                                   SITE_BW_PROD);
+                    if (!ok) break;
+                    uint8_t* slot = sSlot + sl * C::SLOT_BYTES;
+                    if (KV) {
+                        const int t0 = (U.col0 + c) * BW_QPOS;
+                        mbar_arrive_expect_tx(&c_full[sl], 2 * C::TILE_BYTES + C::VEC_BYTES);
+                        bw_load_tile<D>(slot, &tmQ, &c_full[sl], U.b * P.T + t0, 2 * U.g);
+                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmO, &c_full[sl], U.b * P.T + t0,
+                                        2 * U.g);
+                        // -lse2 and -D of the tile's 128 query rows (head 2g, then 2g+1)
+                        float* vec = reinterpret_cast<float*>(slot + 2 * C::TILE_BYTES);
+#pragma unroll
+                        for (int hl = 0; hl < 2; ++hl) {
+                            const size_t off =
+                                (static_cast<size_t>(U.b) * P.H + 2 * U.g + hl) * P.Tp + t0;
+                            bulk_load(vec + hl * 64, P.nlse2 + off, 256, &c_full[sl]);
+                            bulk_load(vec + 128 + hl * 64, P.ndvec + off, 256, &c_full[sl]);
+                        }
+                    } else {
+                        const int key0 = (U.col0 + c) * BW_KEYS;
+                        mbar_arrive_expect_tx(&c_full[sl], 2 * C::TILE_BYTES);
+                        bw_load_tile<D>(slot, &tmK, &c_full[sl], U.b * P.S + key0, U.g);
+                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmV, &c_full[sl], U.b * P.S + key0,
+                                        U.g);
+                    }
+                    ++ct;
+                }
+                ++uw;
+            }
+            // Drain: every copy issued lands before the CTA exits.
+            const uint32_t last = ct < 2u ? ct : 2u;
+            for (uint32_t i = 0; i < last; ++i) {
+                const uint32_t f = ct - 1 - i;
+                mbar_wait_drain(&c_full[f & 1], (f >> 1) & 1, lim);
+            }
+            if (uw > 0) mbar_wait_drain(r_full, (uw - 1) & 1, lim);
+        }
+        __syncwarp();
+    }
+    else if (warp == BW_WARP_MMA) {
+        // ------------------------------------------------------------ UMMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_XY = idesc_bf16(128, 128, false);
+            constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, true);
+            constexpr uint32_t HI = sdesc_hi(1024);  // SBO 1024 B (8 rows x 128 B)
+            // K-major operands (contraction over d): 64-column blocks of 16 KB,
+            // k-step of 16 columns = 32 B inside a block
+            const uint32_t r1_lo = sdesc_lo(smem_u32(sR1), 16);
+            const uint32_t r2_lo = sdesc_lo(smem_u32(sR2), 16);
+            const uint32_t slot_lo = sdesc_lo(smem_u32(sSlot), 16);
+            // the same column tiles read MN-major (contraction over their 128
+            // rows): LBO = 128 rows x 128 B between 64-column blocks
+            const uint32_t slot_lo_mn = sdesc_lo(smem_u32(sSlot), 128 * 128);
+            constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
+            constexpr uint32_t TILE_STEP = C::TILE_BYTES >> 4;
+            uint32_t ct = 0;
+            int uw = 0;
+            bool ok = true;
+            auto kstep = [](int kk) -> uint32_t {
+                return ((kk * 16) / 64) * (16384 >> 4) + (((kk * 16) % 64) / 16) * 2;
+            };
+            for (int r = 0; ok && r * G < P.num_units; ++r) {
+                const int u = bw_sched(r, cta, G);
+                if (u >= P.num_units) continue;
+                BwUnit U;
+                bw_unit<MODE>(P, u, U);
+                if (U.ncols == 0) continue;
+                ok = mbar_wait(r_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                for (int c = 0; c < U.ncols; ++c) {
+                    const int sl = ct & 1;
+                    ok = mbar_wait(&c_full[sl], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // X = R1 C1^T, Y = R2 C2^T (128 x 128, contraction over d).
+                    // X and Y overwrite the P / dS operands of the previous
+                    // tile's accumulations, issued earlier by this thread:
+                    // UMMAs of one thread execute in issue order.
+                    const uint32_t c1_lo = slot_lo + sl * SLOT_STEP;
+                    const uint32_t c2_lo = c1_lo + TILE_STEP;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss_lh(tmem + BW_X_COL, r1_lo + kstep(kk), c1_lo + kstep(kk), HI,
+                                   IDESC_XY, kk != 0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss_lh(tmem + BW_Y_COL, r2_lo + kstep(kk), c2_lo + kstep(kk), HI,
+                                   IDESC_XY, kk != 0);
+                    umma_commit(xy_full);
+                    ok = mbar_wait(z_full, ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                    if (!ok) break;
+                    if (c == 0 && uw > 0) {
+                        ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim, SITE_BW_MMA_ACC);
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    // accumulations: A = bf16 operand in TMEM (128 rows x 128),
+                    // B = a column tile read MN-major (K = its 128 rows, N = d)
+                    const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
+                    const uint32_t c2_mn = c1_mn + TILE_STEP;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t acc = (c == 0 && kk == 0) ? 0u : 1u;
+                        const uint32_t bstep = kk * ((16 * 128) >> 4);
+                        // K indices 16kk..16kk+15 sit at column (kk/4)*64 + (kk%4)*8
+                        // of the operand region (the elementwise warps' layout)
+                        const uint32_t zc = (kk / 4) * 64 + (kk % 4) * 8;
+                        if (KV) {
+                            // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y)
+                            umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c2_mn + bstep, HI,
+                                       IDESC_ACC, acc);
+                            umma_ts_lh(tmem + D, tmem + BW_Y_COL + zc, c1_mn + bstep, HI,
+                                       IDESC_ACC, acc);
+                        } else {
+                            // dq += dS K (dS at X)
+                            umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c1_mn + bstep, HI,
+                                       IDESC_ACC, acc);
+                        }
+                    }
+                    umma_commit(&c_empty[sl]);
+                    ++ct;
+                }
+                if (!ok) break;
+                umma_commit(acc_done);
+                umma_commit(r_empty);
+                ++uw;
+            }
+            // Drain: all issued UMMAs complete before TMEM is released.
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0, lim);
+        }
+        __syncwarp();
+    }
+    else {
+        // ------------------------------------------------------------ elementwise + epilogue
+        // Warps w and w+4 share TMEM lane quadrant w%4 (rows 32(w%4)..+31);
+        // warp w takes columns 0..63 of X and Y, warp w+4 columns 64..127.
+        // KV mode: row = key, column = query row (head 2g + column/64). Q mode:
+        // row = query row (head 2g + row/64), column = key.
+        const int qd = warp & 3, part = warp >> 2;
+        const int r = (qd << 5) | lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
+        const int col0 = part * 64;
+        uint32_t ct = 0;
+        int uw = 0;
+        bool ok = true;
+        for (int rr = 0; ok && rr * G < P.num_units; ++rr) {
+            const int u = bw_sched(rr, cta, G);
+            if (u >= P.num_units) continue;
+            BwUnit U;
+            bw_unit<MODE>(P, u, U);
+            if (U.ncols == 0) {
+                // keys that no query sees: zero gradients (KV mode only; every
+                // query sees at least its own key)
+                if (KV && r < U.rvalid) {
+                    const size_t row = (static_cast<size_t>(U.b) * P.S + U.row0 + r) * P.Hkv + U.g;
+#pragma unroll
+                    for (int c = 0; c < D / 2; c += 8) {
+                        *reinterpret_cast<uint4*>(P.dv + row * D + part * (D / 2) + c) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(P.dk + row * D + part * (D / 2) + c) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+                continue;
+            }
+            // Q mode: this thread's query row, its -lse2 and -D
+            const int hl_row = r >> 6, pr_row = r & 63;
+            const int t_row = U.row0 + pr_row;  // Q mode
+            float row_nl2 = -INFINITY, row_nd = 0.f;
+            if (!KV && t_row < P.T) {
+                const size_t off =
+                    (static_cast<size_t>(U.b) * P.H + 2 * U.g + hl_row) * P.Tp + t_row;
+                row_nl2 = P.nlse2[off];
+                row_nd = P.ndvec[off];
+            }
+            const int key_row = U.row0 + r;  // KV mode
+            for (int c = 0; c < U.ncols; ++c) {
+                const int sl = ct & 1;
+                ok = mbar_wait(xy_full, ct & 1, abort_flag, lim, SITE_BW_EW);
+                if (KV && ok)  // the column tile's lse2 / D, copied with its operands
+                    ok = mbar_wait(&c_full[sl], (ct >> 1) & 1, abort_flag, lim, SITE_BW_EW);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const float* vec =
+                    reinterpret_cast<const float*>(sSlot + sl * C::SLOT_BYTES + 2 * C::TILE_BYTES);
+                const int ccol0 = (U.col0 + c) * (KV ? BW_QPOS : BW_KEYS);  // first t or key
+                // Every pair of the tile visible? (then no per-element mask)
+                bool interior;
+                {
+                    int j_lo, j_hi, t_lo, t_hi;
+                    if (KV) {
+                        j_lo = U.row0; j_hi = U.row0 + BW_KEYS - 1;
+                        t_lo = ccol0;  t_hi = ccol0 + BW_QPOS - 1;
+                    } else {
+                        j_lo = ccol0;  j_hi = ccol0 + BW_KEYS - 1;
+                        t_lo = U.row0; t_hi = U.row0 + BW_QPOS - 1;
+                    }
+                    interior = j_hi <= t_lo + P.q_offset && t_hi < P.T && j_hi < P.S &&
+                               (P.window == 0 || t_hi + P.q_offset - j_lo < P.window);
+                }
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {  // two chunks of 32 columns
+                    const int cb = col0 + 32 * h2;
+                    uint32_t xv[32], yv[32];
+                    tmem_ld32_async(tmem + lane_addr + BW_X_COL + cb, xv);
+                    tmem_ld32_async(tmem + lane_addr + BW_Y_COL + cb, yv);
+                    tmem_wait_ld();
+                    tmem_reg_fence(xv);
+                    tmem_reg_fence(yv);
+                    // the cap's tanh by series when every |u| of this warp's chunk <= 1/4
+                    float amax = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(xv[i])));
+                    const bool poly = __all_sync(0xffffffffu, amax <= P.poly_acc_max);
+                    uint32_t pp[16], pd[16];
+                    // -lse2 / -D of the column pair i, i+1 (KV: per column, from
+                    // the slot; Q: this row's)
+                    auto vec_pair = [&](int i, float2& nl2, float2& nd) {
+                        if (KV) {
+                            nl2 = *reinterpret_cast<const float2*>(vec + cb + i);
+                            nd = *reinterpret_cast<const float2*>(vec + 128 + cb + i);
+                        } else {
+                            nl2 = make_float2(row_nl2, row_nl2);
+                            nd = make_float2(row_nd, row_nd);
+                        }
+                    };
+                    if (interior && (poly || !P.has_cap)) {
+                        // fast path: no mask, packed pairs. P = 2^(s2 - lse2),
+                        // dS = P (dP - D) (1 - tanh^2)
+                        const float2 one = make_float2(1.f, 1.f), mone = make_float2(-1.f, -1.f);
+                        if (P.has_cap) {
+                            const float2 us = make_float2(P.u_scale, P.u_scale);
+                            const float2 c3 = make_float2(-17.0f / 315.0f, -17.0f / 315.0f);
+                            const float2 c2 = make_float2(2.0f / 15.0f, 2.0f / 15.0f);
+                            const float2 c1 = make_float2(-1.0f / 3.0f, -1.0f / 3.0f);
+                            const float2 cl2 = make_float2(P.cap_l2, P.cap_l2);
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2) {
+                                float2 nl2, nd;
+                                vec_pair(i, nl2, nd);
+                                const float2 x = make_float2(__uint_as_float(xv[i]),
+                                                             __uint_as_float(xv[i + 1]));
+                                const float2 y = make_float2(__uint_as_float(yv[i]),
+                                                             __uint_as_float(yv[i + 1]));
+                                const float2 u = mul2(x, us);
+                                const float2 u2 = mul2(u, u);
+                                float2 q = fma2(u2, c3, c2);
+                                q = fma2(u2, q, c1);
+                                q = fma2(u2, q, one);
+                                const float2 th = mul2(u, q);              // tanh(alpha x / C)
+                                const float2 e2 = fma2(th, cl2, nl2);       // s2 - lse2
+                                const float2 dcap = fma2(mul2(th, th), mone, one);
+                                const float p0 = ex2_approx(e2.x), p1 = ex2_approx(e2.y);
+                                const float2 ds = mul2(mul2(make_float2(p0, p1), add2(y, nd)), dcap);
+                                pp[i / 2] = pack_bf16x2(p0, p1);
+                                pd[i / 2] = pack_bf16x2(ds.x, ds.y);
+                            }
+                        } else {
+                            const float2 sl2 = make_float2(P.scale_l2, P.scale_l2);
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2) {
+                                float2 nl2, nd;
+                                vec_pair(i, nl2, nd);
+                                const float2 x = make_float2(__uint_as_float(xv[i]),
+                                                             __uint_as_float(xv[i + 1]));
+                                const float2 y = make_float2(__uint_as_float(yv[i]),
+                                                             __uint_as_float(yv[i + 1]));
+                                const float2 e2 = fma2(x, sl2, nl2);
+                                const float p0 = ex2_approx(e2.x), p1 = ex2_approx(e2.y);
+                                const float2 ds = mul2(make_float2(p0, p1), add2(y, nd));
+                                pp[i / 2] = pack_bf16x2(p0, p1);
+                                pd[i / 2] = pack_bf16x2(ds.x, ds.y);
+                            }
+                        }
+                    } else {
+                        // general path: per-element mask, exact cap when |u| > 1/4
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float2 nl2v, ndv;
+                            vec_pair(i, nl2v, ndv);
+                            float pv[2], dsv[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int cc = cb + i + e;  // column 0..127
+                                int t, j;
+                                if (KV) {
+                                    t = ccol0 + (cc & 63);  // head 2g + cc/64
+                                    j = key_row;
+                                } else {
+                                    t = t_row;
+                                    j = ccol0 + cc;
+                                }
+                                const float nl2 = e ? nl2v.y : nl2v.x;
+                                const float nd = e ? ndv.y : ndv.x;
+                                const int pos = t + P.q_offset;
+                                const bool vis = (j <= pos) &&
+                                                 (P.window == 0 || pos - j < P.window) &&
+                                                 (t < P.T) && (j < P.S);
+                                const float x = __uint_as_float(xv[i + e]);
+                                float s2, dcap;
+                                if (P.has_cap) {
+                                    float th;
+                                    if (poly) {
+                                        th = bw_tanh_series(x * P.u_scale);
+                                    } else {
+                                        // tanh(alpha x / C) = 1 - 2 / (1 + 2^(2 alpha log2(e) x / C))
+                                        const float ex = ex2_approx(x * P.k_exp);
+                                        th = fmaf(-2.0f, rcp_approx(1.0f + ex), 1.0f);
+                                    }
+                                    s2 = P.cap_l2 * th;
+                                    dcap = fmaf(-th, th, 1.0f);
+                                } else {
+                                    s2 = x * P.scale_l2;
+                                    dcap = 1.0f;
+                                }
+                                const float pw = vis ? ex2_approx(s2 + nl2) : 0.0f;
+                                pv[e] = pw;
+                                dsv[e] = pw * (__uint_as_float(yv[i + e]) + nd) * dcap;
+                            }
+                            pp[i / 2] = pack_bf16x2(pv[0], pv[1]);
+                            pd[i / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                        }
+                    }
+                    // bf16 pairs of columns cb .. cb+31 go to TMEM columns
+                    // col0 + 16*h2 .. +15: inside this warp's own X / Y columns,
+                    // already read (chunk 0), never the other warp's (no
+                    // ordering between the two warps of a quadrant is needed)
+                    const uint32_t zc = col0 + 16 * h2;
+                    if (KV) {
+                        tmem_st16(tmem + lane_addr + BW_X_COL + zc, pp);  // P^T
+                        tmem_st16(tmem + lane_addr + BW_Y_COL + zc, pd);  // dS^T
+                    } else {
+                        tmem_st16(tmem + lane_addr + BW_X_COL + zc, pd);  // dS
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(z_full);
+                ++ct;
+            }
+            if (!ok) break;
+            // ---- epilogue: accumulators -> bf16 gradients
+            ok = mbar_wait(acc_done, uw & 1, abort_flag, lim, SITE_BW_EW_ACC);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            constexpr int HALF = D / 2;  // accumulator columns per warp
+            if (KV) {
+                const bool valid = r < U.rvalid;
+                const size_t row = (static_cast<size_t>(U.b) * P.S + key_row) * P.Hkv + U.g;
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {  // a = 0: dv (columns 0..), a = 1: dk (columns D..)
+                    const float f = a ? P.query_scale : 1.0f;
+                    __nv_bfloat16* dst = (a ? P.dk : P.dv) + row * D + part * HALF;
+#pragma unroll 1
+                    for (int c = 0; c < HALF / 16; ++c) {
+                        uint32_t v[16];
+                        tmem_ld16(tmem + lane_addr + a * D + part * HALF + c * 16, v);
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * f,
+                                                __uint_as_float(v[2 * i + 1]) * f);
+                        if (valid) {
+                            uint4* o = reinterpret_cast<uint4*>(dst + c * 16);
+                            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        }
+                    }
+                }
+            } else {
+                const bool valid = pr_row < U.rvalid;
+                const size_t row = (static_cast<size_t>(U.b) * P.T + t_row) * P.H + 2 * U.g + hl_row;
+                __nv_bfloat16* dst = P.dq + row * D + part * HALF;
+#pragma unroll 1
+                for (int c = 0; c < HALF / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + lane_addr + part * HALF + c * 16, v);
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * P.query_scale,
+                                            __uint_as_float(v[2 * i + 1]) * P.query_scale);
+                    if (valid) {
+                        uint4* o = reinterpret_cast<uint4*>(dst + c * 16);
+                        o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_free);
+            ++uw;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == BW_WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, BW_TMEM_COLS);
+    }
+}
+
+}  // namespace g2

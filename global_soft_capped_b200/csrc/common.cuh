@@ -32,6 +32,12 @@ enum WaitSite : unsigned int {
     SITE_SM_O_DONE = 10,
     SITE_DRAIN = 11,
     SITE_SM_PAIR = 12,
+    SITE_BW_PROD = 13,      // backward producer: slot or tile buffers free
+    SITE_BW_MMA = 14,       // backward issuer: operand tiles landed
+    SITE_BW_EW = 15,        // backward elementwise: X / Y in TMEM
+    SITE_BW_MMA_Z = 16,     // backward issuer: P / dS written back
+    SITE_BW_MMA_ACC = 17,   // backward issuer: accumulators read out
+    SITE_BW_EW_ACC = 18,    // backward elementwise: accumulation finished
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -132,6 +138,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Contiguous global -> shared copy of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned), counted on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -71,6 +71,12 @@ WORKLOADS = {
         softcap=50.0, std=1.0, seed=4, num_seqs=16, len_lo=512, len_hi=8192,
         tail_T=1024, tail_S=8192,
         note="9B-shaped ragged packed prefill plus a chunked-prefill tail"),
+    # Training-shaped 27B layer pair for the gradients (dout drawn after q, k, v
+    # from the same generator, N(0, 1) -> bf16)
+    "27b_backward": Workload(
+        "27b_backward", "prefill", H=32, Hkv=16, d=128, window_local=4096,
+        query_scale=144.0 ** -0.5, softcap=50.0, std=1.0, seed=6, B=1, T=8192, S=8192,
+        note="27B-shaped layer pair, forward outputs and upstream gradients for the backward"),
     # Gemma 3-shaped parameter variant of the same layer pair (the research-hub
     # page: window 1024, soft-capping replaced by QK-norm, which acts on the
     # inputs upstream of this kernel, so the cap is off here).
@@ -158,6 +164,17 @@ def varlen_inputs(num_seqs, len_lo, len_hi, H, Hkv, d, std=1.0, seed=0,
     v = _normal_bf16((ck[-1], Hkv, d), std, g)
     return (Ts, Ss, torch.tensor(cq, dtype=torch.int32), torch.tensor(ck, dtype=torch.int32),
             q, k, v)
+
+
+def backward_inputs(B, T, S, H, Hkv, d, std=1.0, seed=0):
+    """q, k, v as prefill_inputs, then the upstream gradient dout (B,T,H,d),
+    fp32 standard normals rounded to bf16, from the same generator."""
+    g = _gen(seed)
+    q = _normal_bf16((B, T, H, d), std, g)
+    k = _normal_bf16((B, S, Hkv, d), std, g)
+    v = _normal_bf16((B, S, Hkv, d), std, g)
+    dout = _normal_bf16((B, T, H, d), 1.0, g)
+    return q, k, v, dout
 
 
 def workload_inputs(name: str):

@@ -220,6 +220,42 @@ G2ATTN_API int g2attn_decode_noalloc(const void* q, const void* k_cache, const v
                           int num_seqs, int total_k, int max_cache_len, int H, int Hkv, int d,
                           float query_scale, float softcap, int window, g2attn_stream_t stream);
 
+/*
+ * Bytes of device workspace g2attn_prefill_backward needs: two fp32 values
+ * (lse in log2 units and D = dout . out) per (b, h, query position), the
+ * positions rounded up to a multiple of 64. 0 for non-positive arguments.
+ */
+G2ATTN_API size_t g2attn_backward_workspace_size(int B, int T, int H);
+
+/*
+ * Gradients of g2attn_prefill (same q, k, v, sizes and parameters) for the
+ * upstream gradient dout of its output. The chain rule runs through the value
+ * mix, the softmax, the soft-cap (derivative 1 - tanh^2(x/C) of C tanh(x/C),
+ * "Gemma 2 Guide", Deep Dive item 1; none when softcap = 0) and the scaled
+ * dot product; dk and dv sum over the two query heads sharing a KV head.
+ *   out (B,T,H,d) bf16 and lse (B,H,T) fp32: the forward's outputs for these
+ *     inputs (the softmax weights are recomputed from lse, not stored).
+ *   dout (B,T,H,d) bf16; dq (B,T,H,d), dk and dv (B,S,Hkv,d) bf16, written in
+ *     full (keys that no query sees get zero gradients).
+ *   workspace: device memory of at least
+ *     g2attn_backward_workspace_size(B, T, H) bytes, 16-byte aligned, owned by
+ *     the caller and overwritten.
+ * Supported: d = 64 and 128 (the 27B and smaller head sizes). d = 256 returns
+ * G2ATTN_ERR_UNSUPPORTED: the fused dk/dv kernel keeps both d-column
+ * accumulators and two 128-column work tiles in the 512 TMEM columns of an SM.
+ * Other limits and errors as g2attn_prefill; lse is required; a workspace that
+ * is missing or too small returns G2ATTN_ERR_WORKSPACE. Three kernels run on
+ * `stream`: a pass computing D and lse*log2(e), the dk/dv kernel (K, V tiles
+ * resident, query tiles streamed) and the dq kernel (query tiles resident).
+ * Source: the Gemma 2 card's "Method" pseudo-code (the forward being
+ * differentiated) and the Guide's derivative of the cap.
+ */
+G2ATTN_API int g2attn_prefill_backward(const void* q, const void* k, const void* v,
+                            const void* out, const float* lse, const void* dout, void* dq,
+                            void* dk, void* dv, int B, int T, int S, int H, int Hkv, int d,
+                            int q_offset, float query_scale, float softcap, int window,
+                            void* workspace, size_t workspace_bytes, g2attn_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 G2ATTN_API const char* g2attn_status_string(int status);
 

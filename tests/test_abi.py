@@ -146,3 +146,35 @@ def test_paged_prefill_rejects_before_launch(lib):
     assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
     bad = list(base); bad[6] = None          # no block table
     assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
+
+
+def test_backward_workspace_size(lib):
+    a = g2.g2attn_backward_workspace_size(1, 8192, 32)
+    assert a == 2 * 1 * 32 * 8192 * 4
+    assert g2.g2attn_backward_workspace_size(2, 65, 4) == 2 * 2 * 4 * 128 * 4  # 64-padded
+    assert g2.g2attn_backward_workspace_size(0, 64, 4) == 0
+
+
+def backward_args(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+             B=1, T=64, S=64, H=8, Hkv=4, d=128, q_offset=0, query_scale=0.0625, softcap=50.0,
+             window=0, workspace=FAKE, workspace_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(lse=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(dout=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(dk=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(q_offset=1), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(softcap=-1.0), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(d=256), g2.G2ATTN_ERR_UNSUPPORTED),               # TMEM budget of the dk/dv kernel
+    (dict(H=6), g2.G2ATTN_ERR_UNSUPPORTED),
+    (dict(workspace=None), g2.G2ATTN_ERR_WORKSPACE),
+    (dict(workspace_bytes=1024), g2.G2ATTN_ERR_WORKSPACE),
+    (dict(workspace=ctypes.c_void_p((1 << 20) + 4)), g2.G2ATTN_ERR_MISALIGNED),
+    (dict(dq=ctypes.c_void_p((1 << 20) + 8)), g2.G2ATTN_ERR_MISALIGNED),
+])
+def test_backward_rejects_before_launch(lib, kw, status):
+    assert g2.g2attn_prefill_backward(*backward_args(**kw)) == status
