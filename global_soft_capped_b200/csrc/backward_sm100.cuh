@@ -196,12 +196,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* r_empty = bars + 1;
     uint64_t* c_full = bars + 2;    // [2]
     uint64_t* c_empty = bars + 4;   // [2]
-    uint64_t* xy_full = bars + 6;   // X and Y of the current column tile are in TMEM
-    uint64_t* z_full = bars + 7;    // P / dS written back (8 warp arrivals)
-    uint64_t* acc_done = bars + 8;  // last accumulation of the unit completed
-    uint64_t* acc_free = bars + 9;  // epilogue read the accumulators (8 warp arrivals)
-    uint64_t* drain = bars + 10;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 11);
+    // Column halves h = 0, 1 (columns 0..63 / 64..127 of X and Y, the column
+    // parts of the elementwise warps) run as a two-stage pipeline:
+    uint64_t* xy_full = bars + 6;   // [2] X and Y of half h of the current tile are in TMEM
+    uint64_t* z_full = bars + 8;    // [2] P / dS of half h written back (4 warp arrivals)
+    uint64_t* acc_done = bars + 10; // last accumulation of the unit completed
+    uint64_t* acc_free = bars + 11; // epilogue read the accumulators (8 warp arrivals)
+    uint64_t* drain = bars + 12;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -213,8 +215,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             mbar_init(&c_full[i], 1);
             mbar_init(&c_empty[i], 1);
         }
-        mbar_init(xy_full, 1);
-        mbar_init(z_full, BW_EW_THREADS / 32);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&xy_full[h], 1);
+            mbar_init(&z_full[h], BW_EW_THREADS / 64);
+        }
         mbar_init(acc_done, 1);
         mbar_init(acc_free, BW_EW_THREADS / 32);
         mbar_init(drain, 1);
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     else if (warp == BW_WARP_MMA) {
         // ------------------------------------------------------------ UMMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_XY = idesc_bf16(128, 128, false);
+            constexpr uint32_t IDESC_XY = idesc_bf16(128, 64, false);  // one column half
             constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, true);
             constexpr uint32_t HI = sdesc_hi(1024);  // SBO 1024 B (8 rows x 128 B)
             // K-major operands (contraction over d): 64-column blocks of 16 KB,
@@ -321,12 +325,56 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const uint32_t slot_lo_mn = sdesc_lo(smem_u32(sSlot), 128 * 128);
             constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
             constexpr uint32_t TILE_STEP = C::TILE_BYTES >> 4;
+            constexpr uint32_t HALF_ROWS = (64 * 128) >> 4;  // rows 64.. of a tile
             uint32_t ct = 0;
             int uw = 0;
             bool ok = true;
             auto kstep = [](int kk) -> uint32_t {
                 return ((kk * 16) / 64) * (16384 >> 4) + (((kk * 16) % 64) / 16) * 2;
             };
+            // X, Y columns [64h, 64h + 64) of the tile in slot sl: rows 64h.. of
+            // the column tiles (N = 64), contraction over d
+            auto issue_xy = [&](int sl, int h) {
+                const uint32_t c1 = slot_lo + sl * SLOT_STEP + h * HALF_ROWS;
+                const uint32_t c2 = c1 + TILE_STEP;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_lh(tmem + BW_X_COL + 64 * h, r1_lo + kstep(kk), c1 + kstep(kk), HI,
+                               IDESC_XY, kk != 0);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_lh(tmem + BW_Y_COL + 64 * h, r2_lo + kstep(kk), c2 + kstep(kk), HI,
+                               IDESC_XY, kk != 0);
+                umma_commit(&xy_full[h]);
+            };
+            // accumulations over the half's 64 rows (K indices 64h..64h+63): A =
+            // the bf16 operand the half's warps wrote at columns 64h + 8(kk%4)
+            auto issue_acc = [&](int sl, int h, bool first) {
+                const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
+                const uint32_t c2_mn = c1_mn + TILE_STEP;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int kk = 4 * h + k4;
+                    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                    const uint32_t bstep = kk * ((16 * 128) >> 4);
+                    const uint32_t zc = 64 * h + 8 * k4;
+                    if (KV) {
+                        // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y)
+                        umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c2_mn + bstep, HI, IDESC_ACC,
+                                   acc);
+                        umma_ts_lh(tmem + D, tmem + BW_Y_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
+                                   acc);
+                    } else {
+                        // dq += dS K (dS at X)
+                        umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
+                                   acc);
+                    }
+                }
+            };
+            // Issue order per tile c (slot sl): XY_0(c) XY_1(c) | z_0 | ACC_0(c)
+            // XY_0(c+1) | z_1 | ACC_1(c) XY_1(c+1). A half's X / Y overwrite
+            // that half's P / dS only after the accumulation reading them was
+            // issued; UMMAs of one thread execute in issue order.
             for (int r = 0; ok && r * G < P.num_units; ++r) {
                 const int u = bw_sched(r, cta, G);
                 if (u >= P.num_units) continue;
@@ -336,57 +384,35 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 ok = mbar_wait(r_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
                 tc_fence_after();
+                ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                issue_xy(ct & 1, 0);
+                issue_xy(ct & 1, 1);
                 for (int c = 0; c < U.ncols; ++c) {
                     const int sl = ct & 1;
-                    ok = mbar_wait(&c_full[sl], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
-                    if (!ok) break;
-                    tc_fence_after();
-                    // X = R1 C1^T, Y = R2 C2^T (128 x 128, contraction over d).
-                    // X and Y overwrite the P / dS operands of the previous
-                    // tile's accumulations, issued earlier by this thread:
-                    // UMMAs of one thread execute in issue order.
-                    const uint32_t c1_lo = slot_lo + sl * SLOT_STEP;
-                    const uint32_t c2_lo = c1_lo + TILE_STEP;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss_lh(tmem + BW_X_COL, r1_lo + kstep(kk), c1_lo + kstep(kk), HI,
-                                   IDESC_XY, kk != 0);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss_lh(tmem + BW_Y_COL, r2_lo + kstep(kk), c2_lo + kstep(kk), HI,
-                                   IDESC_XY, kk != 0);
-                    umma_commit(xy_full);
-                    ok = mbar_wait(z_full, ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                    const bool next = c + 1 < U.ncols;
+                    ok = mbar_wait(&z_full[0], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
                     if (!ok) break;
                     if (c == 0 && uw > 0) {
                         ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim, SITE_BW_MMA_ACC);
                         if (!ok) break;
                     }
                     tc_fence_after();
-                    // accumulations: A = bf16 operand in TMEM (128 rows x 128),
-                    // B = a column tile read MN-major (K = its 128 rows, N = d)
-                    const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
-                    const uint32_t c2_mn = c1_mn + TILE_STEP;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t acc = (c == 0 && kk == 0) ? 0u : 1u;
-                        const uint32_t bstep = kk * ((16 * 128) >> 4);
-                        // K indices 16kk..16kk+15 sit at column (kk/4)*64 + (kk%4)*8
-                        // of the operand region (the elementwise warps' layout)
-                        const uint32_t zc = (kk / 4) * 64 + (kk % 4) * 8;
-                        if (KV) {
-                            // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y)
-                            umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c2_mn + bstep, HI,
-                                       IDESC_ACC, acc);
-                            umma_ts_lh(tmem + D, tmem + BW_Y_COL + zc, c1_mn + bstep, HI,
-                                       IDESC_ACC, acc);
-                        } else {
-                            // dq += dS K (dS at X)
-                            umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c1_mn + bstep, HI,
-                                       IDESC_ACC, acc);
-                        }
+                    issue_acc(sl, 0, c == 0);
+                    if (next) {
+                        ok = mbar_wait(&c_full[sl ^ 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
+                                       SITE_BW_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_xy(sl ^ 1, 0);
                     }
+                    ok = mbar_wait(&z_full[1], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_acc(sl, 1, false);
                     umma_commit(&c_empty[sl]);
+                    if (next) issue_xy(sl ^ 1, 1);
                     ++ct;
                 }
                 if (!ok) break;
@@ -446,7 +472,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const int key_row = U.row0 + r;  // KV mode
             for (int c = 0; c < U.ncols; ++c) {
                 const int sl = ct & 1;
-                ok = mbar_wait(xy_full, ct & 1, abort_flag, lim, SITE_BW_EW);
+                ok = mbar_wait(&xy_full[part], ct & 1, abort_flag, lim, SITE_BW_EW);
                 if (KV && ok)  // the column tile's lse2 / D, copied with its operands
                     ok = mbar_wait(&c_full[sl], (ct >> 1) & 1, abort_flag, lim, SITE_BW_EW);
                 ok = __all_sync(0xffffffffu, ok);
@@ -607,7 +633,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(z_full);
+                if (lane == 0) mbar_arrive(&z_full[part]);
                 ++ct;
             }
             if (!ok) break;
