@@ -178,6 +178,32 @@ __device__ __forceinline__ void bw_load_tile(uint8_t* dst, const CUtensorMap* ma
     for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * 16384, map, bar, c * 64, row, head);
 }
 
+// HALF (= D/2) accumulator columns of this thread's row, times f, as bf16 to
+// dst (when valid): all loads in flight before one wait.
+template <int HALF>
+__device__ __forceinline__ void bw_store_acc(uint32_t taddr, __nv_bfloat16* dst, float f,
+                                             bool valid) {
+    static_assert(HALF % 32 == 0, "accumulator chunks");
+    uint32_t v[HALF / 32][32];
+#pragma unroll
+    for (int j = 0; j < HALF / 32; ++j) tmem_ld32_async(taddr + 32 * j, v[j]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < HALF / 32; ++j) {
+        tmem_reg_fence(v[j]);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[j][2 * i]) * f, __uint_as_float(v[j][2 * i + 1]) * f);
+        if (valid) {
+            uint4* o = reinterpret_cast<uint4*>(dst + 32 * j);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                o[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+    }
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(BW_THREADS, 1)
     bwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
@@ -650,41 +676,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 for (int a = 0; a < 2; ++a) {  // a = 0: dv (columns 0..), a = 1: dk (columns D..)
                     const float f = a ? P.query_scale : 1.0f;
                     __nv_bfloat16* dst = (a ? P.dk : P.dv) + row * D + part * HALF;
-#pragma unroll 1
-                    for (int c = 0; c < HALF / 16; ++c) {
-                        uint32_t v[16];
-                        tmem_ld16(tmem + lane_addr + a * D + part * HALF + c * 16, v);
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * f,
-                                                __uint_as_float(v[2 * i + 1]) * f);
-                        if (valid) {
-                            uint4* o = reinterpret_cast<uint4*>(dst + c * 16);
-                            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                        }
-                    }
+                    bw_store_acc<HALF>(tmem + lane_addr + a * D + part * HALF, dst, f, valid);
                 }
             } else {
                 const bool valid = pr_row < U.rvalid;
                 const size_t row = (static_cast<size_t>(U.b) * P.T + t_row) * P.H + 2 * U.g + hl_row;
                 __nv_bfloat16* dst = P.dq + row * D + part * HALF;
-#pragma unroll 1
-                for (int c = 0; c < HALF / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_ld16(tmem + lane_addr + part * HALF + c * 16, v);
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * P.query_scale,
-                                            __uint_as_float(v[2 * i + 1]) * P.query_scale);
-                    if (valid) {
-                        uint4* o = reinterpret_cast<uint4*>(dst + c * 16);
-                        o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
-                }
+                bw_store_acc<HALF>(tmem + lane_addr + part * HALF, dst, P.query_scale, valid);
             }
             tc_fence_before();
             __syncwarp();

@@ -596,6 +596,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         constexpr int HC = PF_BN / PF_NSPLIT;           // key columns per part
         static_assert(HC % 32 == 0 && (D / PF_NSPLIT) % 16 == 0, "softmax split");
         constexpr int OC = D / PF_NSPLIT;               // O columns per part
+        constexpr int EC = OC >= 64 ? 64 : OC;          // O columns per TMEM round trip
+        static_assert(OC % EC == 0 && EC % 32 == 0, "O chunks");
         const int qd = warp & 3;                        // TMEM lane quadrant
         const int part = warp >> 2;                     // column part of this warp
         const int r = (qd << 5) | lane;                 // MMA row == TMEM lane
@@ -731,13 +733,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
                     const uint32_t o_addr = tmem + lane_addr + part * OC;
 #pragma unroll 1
-                    for (int c = 0; c < OC / 16; ++c) {
-                        uint32_t v[16];
-                        tmem_ld16(o_addr + c * 16, v);
+                    for (int c = 0; c < OC / 32; ++c) {  // 32 columns per TMEM round trip
+                        uint32_t v[32];
+                        tmem_ld32(o_addr + c * 32, v);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
+                        for (int i = 0; i < 32; ++i)
                             v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-                        tmem_st16(o_addr + c * 16, v);
+                        tmem_st32(o_addr + c * 32, v);
                     }
                     tmem_wait_st();
                     l *= f;
@@ -843,18 +845,26 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             __nv_bfloat16* optr = P.out + orow * D + part * OC;
             const uint32_t o_addr = tmem + lane_addr + part * OC;
 #pragma unroll 1
-            for (int c = 0; c < OC / 16; ++c) {
-                uint32_t v[16];
-                tmem_ld16(o_addr + c * 16, v);
-                uint32_t pkk[8];
+            for (int c = 0; c < OC / EC; ++c) {  // EC columns per TMEM round trip
+                uint32_t v[EC / 32][32];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    pkk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
-                                         __uint_as_float(v[2 * i + 1]) * inv_l);
-                if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(optr + c * 16);
-                    dst[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
-                    dst[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
+                for (int j = 0; j < EC / 32; ++j) tmem_ld32_async(o_addr + c * EC + 32 * j, v[j]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < EC / 32; ++j) {
+                    tmem_reg_fence(v[j]);
+                    uint32_t pkk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pkk[i] = pack_bf16x2(__uint_as_float(v[j][2 * i]) * inv_l,
+                                             __uint_as_float(v[j][2 * i + 1]) * inv_l);
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(optr + c * EC + 32 * j);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            dst[q4] = make_uint4(pkk[4 * q4], pkk[4 * q4 + 1], pkk[4 * q4 + 2],
+                                                 pkk[4 * q4 + 3]);
+                    }
                 }
             }
             if (valid && part == 0 && P.lse != nullptr) {
