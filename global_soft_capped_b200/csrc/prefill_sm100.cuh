@@ -105,6 +105,7 @@ struct PfParams {
     float u_scale;  // alpha/C             (cap on)
     float poly_acc_max;  // largest |q.k| for which |alpha q.k / C| <= PF_POLY_U_MAX
     int has_cap;
+    int out_align32;  // out is 32-byte aligned: the epilogue stores 32 bytes at a time
     unsigned long long timeout_ns;
 };
 
@@ -859,11 +860,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         pkk[i] = pack_bf16x2(__uint_as_float(v[j][2 * i]) * inv_l,
                                              __uint_as_float(v[j][2 * i + 1]) * inv_l);
                     if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(optr + c * EC + 32 * j);
+                        __nv_bfloat16* dst = optr + c * EC + 32 * j;
+                        if (P.out_align32) {  // two 32-byte stores: one full sector each
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            dst[q4] = make_uint4(pkk[4 * q4], pkk[4 * q4 + 1], pkk[4 * q4 + 2],
-                                                 pkk[4 * q4 + 3]);
+                            for (int q8 = 0; q8 < 2; ++q8)
+                                st_global_v8(dst + 16 * q8, pkk[8 * q8], pkk[8 * q8 + 1],
+                                             pkk[8 * q8 + 2], pkk[8 * q8 + 3], pkk[8 * q8 + 4],
+                                             pkk[8 * q8 + 5], pkk[8 * q8 + 6], pkk[8 * q8 + 7]);
+                        } else {
+                            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                d4[q4] = make_uint4(pkk[4 * q4], pkk[4 * q4 + 1], pkk[4 * q4 + 2],
+                                                    pkk[4 * q4 + 3]);
+                        }
                     }
                 }
             }

@@ -102,3 +102,19 @@ def test_full_size_sampled_rows(name, layer):
     go = torch.stack([oc[b, i, h] for b, i, h in rows])
     gl = torch.stack([lc[b, h, i] for b, i, h in rows])
     check(go, ro, gl, rl, f"{name} {layer} sampled")
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_output_only_16_byte_aligned(d):
+    """The epilogue stores 32 bytes at a time when out is 32-byte aligned and
+    16 bytes otherwise; an output buffer offset by 16 bytes gives the same
+    bits as an aligned one."""
+    q, k, v = (t.cuda() for t in prefill_inputs(1, 200, 200, 4, 2, d, 1.0, 17))
+    ref, lse = g2.prefill(q, k, v, query_scale=d ** -0.5, window=70)
+    n = ref.numel()
+    buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    out = buf[8:8 + n].view(ref.shape)  # 16-byte aligned, not 32
+    assert out.data_ptr() % 32 == 16
+    g2.prefill(q, k, v, query_scale=d ** -0.5, window=70, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
