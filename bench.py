@@ -172,11 +172,27 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def aggregate_over_ranks(total_ms, nsteps, step_flops, world, device):
+    """Whole-job numbers of a replica run: every rank ran nsteps steps of
+    step_flops each; the job time is the slowest rank's device time (max over
+    ranks, one all-reduce). Returns (ms per step, TFLOP/s of all ranks)."""
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_per_step = float(t.item()) / nsteps
+    return ms_per_step, step_flops * world / (ms_per_step * 1e-3) / 1e12
+
+
+def replica_seed(base_seed, rank):
+    """Each replica draws its own inputs (independent units, no exchange)."""
+    return base_seed + rank
+
+
 def run_ours(args, rank, world, dev):
     import global_soft_capped_b200 as g2
     g2.load_library()
     w = WORKLOADS[WORKLOAD]
-    q, k, v = prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed + rank)
+    q, k, v = prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, replica_seed(w.seed, rank))
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     outs = {lay: torch.empty_like(qd) for lay in ("local", "global")}
     lses = {lay: torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
@@ -219,12 +235,7 @@ def run_ours(args, rank, world, dev):
     loc = [ev[i][0].elapsed_time(ev[i][1]) for i in range(nsteps)]
     glo = [ev[i][1].elapsed_time(ev[i][2]) for i in range(nsteps)]
     total_ms = sum(loc) + sum(glo)
-    total_ms_t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(total_ms_t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(total_ms_t.item())
-    ms_per_step = total_ms / nsteps
-    value = step_flops * world / (ms_per_step * 1e-3) / 1e12
+    ms_per_step, value = aggregate_over_ranks(total_ms, nsteps, step_flops, world, dev)
 
     pk, pk_kind = peaks()
     avg_loc, avg_glo = sum(loc) / nsteps, sum(glo) / nsteps
