@@ -317,7 +317,7 @@ int noalloc_scratch(void** out) {
 }
 
 // Backward: query-side positions padded to whole 64-position tiles in the
-// workspace (lse2 and D, fp32 each).
+// workspace (-lse*log2(e) and -D, fp32 each).
 long long bwd_tp(int T) { return (static_cast<long long>(T) + 63) / 64 * 64; }
 
 size_t bwd_ws_bytes(int B, int T, int H) {
@@ -350,7 +350,7 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
         return G2ATTN_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return G2ATTN_ERR_CUDA;
-    // D = dout . out and lse * log2(e) per (b, h, position)
+    // -D = -(dout . out) and -lse * log2(e) per (b, h, position)
     const long long rows = static_cast<long long>(P.B) * P.H * P.Tp;
     const long long threads = rows * (D / 8);
     const long long blocks = (threads + 255) / 256;
