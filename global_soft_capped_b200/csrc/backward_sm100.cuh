@@ -48,7 +48,7 @@ template <int D>
 struct BwCfg {
     static_assert(D == 64 || D == 128, "backward kernels are built for d = 64 and 128");
     static constexpr int TILE_BYTES = 128 * D * 2;         // one 128-row operand tile
-    static constexpr int VEC_BYTES = 2 * 128 * 4;          // lse2 and D of 128 query rows
+    static constexpr int VEC_BYTES = 2 * 128 * 4;          // -lse2 and -D of 128 query rows
     static constexpr int SLOT_BYTES = 2 * TILE_BYTES + VEC_BYTES;
     static constexpr int SMEM_TILES = 2 * TILE_BYTES + 2 * SLOT_BYTES;  // R1, R2, 2 column slots
     static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024;
