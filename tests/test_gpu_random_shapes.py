@@ -1,12 +1,14 @@
 """Seeded random shapes against the fp64 oracle (full tensors).
 
-A fixed generator draws dense, varlen and gradient cases. The ranges are:
+A fixed generator draws dense, varlen, gradient and decode cases. The ranges are:
 * head sizes 64 / 128 / 256, with d = 256 running on CTA pairs;
 * 1–3 KV heads with two query heads each, batch 1–3;
 * S up to 700, 1 <= T <= S, any valid q_offset;
 * no window, or any window size;
 * cap 50, 5 or off, several query scales;
-* varlen packings with empty and single-token sequences.
+* varlen packings with empty and single-token sequences;
+* decode from linear, ring (power-of-two slots >= window) and paged (16-256-row
+  blocks) caches, with 1-12 sequences of up to 3000 tokens.
 
 Each case is small enough for the oracle to finish in a second or two, and
 together they hit ragged tails, windows that start or end inside a tile, and
@@ -116,5 +118,52 @@ def test_random_backward(case):
         assert rel <= 1e-2 and mx <= 2e-2, (name, case, rel, mx)
 
 
-def test_device_error_word_clear():
+def _decode_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        layout = ("linear", "ring", "paged")[i % 3]
+        d = int(rng.choice([64, 128, 256]))
+        Hkv = int(rng.integers(1, 4))
+        lengths = [int(x) for x in rng.integers(1, 3001, size=int(rng.integers(1, 13)))]
+        if layout == "ring":
+            W = int(rng.integers(1, 2049))
+            R = 1 << int(np.ceil(np.log2(W)))  # a power of two >= the window
+        else:
+            W = 0 if rng.random() < 0.4 else int(rng.integers(1, 3000))
+            R = 0
+        bs = int(rng.choice([16, 32, 64, 128, 256]))
+        cap = float(rng.choice([50.0, 0.0]))
+        cases.append((layout, lengths, 2 * Hkv, Hkv, d, W, R, bs, cap, int(rng.integers(0, 1 << 30))))
+    return cases
+
+
+DECODE = _decode_cases(12, 5150)
+
+
+@pytest.mark.parametrize("case", DECODE, ids=[str(i) for i in range(len(DECODE))])
+def test_random_decode(case):
+    from test_gpu_decode_layouts import to_paged, to_ring
+    from global_soft_capped_b200.inputs import decode_inputs
+    layout, lengths, H, Hkv, d, W, R, bs, cap, seed = case
+    lengths, cu, q, k, v = decode_inputs(0, 0, 0, H, Hkv, d, seed=seed, lengths=lengths)
+    alpha = d ** -0.5
+    sl = torch.tensor(lengths, dtype=torch.int32)
+    if layout == "linear":
+        out, lse = g2.decode(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lengths),
+                             query_scale=alpha, softcap=cap, window=W)
+    elif layout == "ring":
+        kr, vr = to_ring(lengths, cu, k, R), to_ring(lengths, cu, v, R)
+        out, lse = g2.decode_ring(q.cuda(), kr.cuda(), vr.cuda(), sl.cuda(), W,
+                                  query_scale=alpha, softcap=cap)
+    else:
+        kb, vb, table = to_paged(lengths, cu, k, v, bs, seed=seed % 1000)
+        out, lse = g2.decode_paged(q.cuda(), kb.cuda(), vb.cuda(), table.cuda(), sl.cuda(),
+                                   max(lengths), query_scale=alpha, softcap=cap, window=W)
+    torch.cuda.synchronize()
+    ro, rl = oracle.decode(q, k, v, cu, query_scale=alpha, softcap=cap, window=W)
+    check(out, ro, lse, rl, what=str(case))
+
+
+def test_zz_device_error_word_clear():
     assert g2.g2attn_get_device_error() == g2.G2ATTN_OK
