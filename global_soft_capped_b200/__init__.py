@@ -6,7 +6,8 @@ Two layers:
   ``g2attn_prefill_varlen``, ``g2attn_prefill_paged``, ``g2attn_decode_workspace_size``,
   ``g2attn_decode``, ``g2attn_decode_ring``, ``g2attn_decode_paged``,
   ``g2attn_decode_noalloc``, ``g2attn_backward_workspace_size``,
-  ``g2attn_prefill_backward``, ``g2attn_status_string``,
+  ``g2attn_prefill_backward``, ``g2attn_varlen_backward_workspace_size``,
+  ``g2attn_prefill_varlen_backward``, ``g2attn_status_string``,
   ``g2attn_get_device_error``,
   ``g2attn_selftest_wait_timeout``): plain argument marshalling of integers,
   floats and raw pointers through ctypes, returning the status code.
@@ -46,6 +47,8 @@ EXPORTS = (
     "g2attn_decode_noalloc",
     "g2attn_backward_workspace_size",
     "g2attn_prefill_backward",
+    "g2attn_varlen_backward_workspace_size",
+    "g2attn_prefill_varlen_backward",
     "g2attn_status_string",
     "g2attn_get_device_error",
     "g2attn_selftest_wait_timeout",
@@ -92,6 +95,10 @@ def load_library():
     lib.g2attn_backward_workspace_size.restype = SZ
     lib.g2attn_prefill_backward.argtypes = [P] * 9 + [I] * 7 + [F, F, I, P, SZ, P]
     lib.g2attn_prefill_backward.restype = I
+    lib.g2attn_varlen_backward_workspace_size.argtypes = [I, I, I]
+    lib.g2attn_varlen_backward_workspace_size.restype = SZ
+    lib.g2attn_prefill_varlen_backward.argtypes = [P] * 11 + [I] * 8 + [F, F, I, P, SZ, P]
+    lib.g2attn_prefill_varlen_backward.restype = I
     lib.g2attn_status_string.argtypes = [I]
     lib.g2attn_status_string.restype = ctypes.c_char_p
     lib.g2attn_get_device_error.argtypes = []
@@ -137,6 +144,20 @@ def g2attn_prefill_backward(q, k, v, out, lse, dout, dq, dk, dv, B, T, S, H, Hkv
     return load_library().g2attn_prefill_backward(q, k, v, out, lse, dout, dq, dk, dv, B, T, S,
                                                   H, Hkv, d, q_offset, query_scale, softcap,
                                                   window, workspace, workspace_bytes, stream)
+
+
+def g2attn_varlen_backward_workspace_size(num_seqs, total_q, H):
+    return load_library().g2attn_varlen_backward_workspace_size(num_seqs, total_q, H)
+
+
+def g2attn_prefill_varlen_backward(q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q,
+                                   cu_seqlens_k, num_seqs, total_q, total_k, max_T, max_S, H,
+                                   Hkv, d, query_scale, softcap, window, workspace,
+                                   workspace_bytes, stream):
+    return load_library().g2attn_prefill_varlen_backward(
+        q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
+        total_k, max_T, max_S, H, Hkv, d, query_scale, softcap, window, workspace,
+        workspace_bytes, stream)
 
 
 def g2attn_decode_workspace_size(num_seqs, H, d, max_cache_len):
@@ -282,6 +303,31 @@ def prefill_backward(q, k, v, out, lse, dout, *, q_offset=0, query_scale=1.0, so
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     if st != G2ATTN_OK:
         raise G2AttnError(st, "g2attn_prefill_backward")
+    return dq, dk, dv
+
+
+def prefill_varlen_backward(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_T, max_S,
+                            *, query_scale=1.0, softcap=50.0, window=0, workspace=None, dq=None,
+                            dk=None, dv=None, stream=None):
+    """Gradients of :func:`prefill_varlen`: returns (dq, dk, dv), packed like q, k, v."""
+    import torch
+    _check_bf16(q, k, v, out, dout)
+    total_q, H, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    num_seqs = cu_seqlens_q.numel() - 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        n = g2attn_varlen_backward_workspace_size(num_seqs, total_q, H)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    st = g2attn_prefill_varlen_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), num_seqs, total_q, total_k,
+        int(max_T), int(max_S), H, Hkv, d, float(query_scale), float(softcap), int(window),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != G2ATTN_OK:
+        raise G2AttnError(st, "g2attn_prefill_varlen_backward")
     return dq, dk, dv
 
 

@@ -369,9 +369,122 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
     return launch_bwd<D, g2::BW_Q>(mq, mo, mk, mv, P, q_tiles * BG, sms, st);
 }
 
+// Varlen backward workspace: -lse2 and -D as (H, wmax) fp32 each, then the
+// int prefix wq[num_seqs + 1]. wmax bounds the padded query count.
+long long bwd_vl_wmax(int num_seqs, int total_q) {
+    return (static_cast<long long>(total_q) + 64ll * num_seqs + 63) / 64 * 64;
+}
+
+size_t bwd_vl_ws_bytes(int num_seqs, int total_q, int H) {
+    return 2ull * H * bwd_vl_wmax(num_seqs, total_q) * sizeof(float) +
+           (static_cast<size_t>(num_seqs) + 1) * sizeof(int);
+}
+
+template <int D>
+int launch_backward_varlen(const void* q, const void* k, const void* v, const void* out,
+                           const float* lse, const void* dout, int total_q, int total_k,
+                           g2::BwParams& P, cudaStream_t st) {
+    CUtensorMap mq, mo, mk, mv;
+    if (!make_map(&mq, q, D, total_q, P.H, g2::BW_QPOS, 2) ||
+        !make_map(&mo, dout, D, total_q, P.H, g2::BW_QPOS, 2) ||
+        !make_map(&mk, k, D, total_k, P.Hkv, g2::BW_KEYS, 1) ||
+        !make_map(&mv, v, D, total_k, P.Hkv, g2::BW_KEYS, 1))
+        return G2ATTN_ERR_CUDA;
+    const int sms = num_sms();
+    if (sms <= 0) return G2ATTN_ERR_CUDA;
+    g2::bwd_wq_prefix<<<1, 32, 0, st>>>(P.cu_q, P.num_seqs, total_q, const_cast<int*>(P.wq));
+    if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
+    const long long threads = static_cast<long long>(P.H) * P.wmax * (D / 8);
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    g2::bwd_prep_varlen<D><<<static_cast<int>(blocks), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse,
+        P.cu_q, P.wq, const_cast<float*>(P.nlse2), const_cast<float*>(P.ndvec), P.num_seqs, P.H,
+        total_q, P.wmax);
+    if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
+    // Units are counted on the device from cu_seqlens; the grids come from
+    // upper bounds and surplus units are skipped by the kernels.
+    const long long kv_ub = (static_cast<long long>(total_k) / g2::BW_KEYS + P.num_seqs) * P.Hkv;
+    const long long q_ub = (static_cast<long long>(total_q) / g2::BW_QPOS + P.num_seqs) * P.Hkv;
+    if (kv_ub > INT32_MAX || q_ub > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    int rc = launch_bwd<D, g2::BW_KV>(mq, mo, mk, mv, P, static_cast<int>(kv_ub), sms, st);
+    if (rc) return rc;
+    return launch_bwd<D, g2::BW_Q>(mq, mo, mk, mv, P, static_cast<int>(q_ub), sms, st);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t g2attn_varlen_backward_workspace_size(int num_seqs, int total_q, int H) {
+    if (num_seqs <= 0 || total_q <= 0 || H <= 0) return 0;
+    return bwd_vl_ws_bytes(num_seqs, total_q, H);
+}
+
+int g2attn_prefill_varlen_backward(const void* q, const void* k, const void* v, const void* out,
+                                   const float* lse, const void* dout, void* dq, void* dk,
+                                   void* dv, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                   int num_seqs, int total_q, int total_k, int max_T, int max_S,
+                                   int H, int Hkv, int d, float query_scale, float softcap,
+                                   int window, void* workspace, size_t workspace_bytes,
+                                   g2attn_stream_t stream) {
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !cu_seqlens_q ||
+        !cu_seqlens_k)
+        return G2ATTN_ERR_INVALID_ARG;
+    if (num_seqs <= 0 || total_q <= 0 || total_k <= 0 || max_T <= 0 || max_S <= 0 ||
+        max_T > max_S || max_T > total_q || max_S > total_k)
+        return G2ATTN_ERR_INVALID_ARG;
+    int rc = check_common(H, Hkv, d, query_scale, softcap, window);
+    if (rc) return rc;
+    if (d != 64 && d != 128) return G2ATTN_ERR_UNSUPPORTED;
+    if (num_seqs > g2::BwCfg<64>::MAX_SEQ_TABLE) return G2ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+        return G2ATTN_ERR_MISALIGNED;
+    if (static_cast<long long>(H) * bwd_vl_wmax(num_seqs, total_q) > INT32_MAX)
+        return G2ATTN_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < bwd_vl_ws_bytes(num_seqs, total_q, H))
+        return G2ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return G2ATTN_ERR_MISALIGNED;
+    g2::BwParams P{};
+    P.dq = static_cast<__nv_bfloat16*>(dq);
+    P.dk = static_cast<__nv_bfloat16*>(dk);
+    P.dv = static_cast<__nv_bfloat16*>(dv);
+    P.B = 1;
+    P.T = max_T;
+    P.S = max_S;
+    P.H = H;
+    P.Hkv = Hkv;
+    P.window = window;
+    P.varlen = 1;
+    P.num_seqs = num_seqs;
+    P.cu_q = cu_seqlens_q;
+    P.cu_k = cu_seqlens_k;
+    P.total_q = total_q;
+    P.total_k = total_k;
+    P.wmax = static_cast<int>(bwd_vl_wmax(num_seqs, total_q));
+    float* ws = static_cast<float*>(workspace);
+    P.nlse2 = ws;
+    P.ndvec = ws + static_cast<size_t>(H) * P.wmax;
+    P.wq = reinterpret_cast<const int*>(ws + 2 * static_cast<size_t>(H) * P.wmax);
+    int has_cap = 0;
+    fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, has_cap);
+    P.has_cap = has_cap;
+    P.query_scale = query_scale;
+    {  // the same series window as the forward's fast path
+        g2::PfParams F{};
+        fill_poly(query_scale, softcap, F);
+        P.u_scale = F.u_scale;
+        P.poly_acc_max = F.poly_acc_max;
+    }
+    P.timeout_ns = wait_limit_ns();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 64)
+        return launch_backward_varlen<64>(q, k, v, out, lse, dout, total_q, total_k, P, st);
+    return launch_backward_varlen<128>(q, k, v, out, lse, dout, total_q, total_k, P, st);
+}
 
 size_t g2attn_backward_workspace_size(int B, int T, int H) {
     if (B <= 0 || T <= 0 || H <= 0) return 0;
@@ -494,6 +607,7 @@ int g2attn_prefill_varlen(const void* q, const void* k, const void* v, void* out
     P.window = window;
     P.varlen = 1;
     P.total_q = total_q;
+    P.total_k = total_k;
     // Units are enumerated on the device from cu_seqlens_q; the grid is sized
     // from an upper bound and surplus units are skipped by the kernel.
     const long long ub = (static_cast<long long>(total_q) / g2::PF_QPOS + num_seqs) * Hkv;

@@ -51,7 +51,9 @@ struct BwCfg {
     static constexpr int VEC_BYTES = 2 * 128 * 4;          // -lse2 and -D of 128 query rows
     static constexpr int SLOT_BYTES = 2 * TILE_BYTES + VEC_BYTES;
     static constexpr int SMEM_TILES = 2 * TILE_BYTES + 2 * SLOT_BYTES;  // R1, R2, 2 column slots
-    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024;
+    static constexpr int MAX_SEQ_TABLE = 1024;                  // varlen: sequences per launch
+    static constexpr int VL_BYTES = 4 * (MAX_SEQ_TABLE + 1);    // unit prefix over sequences
+    static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + VL_BYTES;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -59,10 +61,19 @@ struct BwParams {
     __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
-    const float* nlse2;  // (B, H, Tp): -lse * log2(e); -inf at positions >= T
-    const float* ndvec;  // (B, H, Tp): -D = -(dout . out); 0 at positions >= T
+    // -lse * log2(e) and -D = -(dout . out) per (head, query position), with
+    // each sequence's positions padded to whole 64-position tiles (-inf / 0):
+    // dense (B, H, Tp); varlen (H, Wmax), sequence s at columns wq[s] ..
+    const float* nlse2;
+    const float* ndvec;
     int B, T, S, H, Hkv, Tp;
     int q_offset, window;
+    // varlen (packed sequences): T_s, S_s from cu_q / cu_k, q_offset_s = S_s - T_s
+    const int* cu_q;
+    const int* cu_k;
+    const int* wq;  // [num_seqs + 1] padded prefix of T_s (workspace columns)
+    int num_seqs, varlen, wmax;
+    int total_q, total_k;  // packed extents: sequence rows are clamped into them
     int num_units;
     int row_tiles;      // KV: key tiles per (b, g); Q: query tiles per (b, g)
     float k_exp;        // 2 alpha log2(e) / C   (cap on)
@@ -86,38 +97,80 @@ __device__ __forceinline__ float bw_tanh_series(float u) {
 }
 
 struct BwUnit {
-    int b, g;
+    int g;
+    int T, S, qoff;   // the sequence: queries, keys, position of query 0
+    int qbase, kbase; // packed row of its first query / key
+    long long wbase;  // workspace column of its position 0 for head 0 ...
+    long long wstride;  // ... and the stride between heads
     int row0;     // KV: first key; Q: first query position (row index t within the sequence)
     int rvalid;   // KV: keys in the tile (<= 128); Q: positions in the tile (<= 64)
     int col0;     // first column tile index (KV: 64-position tiles; Q: 128-key tiles)
     int ncols;    // column tiles (0: no visible pair; KV units then store zeros)
 };
 
-// KV units: key tiles ascending (the earliest keys see the most queries), then
-// batch, then KV head. Q units: query tiles descending, then batch, then head.
+// Rows [*base, *base + *len) of sequence s in a packed tensor of `total` rows
+// described by cu[]: clamped into [0, total), so that malformed offsets can
+// give wrong results but never an access outside the tensors.
+__device__ __forceinline__ void bw_seq_rows(const int* cu, int s, int total, int* base,
+                                            int* len) {
+    const int b0 = min(max(cu[s], 0), total);
+    const int b1 = min(max(cu[s + 1], b0), total);
+    *base = b0;
+    *len = b1 - b0;
+}
+
+// Units. Dense: KV units take key tiles ascending (the earliest keys see the
+// most queries), then batch, then KV head; Q units take query tiles
+// descending, then batch, then head. Varlen: sequence by sequence (the unit
+// prefix `cum` over sequences), within a sequence as dense.
 template <int MODE>
-__device__ __forceinline__ void bw_unit(const BwParams& P, int u, BwUnit& U) {
-    const int BG = P.B * P.Hkv;
-    const int rt = u / BG, rem = u % BG;
-    U.b = rem / P.Hkv;
-    U.g = rem % P.Hkv;
+__device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, int u, BwUnit& U) {
+    int rt, tiles;
+    if (!P.varlen) {
+        const int BG = P.B * P.Hkv;
+        rt = u / BG;
+        const int rem = u % BG, b = rem / P.Hkv;
+        U.g = rem % P.Hkv;
+        U.T = P.T;
+        U.S = P.S;
+        U.qoff = P.q_offset;
+        U.qbase = b * P.T;
+        U.kbase = b * P.S;
+        U.wbase = static_cast<long long>(b) * P.H * P.Tp;
+        U.wstride = P.Tp;
+        tiles = P.row_tiles;
+    } else {
+        int lo = 0, hi = P.num_seqs - 1;  // largest s with cum[s] <= u
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cum[mid] <= u) lo = mid; else hi = mid - 1;
+        }
+        const int s = lo, lu = u - cum[s];
+        U.g = lu % P.Hkv;
+        rt = lu / P.Hkv;
+        bw_seq_rows(P.cu_q, s, P.total_q, &U.qbase, &U.T);
+        bw_seq_rows(P.cu_k, s, P.total_k, &U.kbase, &U.S);
+        U.qoff = U.S - U.T;
+        U.wbase = P.wq[s];
+        U.wstride = P.wmax;
+        tiles = MODE == BW_KV ? (U.S + BW_KEYS - 1) / BW_KEYS : (U.T + BW_QPOS - 1) / BW_QPOS;
+    }
     if (MODE == BW_KV) {
         U.row0 = rt * BW_KEYS;
-        U.rvalid = min(BW_KEYS, P.S - U.row0);
-        // query rows t whose position t + q_offset sees a key of the tile
-        const int t_lo = max(0, U.row0 - P.q_offset);
-        const int t_hi = P.window > 0
-                             ? min(P.T - 1, U.row0 + BW_KEYS - 1 + P.window - 1 - P.q_offset)
-                             : P.T - 1;
+        U.rvalid = min(BW_KEYS, U.S - U.row0);
+        // query rows t whose position t + qoff sees a key of the tile
+        const int t_lo = max(0, U.row0 - U.qoff);
+        const int t_hi = P.window > 0 ? min(U.T - 1, U.row0 + BW_KEYS - 1 + P.window - 1 - U.qoff)
+                                      : U.T - 1;
         U.col0 = t_lo / BW_QPOS;
         U.ncols = (t_lo <= t_hi) ? t_hi / BW_QPOS - U.col0 + 1 : 0;
     } else {
-        const int qt = P.row_tiles - 1 - rt;
+        const int qt = tiles - 1 - rt;
         U.row0 = qt * BW_QPOS;
-        U.rvalid = min(BW_QPOS, P.T - U.row0);
-        const int p_min = U.row0 + P.q_offset, p_max = p_min + U.rvalid - 1;
+        U.rvalid = min(BW_QPOS, U.T - U.row0);
+        const int p_min = U.row0 + U.qoff, p_max = p_min + U.rvalid - 1;
         const int j_lo = P.window > 0 ? max(0, p_min - P.window + 1) : 0;
-        const int j_hi = min(p_max, P.S - 1);
+        const int j_hi = min(p_max, U.S - 1);
         U.col0 = j_lo / BW_KEYS;
         U.ncols = j_hi / BW_KEYS - U.col0 + 1;
     }
@@ -159,6 +212,80 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict_
     if (in_range && sub == 0) {
         ndvec[row] = -acc;
         nlse2[row] = (t < T) ? lse[bh * T + t] * -1.4426950408889634f : -INFINITY;
+    }
+}
+
+// Varlen: wq[s] = sum over s' < s of T_s' rounded up to 64 (the workspace
+// column where sequence s starts), wq[num_seqs] = the total. One block.
+__global__ void __launch_bounds__(32) bwd_wq_prefix(const int* __restrict__ cu_q, int num_seqs,
+                                                    int total_q, int* wq) {
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int s0 = 0; s0 < num_seqs; s0 += 32) {
+        const int q = s0 + lane;
+        int qb = 0, t = 0;
+        if (q < num_seqs) bw_seq_rows(cu_q, q, total_q, &qb, &t);
+        const int x = (t + 63) / 64 * 64;
+        int incl = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (q < num_seqs) wq[q] = carry + incl - x;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) wq[num_seqs] = carry;
+}
+
+// Varlen form of bwd_prep over workspace columns w in [0, wmax) of every head:
+// sequence s owns columns wq[s] .. wq[s+1]-1 (its positions, then padding);
+// lse is (H, total_q) packed. Columns past wq[num_seqs] are left untouched.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_varlen(
+    const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const int* __restrict__ cu_q, const int* __restrict__ wq,
+    float* nlse2, float* ndvec, int num_seqs, int H, int total_q, int wmax) {
+    constexpr int LPR = D / 8;  // lanes per row
+    const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / LPR;
+    const int sub = threadIdx.x % LPR;
+    const long long nrows = static_cast<long long>(H) * wmax;
+    const int w = static_cast<int>(row % wmax);
+    const int h = static_cast<int>(row / wmax);
+    const bool in_range = row < nrows && w < wq[num_seqs];  // whole warp shuffles below
+    int s = 0;
+    if (in_range) {  // largest s with wq[s] <= w
+        int lo = 0, hi = num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (wq[mid] <= w) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+    }
+    int qb = 0, tl = 0;
+    if (in_range) bw_seq_rows(cu_q, s, total_q, &qb, &tl);
+    const int t = in_range ? w - wq[s] : 0;
+    const bool valid = in_range && t < tl;
+    const long long prow = valid ? static_cast<long long>(qb) + t : 0;
+    float acc = 0.f;
+    if (valid) {
+        const size_t off = (static_cast<size_t>(prow) * H + h) * D + sub * 8;
+        const uint4 o = *reinterpret_cast<const uint4*>(out + off);
+        const uint4 g = *reinterpret_cast<const uint4*>(dout + off);
+        const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc = fmaf(__uint_as_float(ow[i] << 16), __uint_as_float(gw[i] << 16), acc);
+            acc = fmaf(__uint_as_float(ow[i] & 0xFFFF0000u), __uint_as_float(gw[i] & 0xFFFF0000u),
+                       acc);
+        }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (in_range && sub == 0) {
+        ndvec[row] = -acc;
+        nlse2[row] = valid ? lse[static_cast<size_t>(h) * total_q + prow] * -1.4426950408889634f
+                           : -INFINITY;
     }
 }
 
@@ -231,6 +358,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* drain = bars + 12;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);  // varlen unit prefix
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -251,6 +379,32 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (P.varlen) {  // units of each sequence (Hkv x its row tiles), then an exclusive scan
+        const int ns = P.num_seqs;
+        for (int q = threadIdx.x; q < ns; q += blockDim.x) {
+            int qb, t, kb, sk;
+            bw_seq_rows(P.cu_q, q, P.total_q, &qb, &t);
+            bw_seq_rows(P.cu_k, q, P.total_k, &kb, &sk);
+            cum[q] = P.Hkv * (KV ? (sk + BW_KEYS - 1) / BW_KEYS : (t + BW_QPOS - 1) / BW_QPOS);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int carry = 0;
+            for (int s0 = 0; s0 < ns; s0 += 32) {
+                const int q = s0 + lane;
+                const int x = (q < ns) ? cum[q] : 0;
+                int incl = x;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += y;
+                }
+                if (q < ns) cum[q] = carry + incl - x;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) cum[ns] = carry;
+        }
+    }
     if (warp == BW_WARP_MMA) {
         tmem_alloc(tmem_holder, BW_TMEM_COLS);
         tmem_relinquish();
@@ -268,6 +422,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const int G = gridDim.x;
     const int cta = blockIdx.x;
     const uint64_t lim = P.timeout_ns;
+    const int num_units = P.varlen ? min(P.num_units, cum[P.num_seqs]) : P.num_units;
 
     if (warp == BW_WARP_PRODUCER) {
         // ------------------------------------------------------------ producer
@@ -275,11 +430,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             uint32_t ct = 0;  // column tiles loaded so far
             int uw = 0;       // units with work so far
             bool ok = true;
-            for (int r = 0; ok && r * G < P.num_units; ++r) {
+            for (int r = 0; ok && r * G < num_units; ++r) {
                 const int u = bw_sched(r, cta, G);
-                if (u >= P.num_units) continue;
+                if (u >= num_units) continue;
                 BwUnit U;
-                bw_unit<MODE>(P, u, U);
+                bw_unit<MODE>(P, cum, u, U);
                 if (U.ncols == 0) continue;
                 if (uw > 0) {
                     ok = mbar_wait(r_empty, (uw - 1) & 1, abort_flag, lim, SITE_BW_PROD);
@@ -287,11 +442,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
                 mbar_arrive_expect_tx(r_full, 2 * C::TILE_BYTES);
                 if (KV) {
-                    bw_load_tile<D>(sR1, &tmK, r_full, U.b * P.S + U.row0, U.g);
-                    bw_load_tile<D>(sR2, &tmV, r_full, U.b * P.S + U.row0, U.g);
+                    bw_load_tile<D>(sR1, &tmK, r_full, U.kbase + U.row0, U.g);
+                    bw_load_tile<D>(sR2, &tmV, r_full, U.kbase + U.row0, U.g);
                 } else {
-                    bw_load_tile<D>(sR1, &tmQ, r_full, U.b * P.T + U.row0, 2 * U.g);
-                    bw_load_tile<D>(sR2, &tmO, r_full, U.b * P.T + U.row0, 2 * U.g);
+                    bw_load_tile<D>(sR1, &tmQ, r_full, U.qbase + U.row0, 2 * U.g);
+                    bw_load_tile<D>(sR2, &tmO, r_full, U.qbase + U.row0, 2 * U.g);
                 }
                 for (int c = 0; c < U.ncols; ++c) {
                     const int sl = ct & 1;
@@ -302,23 +457,23 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (KV) {
                         const int t0 = (U.col0 + c) * BW_QPOS;
                         mbar_arrive_expect_tx(&c_full[sl], 2 * C::TILE_BYTES + C::VEC_BYTES);
-                        bw_load_tile<D>(slot, &tmQ, &c_full[sl], U.b * P.T + t0, 2 * U.g);
-                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmO, &c_full[sl], U.b * P.T + t0,
+                        bw_load_tile<D>(slot, &tmQ, &c_full[sl], U.qbase + t0, 2 * U.g);
+                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmO, &c_full[sl], U.qbase + t0,
                                         2 * U.g);
                         // -lse2 and -D of the tile's 128 query rows (head 2g, then 2g+1)
                         float* vec = reinterpret_cast<float*>(slot + 2 * C::TILE_BYTES);
 #pragma unroll
                         for (int hl = 0; hl < 2; ++hl) {
-                            const size_t off =
-                                (static_cast<size_t>(U.b) * P.H + 2 * U.g + hl) * P.Tp + t0;
+                            const size_t off = static_cast<size_t>(U.wbase) +
+                                               (2 * U.g + hl) * U.wstride + t0;
                             bulk_load(vec + hl * 64, P.nlse2 + off, 256, &c_full[sl]);
                             bulk_load(vec + 128 + hl * 64, P.ndvec + off, 256, &c_full[sl]);
                         }
                     } else {
                         const int key0 = (U.col0 + c) * BW_KEYS;
                         mbar_arrive_expect_tx(&c_full[sl], 2 * C::TILE_BYTES);
-                        bw_load_tile<D>(slot, &tmK, &c_full[sl], U.b * P.S + key0, U.g);
-                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmV, &c_full[sl], U.b * P.S + key0,
+                        bw_load_tile<D>(slot, &tmK, &c_full[sl], U.kbase + key0, U.g);
+                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmV, &c_full[sl], U.kbase + key0,
                                         U.g);
                     }
                     ++ct;
@@ -401,11 +556,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             // XY_0(c+1) | z_1 | ACC_1(c) XY_1(c+1). A half's X / Y overwrite
             // that half's P / dS only after the accumulation reading them was
             // issued; UMMAs of one thread execute in issue order.
-            for (int r = 0; ok && r * G < P.num_units; ++r) {
+            for (int r = 0; ok && r * G < num_units; ++r) {
                 const int u = bw_sched(r, cta, G);
-                if (u >= P.num_units) continue;
+                if (u >= num_units) continue;
                 BwUnit U;
-                bw_unit<MODE>(P, u, U);
+                bw_unit<MODE>(P, cum, u, U);
                 if (U.ncols == 0) continue;
                 ok = mbar_wait(r_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
@@ -465,16 +620,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         uint32_t ct = 0;
         int uw = 0;
         bool ok = true;
-        for (int rr = 0; ok && rr * G < P.num_units; ++rr) {
+        for (int rr = 0; ok && rr * G < num_units; ++rr) {
             const int u = bw_sched(rr, cta, G);
-            if (u >= P.num_units) continue;
+            if (u >= num_units) continue;
             BwUnit U;
-            bw_unit<MODE>(P, u, U);
+            bw_unit<MODE>(P, cum, u, U);
             if (U.ncols == 0) {
                 // keys that no query sees: zero gradients (KV mode only; every
                 // query sees at least its own key)
                 if (KV && r < U.rvalid) {
-                    const size_t row = (static_cast<size_t>(U.b) * P.S + U.row0 + r) * P.Hkv + U.g;
+                    const size_t row = (static_cast<size_t>(U.kbase) + U.row0 + r) * P.Hkv + U.g;
 #pragma unroll
                     for (int c = 0; c < D / 2; c += 8) {
                         *reinterpret_cast<uint4*>(P.dv + row * D + part * (D / 2) + c) =
@@ -489,9 +644,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const int hl_row = r >> 6, pr_row = r & 63;
             const int t_row = U.row0 + pr_row;  // Q mode
             float row_nl2 = -INFINITY, row_nd = 0.f;
-            if (!KV && t_row < P.T) {
+            if (!KV && t_row < U.T) {
                 const size_t off =
-                    (static_cast<size_t>(U.b) * P.H + 2 * U.g + hl_row) * P.Tp + t_row;
+                    static_cast<size_t>(U.wbase) + (2 * U.g + hl_row) * U.wstride + t_row;
                 row_nl2 = P.nlse2[off];
                 row_nd = P.ndvec[off];
             }
@@ -518,8 +673,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         j_lo = ccol0;  j_hi = ccol0 + BW_KEYS - 1;
                         t_lo = U.row0; t_hi = U.row0 + BW_QPOS - 1;
                     }
-                    interior = j_hi <= t_lo + P.q_offset && t_hi < P.T && j_hi < P.S &&
-                               (P.window == 0 || t_hi + P.q_offset - j_lo < P.window);
+                    interior = j_hi <= t_lo + U.qoff && t_hi < U.T && j_hi < U.S &&
+                               (P.window == 0 || t_hi + U.qoff - j_lo < P.window);
                 }
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {  // two chunks of 32 columns
@@ -615,10 +770,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                 }
                                 const float nl2 = e ? nl2v.y : nl2v.x;
                                 const float nd = e ? ndv.y : ndv.x;
-                                const int pos = t + P.q_offset;
+                                const int pos = t + U.qoff;
                                 const bool vis = (j <= pos) &&
                                                  (P.window == 0 || pos - j < P.window) &&
-                                                 (t < P.T) && (j < P.S);
+                                                 (t < U.T) && (j < U.S);
                                 const float x = __uint_as_float(xv[i + e]);
                                 float s2, dcap;
                                 if (P.has_cap) {
@@ -671,7 +826,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             constexpr int HALF = D / 2;  // accumulator columns per warp
             if (KV) {
                 const bool valid = r < U.rvalid;
-                const size_t row = (static_cast<size_t>(U.b) * P.S + key_row) * P.Hkv + U.g;
+                const size_t row = (static_cast<size_t>(U.kbase) + key_row) * P.Hkv + U.g;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {  // a = 0: dv (columns 0..), a = 1: dk (columns D..)
                     const float f = a ? P.query_scale : 1.0f;
@@ -680,7 +835,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
             } else {
                 const bool valid = pr_row < U.rvalid;
-                const size_t row = (static_cast<size_t>(U.b) * P.T + t_row) * P.H + 2 * U.g + hl_row;
+                const size_t row = (static_cast<size_t>(U.qbase) + t_row) * P.H + 2 * U.g + hl_row;
                 __nv_bfloat16* dst = P.dq + row * D + part * HALF;
                 bw_store_acc<HALF>(tmem + lane_addr + part * HALF, dst, P.query_scale, valid);
             }

@@ -97,6 +97,7 @@ struct PfParams {
     int kv_block_shift, kv_max_blocks, kv_num_blocks;
     int paged;
     int total_q;      // packed query rows (dense: B*T); lse head stride for varlen
+    int total_k;      // packed key rows (varlen, packed K/V)
     int num_units;
     int max_units_per_seq_tiles;  // dense: q tiles per sequence
     float k_exp;    // 2*alpha*log2(e)/C   (cap on)
@@ -132,6 +133,17 @@ struct VlTables {
     int* order;  // [num_seqs] sequences ranked by work, descending
     int* cum;    // [num_seqs + 1] units before each ranked sequence; cum[num_seqs] = total
 };
+
+// Rows [*base, *base + *len) of sequence s in a packed tensor of `total` rows
+// described by cu[]: clamped into [0, total), so that malformed offsets can
+// give wrong results but never an access outside the tensor.
+__device__ __forceinline__ void pf_seq_rows(const int* cu, int s, int total, int* base,
+                                            int* len) {
+    const int b0 = min(max(cu[s], 0), total);
+    const int b1 = min(max(cu[s + 1], b0), total);
+    *base = b0;
+    *len = b1 - b0;
+}
 
 // KV tiles visited by query tile t0 of a sequence (T queries at the end of S keys).
 __device__ __forceinline__ int pf_tiles(int t0, int T, int S, int window) {
@@ -174,14 +186,12 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, in
         }
         seq = V.order[lo];
         const int lu = u - V.cum[lo];
-        qbase = P.cu_q[seq];
-        Tq = P.cu_q[seq + 1] - qbase;
+        pf_seq_rows(P.cu_q, seq, P.total_q, &qbase, &Tq);
         if (P.paged) {
             kbase = 0;
             Sk = max(Tq, min(P.kv_lens[seq], P.kv_max_blocks << P.kv_block_shift));
         } else {
-            kbase = P.cu_k[seq];
-            Sk = P.cu_k[seq + 1] - kbase;
+            pf_seq_rows(P.cu_k, seq, P.total_k, &kbase, &Sk);
         }
         const int nq = (Tq + QT - 1) / QT;
         U.g = lu % P.Hkv;
@@ -284,9 +294,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     if (P.varlen) {  // per-launch schedule (see VlTables)
         const int ns = P.num_seqs;
         for (int s = threadIdx.x; s < ns; s += blockDim.x) {
-            const int t = max(0, P.cu_q[s + 1] - P.cu_q[s]);
+            int qb, t, kb = 0, skr = 0;
+            pf_seq_rows(P.cu_q, s, P.total_q, &qb, &t);
+            if (!P.paged) pf_seq_rows(P.cu_k, s, P.total_k, &kb, &skr);
             const int sk = max(t, P.paged ? min(P.kv_lens[s], P.kv_max_blocks << P.kv_block_shift)
-                                          : P.cu_k[s + 1] - P.cu_k[s]);
+                                          : skr);
             int w = 0;
             for (int t0 = 0; t0 < t; t0 += PF_QPOS) w += pf_tiles(t0, t, sk, P.window);
             vt.work[s] = w;
@@ -304,7 +316,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         __syncthreads();
         for (int r = threadIdx.x; r < ns; r += blockDim.x) {
             const int s = vt.order[r];
-            const int t = max(0, P.cu_q[s + 1] - P.cu_q[s]);
+            int qb, t;
+            pf_seq_rows(P.cu_q, s, P.total_q, &qb, &t);
             vt.cum[r] = P.Hkv * ((t + CG * PF_QPOS - 1) / (CG * PF_QPOS));
         }
         __syncthreads();

@@ -256,6 +256,36 @@ G2ATTN_API int g2attn_prefill_backward(const void* q, const void* k, const void*
                             int q_offset, float query_scale, float softcap, int window,
                             void* workspace, size_t workspace_bytes, g2attn_stream_t stream);
 
+/*
+ * Bytes of device workspace g2attn_prefill_varlen_backward needs: -lse*log2(e)
+ * and -D per (head, query position) with every sequence padded to a multiple
+ * of 64 positions (bounded by total_q + 64*num_seqs per head), plus
+ * num_seqs + 1 ints. 0 for non-positive arguments.
+ */
+G2ATTN_API size_t g2attn_varlen_backward_workspace_size(int num_seqs, int total_q, int H);
+
+/*
+ * Gradients of g2attn_prefill_varlen: the packed layout, cu_seqlens and limits
+ * of that call, with out and lse its outputs (lse (H, total_q) fp32) and dout
+ * packed like q.
+ *   dq like q, dk and dv like k and v (bf16), written in full.
+ *   workspace: at least g2attn_varlen_backward_workspace_size(num_seqs,
+ *     total_q, H) bytes, 16-byte aligned, overwritten.
+ * Sequence rows derived from cu_seqlens are clamped into [0, total_q) and
+ * [0, total_k): malformed offsets give undefined results but no access
+ * outside the tensors. Supported: d = 64 and 128; num_seqs <= 1024.
+ * Other errors as g2attn_prefill_backward. Four kernels run on `stream`: the
+ * padded-prefix and D passes, the dk/dv kernel and the dq kernel.
+ * Source: as g2attn_prefill_backward; the packing is this library's.
+ */
+G2ATTN_API int g2attn_prefill_varlen_backward(const void* q, const void* k, const void* v,
+                                   const void* out, const float* lse, const void* dout,
+                                   void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                                   const int* cu_seqlens_k, int num_seqs, int total_q,
+                                   int total_k, int max_T, int max_S, int H, int Hkv, int d,
+                                   float query_scale, float softcap, int window, void* workspace,
+                                   size_t workspace_bytes, g2attn_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 G2ATTN_API const char* g2attn_status_string(int status);
 

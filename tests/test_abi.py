@@ -178,3 +178,38 @@ def backward_args(**kw):
 ])
 def test_backward_rejects_before_launch(lib, kw, status):
     assert g2.g2attn_prefill_backward(*backward_args(**kw)) == status
+
+
+def test_varlen_backward_workspace_size(lib):
+    wmax = (100 + 64 * 3 + 63) // 64 * 64      # every sequence padded to whole tiles
+    assert g2.g2attn_varlen_backward_workspace_size(3, 100, 8) == 2 * 8 * wmax * 4 + 4 * 4
+    assert g2.g2attn_varlen_backward_workspace_size(0, 100, 8) == 0
+    assert g2.g2attn_varlen_backward_workspace_size(3, 0, 8) == 0
+
+
+def varlen_backward_args(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+             cu_q=FAKE, cu_k=FAKE, num_seqs=2, total_q=128, total_k=256, max_T=64, max_S=128,
+             H=8, Hkv=4, d=128, query_scale=0.0625, softcap=50.0, window=0, workspace=FAKE,
+             workspace_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cu_q=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(cu_k=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(lse=None), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(num_seqs=0), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(max_T=129), g2.G2ATTN_ERR_INVALID_ARG),             # above max_S
+    (dict(max_S=257), g2.G2ATTN_ERR_INVALID_ARG),             # above total_k
+    (dict(window=-2), g2.G2ATTN_ERR_INVALID_ARG),
+    (dict(d=256), g2.G2ATTN_ERR_UNSUPPORTED),
+    (dict(Hkv=3), g2.G2ATTN_ERR_UNSUPPORTED),
+    (dict(num_seqs=1025), g2.G2ATTN_ERR_UNSUPPORTED),         # the kernels' sequence table
+    (dict(workspace_bytes=64), g2.G2ATTN_ERR_WORKSPACE),
+    (dict(workspace=ctypes.c_void_p((1 << 20) + 4)), g2.G2ATTN_ERR_MISALIGNED),
+    (dict(cu_k=ctypes.c_void_p((1 << 20) + 2)), g2.G2ATTN_ERR_MISALIGNED),
+])
+def test_varlen_backward_rejects_before_launch(lib, kw, status):
+    assert g2.g2attn_prefill_varlen_backward(*varlen_backward_args(**kw)) == status
