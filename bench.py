@@ -18,7 +18,8 @@ Printed (rank 0, one JSON line): the contract keys, plus
   extra         9B pair (local/global separately), 27B decode (KV GB/s,
                 tokens/s), the 9B ragged varlen prefill, the Gemma 3-shaped
                 variant of the 2B pair (window 1024, no cap) and the gradients
-                of the 27B-shaped pair (useful backward TFLOP/s)
+                of the 27B-shaped pair, dense and as a packed batch of 8
+                sequences (useful backward TFLOP/s)
 
 `--impl reference` times the fp64 oracle (the reference arm of this build)
 on the host cores on bounded samples of the same workload.
@@ -44,7 +45,8 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from global_soft_capped_b200.inputs import (  # noqa: E402
-    WORKLOADS, backward_inputs, decode_inputs, prefill_inputs, varlen_inputs)
+    WORKLOADS, backward_inputs, decode_inputs, prefill_inputs, varlen_backward_inputs,
+    varlen_inputs)
 
 METRIC = "useful attention TFLOP/s (prefill) and KV GB/s (decode) vs B200 roofline"
 WORKLOAD = "2b"
@@ -498,6 +500,29 @@ def extra_workloads(g2, dev, stream, flush):
         rb[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
                    "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
     res["27b_backward"] = rb
+    del q, k, v, dout, dq, dk, dv, ws, out, lse
+
+    # gradients of a 27B-shaped packed batch (8 sequences of 512-8192 tokens)
+    w = WORKLOADS["27b_varlen_backward"]
+    Ts, Ss, cq, ck, q, k, v, dout = varlen_backward_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H,
+                                                           w.Hkv, w.d, w.std, w.seed)
+    q, k, v, dout, cq, ck = (t.to(dev) for t in (q, k, v, dout, cq, ck))
+    n = g2.g2attn_varlen_backward_workspace_size(len(Ts), q.shape[0], w.H)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rvb = {"tokens": int(sum(Ts))}
+    for lay, win in (("local", w.window_local), ("global", 0)):
+        out, lse = g2.prefill_varlen(q, k, v, cq, ck, max(Ts), max(Ss), query_scale=w.query_scale,
+                                     softcap=w.softcap, window=win, stream=stream)
+        f = 2.5 * varlen_flops(Ts, Ss, w.H, w.d, win)
+        med, best = time_launches(
+            lambda: g2.prefill_varlen_backward(q, k, v, out, lse, dout, cq, ck, max(Ts), max(Ss),
+                                               query_scale=w.query_scale, softcap=w.softcap,
+                                               window=win, workspace=ws, dq=dq, dk=dk, dv=dv,
+                                               stream=stream), flush, stream)
+        rvb[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                    "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+    res["27b_varlen_backward"] = rvb
     return res
 
 
@@ -571,7 +596,16 @@ def run_single(args, dev):
     w = WORKLOADS[name]
     win = w.window_local if lay == "local" else 0
     stream = torch.cuda.current_stream()
-    if name == "27b_backward":
+    if name == "27b_varlen_backward":
+        Ts, Ss, cq, ck, q, k, v, dout = varlen_backward_inputs(w.num_seqs, w.len_lo, w.len_hi,
+                                                               w.H, w.Hkv, w.d, w.std, w.seed)
+        q, k, v, dout, cq, ck = (t.to(dev) for t in (q, k, v, dout, cq, ck))
+        out, lse = g2.prefill_varlen(q, k, v, cq, ck, max(Ts), max(Ss), query_scale=w.query_scale,
+                                     softcap=w.softcap, window=win, stream=stream)
+        fn = lambda: g2.prefill_varlen_backward(q, k, v, out, lse, dout, cq, ck, max(Ts),
+                                                max(Ss), query_scale=w.query_scale,
+                                                softcap=w.softcap, window=win, stream=stream)
+    elif name == "27b_backward":
         q, k, v, dout = (t.to(dev) for t in backward_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d,
                                                              w.std, w.seed))
         out, lse = g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap, window=win,

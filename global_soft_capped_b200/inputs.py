@@ -77,6 +77,12 @@ WORKLOADS = {
         "27b_backward", "prefill", H=32, Hkv=16, d=128, window_local=4096,
         query_scale=144.0 ** -0.5, softcap=50.0, std=1.0, seed=6, B=1, T=8192, S=8192,
         note="27B-shaped layer pair, forward outputs and upstream gradients for the backward"),
+    # Packed training batch of the same 27B shape: 8 self-attention sequences of
+    # 512-8192 tokens, dout drawn after q, k, v from the same generator
+    "27b_varlen_backward": Workload(
+        "27b_varlen_backward", "varlen", H=32, Hkv=16, d=128, window_local=4096,
+        query_scale=144.0 ** -0.5, softcap=50.0, std=1.0, seed=7, num_seqs=8, len_lo=512,
+        len_hi=8192, note="27B-shaped packed batch, gradients of the packed layer pair"),
     # Gemma 3-shaped parameter variant of the same layer pair (the research-hub
     # page: window 1024, soft-capping replaced by QK-norm, which acts on the
     # inputs upstream of this kernel, so the cap is off here).
@@ -145,7 +151,11 @@ def varlen_inputs(num_seqs, len_lo, len_hi, H, Hkv, d, std=1.0, seed=0,
     with explicit (T_i, S_i) pairs. Returns (T_list, S_list, cu_seqlens_q,
     cu_seqlens_k, q (sum T,H,d), k (sum S,Hkv,d), v).
     """
-    g = _gen(seed)
+    return _varlen_draw(_gen(seed), num_seqs, len_lo, len_hi, H, Hkv, d, std, tail_T, tail_S,
+                        seq_lens)
+
+
+def _varlen_draw(g, num_seqs, len_lo, len_hi, H, Hkv, d, std, tail_T, tail_S, seq_lens):
     if seq_lens is None:
         ls = _lengths(num_seqs, len_lo, len_hi, g)
         Ts, Ss = list(ls), list(ls)
@@ -164,6 +174,16 @@ def varlen_inputs(num_seqs, len_lo, len_hi, H, Hkv, d, std=1.0, seed=0,
     v = _normal_bf16((ck[-1], Hkv, d), std, g)
     return (Ts, Ss, torch.tensor(cq, dtype=torch.int32), torch.tensor(ck, dtype=torch.int32),
             q, k, v)
+
+
+def varlen_backward_inputs(num_seqs, len_lo, len_hi, H, Hkv, d, std=1.0, seed=0):
+    """varlen_inputs (no tail), then the upstream gradient dout (sum T,H,d),
+    fp32 standard normals rounded to bf16, from the same generator."""
+    g = _gen(seed)
+    Ts, Ss, cq, ck, q, k, v = _varlen_draw(g, num_seqs, len_lo, len_hi, H, Hkv, d, std, 0, 0,
+                                           None)
+    dout = _normal_bf16(tuple(q.shape), 1.0, g)
+    return Ts, Ss, cq, ck, q, k, v, dout
 
 
 def backward_inputs(B, T, S, H, Hkv, d, std=1.0, seed=0):
