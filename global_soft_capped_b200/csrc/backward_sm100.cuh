@@ -52,7 +52,8 @@ struct BwCfg {
     static constexpr int SLOT_BYTES = 2 * TILE_BYTES + VEC_BYTES;
     static constexpr int SMEM_TILES = 2 * TILE_BYTES + 2 * SLOT_BYTES;  // R1, R2, 2 column slots
     static constexpr int MAX_SEQ_TABLE = 1024;                  // varlen: sequences per launch
-    static constexpr int VL_BYTES = 4 * (MAX_SEQ_TABLE + 1);    // unit prefix over sequences
+    // varlen: per-sequence work, sequences ranked by it, unit prefix in rank order
+    static constexpr int VL_BYTES = 4 * (3 * MAX_SEQ_TABLE + 1);
     static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + VL_BYTES;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -96,6 +97,11 @@ __device__ __forceinline__ float bw_tanh_series(float u) {
     return u * q;
 }
 
+template <bool B>
+struct BwMask {
+    static constexpr bool value = B;
+};
+
 struct BwUnit {
     int g;
     int T, S, qoff;   // the sequence: queries, keys, position of query 0
@@ -119,12 +125,44 @@ __device__ __forceinline__ void bw_seq_rows(const int* cu, int s, int total, int
     *len = b1 - b0;
 }
 
-// Units. Dense: KV units take key tiles ascending (the earliest keys see the
-// most queries), then batch, then KV head; Q units take query tiles
-// descending, then batch, then head. Varlen: sequence by sequence (the unit
-// prefix `cum` over sequences), within a sequence as dense.
+// Row tile rt (of `tiles`) of a sequence with U.T queries at the end of U.S
+// keys: its rows and the column tiles that hold a visible pair. KV: key tiles
+// ascending (the earliest keys see the most queries); Q: query tiles
+// descending (the latest queries see the most keys).
 template <int MODE>
-__device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, int u, BwUnit& U) {
+__device__ __forceinline__ void bw_tile_cols(int rt, int tiles, int window, BwUnit& U) {
+    if (MODE == BW_KV) {
+        U.row0 = rt * BW_KEYS;
+        U.rvalid = min(BW_KEYS, U.S - U.row0);
+        // query rows t whose position t + qoff sees a key of the tile
+        const int t_lo = max(0, U.row0 - U.qoff);
+        const int t_hi = window > 0 ? min(U.T - 1, U.row0 + BW_KEYS - 1 + window - 1 - U.qoff)
+                                    : U.T - 1;
+        U.col0 = t_lo / BW_QPOS;
+        U.ncols = (t_lo <= t_hi) ? t_hi / BW_QPOS - U.col0 + 1 : 0;
+    } else {
+        const int qt = tiles - 1 - rt;
+        U.row0 = qt * BW_QPOS;
+        U.rvalid = min(BW_QPOS, U.T - U.row0);
+        const int p_min = U.row0 + U.qoff, p_max = p_min + U.rvalid - 1;
+        const int j_lo = window > 0 ? max(0, p_min - window + 1) : 0;
+        const int j_hi = min(p_max, U.S - 1);
+        U.col0 = j_lo / BW_KEYS;
+        U.ncols = j_hi >= j_lo ? j_hi / BW_KEYS - U.col0 + 1 : 0;
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ int bw_row_tiles(int T, int S) {
+    return MODE == BW_KV ? (S + BW_KEYS - 1) / BW_KEYS : (T + BW_QPOS - 1) / BW_QPOS;
+}
+
+// Units. Dense: row tiles in the order of bw_tile_cols, then batch, then KV
+// head. Varlen: sequence by sequence, heaviest first (`order`, with the unit
+// prefix `cum` in that order), within a sequence as dense.
+template <int MODE>
+__device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, const int* order,
+                                        int u, BwUnit& U) {
     int rt, tiles;
     if (!P.varlen) {
         const int BG = P.B * P.Hkv;
@@ -145,7 +183,7 @@ __device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, int u
             const int mid = (lo + hi + 1) >> 1;
             if (cum[mid] <= u) lo = mid; else hi = mid - 1;
         }
-        const int s = lo, lu = u - cum[s];
+        const int s = order[lo], lu = u - cum[lo];
         U.g = lu % P.Hkv;
         rt = lu / P.Hkv;
         bw_seq_rows(P.cu_q, s, P.total_q, &U.qbase, &U.T);
@@ -153,27 +191,9 @@ __device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, int u
         U.qoff = U.S - U.T;
         U.wbase = P.wq[s];
         U.wstride = P.wmax;
-        tiles = MODE == BW_KV ? (U.S + BW_KEYS - 1) / BW_KEYS : (U.T + BW_QPOS - 1) / BW_QPOS;
+        tiles = bw_row_tiles<MODE>(U.T, U.S);
     }
-    if (MODE == BW_KV) {
-        U.row0 = rt * BW_KEYS;
-        U.rvalid = min(BW_KEYS, U.S - U.row0);
-        // query rows t whose position t + qoff sees a key of the tile
-        const int t_lo = max(0, U.row0 - U.qoff);
-        const int t_hi = P.window > 0 ? min(U.T - 1, U.row0 + BW_KEYS - 1 + P.window - 1 - U.qoff)
-                                      : U.T - 1;
-        U.col0 = t_lo / BW_QPOS;
-        U.ncols = (t_lo <= t_hi) ? t_hi / BW_QPOS - U.col0 + 1 : 0;
-    } else {
-        const int qt = tiles - 1 - rt;
-        U.row0 = qt * BW_QPOS;
-        U.rvalid = min(BW_QPOS, U.T - U.row0);
-        const int p_min = U.row0 + U.qoff, p_max = p_min + U.rvalid - 1;
-        const int j_lo = P.window > 0 ? max(0, p_min - P.window + 1) : 0;
-        const int j_hi = min(p_max, U.S - 1);
-        U.col0 = j_lo / BW_KEYS;
-        U.ncols = j_hi / BW_KEYS - U.col0 + 1;
-    }
+    bw_tile_cols<MODE>(rt, tiles, P.window, U);
 }
 
 // -D_i = -(dout_i . out_i) (fp32 sum of bf16 products) and -lse_i * log2(e),
@@ -358,7 +378,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* drain = bars + 12;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);  // varlen unit prefix
+    // varlen tables: cum[num_seqs + 1] (unit prefix in rank order), order[], work[]
+    int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
+    int* order = cum + C::MAX_SEQ_TABLE + 1;
+    int* work = order + C::MAX_SEQ_TABLE;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -379,13 +402,41 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (P.varlen) {  // units of each sequence (Hkv x its row tiles), then an exclusive scan
+    if (P.varlen) {
+        // work of each sequence (column tiles of all its row tiles, one KV
+        // head), its rank (heaviest first, ties by index), then the units
+        // (Hkv x row tiles) of the ranked sequences as an exclusive scan
         const int ns = P.num_seqs;
         for (int q = threadIdx.x; q < ns; q += blockDim.x) {
+            BwUnit W;
+            int qb, kb;
+            bw_seq_rows(P.cu_q, q, P.total_q, &qb, &W.T);
+            bw_seq_rows(P.cu_k, q, P.total_k, &kb, &W.S);
+            W.qoff = W.S - W.T;
+            const int tiles = W.T > 0 ? bw_row_tiles<MODE>(W.T, W.S) : 0;
+            int w = 0;
+            for (int rt = 0; rt < tiles; ++rt) {
+                bw_tile_cols<MODE>(rt, tiles, P.window, W);
+                w += max(W.ncols, 0);
+            }
+            work[q] = w;
+        }
+        __syncthreads();
+        for (int q = threadIdx.x; q < ns; q += blockDim.x) {
+            const int wq = work[q];
+            int rank = 0;
+            for (int q2 = 0; q2 < ns; ++q2) {
+                const int w2 = work[q2];
+                rank += (w2 > wq) || (w2 == wq && q2 < q);
+            }
+            order[rank] = q;
+        }
+        __syncthreads();
+        for (int k = threadIdx.x; k < ns; k += blockDim.x) {
             int qb, t, kb, sk;
-            bw_seq_rows(P.cu_q, q, P.total_q, &qb, &t);
-            bw_seq_rows(P.cu_k, q, P.total_k, &kb, &sk);
-            cum[q] = P.Hkv * (KV ? (sk + BW_KEYS - 1) / BW_KEYS : (t + BW_QPOS - 1) / BW_QPOS);
+            bw_seq_rows(P.cu_q, order[k], P.total_q, &qb, &t);
+            bw_seq_rows(P.cu_k, order[k], P.total_k, &kb, &sk);
+            cum[k] = P.Hkv * bw_row_tiles<MODE>(t, sk);
         }
         __syncthreads();
         if (warp == 0) {
@@ -434,7 +485,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const int u = bw_sched(r, cta, G);
                 if (u >= num_units) continue;
                 BwUnit U;
-                bw_unit<MODE>(P, cum, u, U);
+                bw_unit<MODE>(P, cum, order, u, U);
                 if (U.ncols == 0) continue;
                 if (uw > 0) {
                     ok = mbar_wait(r_empty, (uw - 1) & 1, abort_flag, lim, SITE_BW_PROD);
@@ -560,7 +611,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const int u = bw_sched(r, cta, G);
                 if (u >= num_units) continue;
                 BwUnit U;
-                bw_unit<MODE>(P, cum, u, U);
+                bw_unit<MODE>(P, cum, order, u, U);
                 if (U.ncols == 0) continue;
                 ok = mbar_wait(r_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
@@ -624,7 +675,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const int u = bw_sched(rr, cta, G);
             if (u >= num_units) continue;
             BwUnit U;
-            bw_unit<MODE>(P, cum, u, U);
+            bw_unit<MODE>(P, cum, order, u, U);
             if (U.ncols == 0) {
                 // keys that no query sees: zero gradients (KV mode only; every
                 // query sees at least its own key)
@@ -676,6 +727,27 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     interior = j_hi <= t_lo + U.qoff && t_hi < U.T && j_hi < U.S &&
                                (P.window == 0 || t_hi + U.qoff - j_lo < P.window);
                 }
+                // This thread's visible column indices [vlo, vhi] (KV: query
+                // rows t of its key; Q: keys j of its query row), as an offset
+                // and unsigned span; an empty range never matches.
+                int vlo;
+                unsigned vspan;
+                {
+                    int lo, hi;
+                    if (KV) {
+                        lo = key_row - U.qoff;
+                        hi = P.window > 0 ? min(U.T - 1, lo + P.window - 1) : U.T - 1;
+                        if (key_row >= U.S) hi = lo - 1;
+                    } else {
+                        const int pos = t_row + U.qoff;
+                        lo = P.window > 0 ? max(0, pos - P.window + 1) : 0;
+                        hi = min(pos, U.S - 1);
+                        if (t_row >= U.T) hi = lo - 1;
+                    }
+                    if (hi < lo) { lo = 1 << 30; hi = lo; }
+                    vlo = lo;
+                    vspan = static_cast<unsigned>(hi - lo);
+                }
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {  // two chunks of 32 columns
                     const int cb = col0 + 32 * h2;
@@ -702,9 +774,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             nd = make_float2(row_nd, row_nd);
                         }
                     };
-                    if (interior && (poly || !P.has_cap)) {
-                        // fast path: no mask, packed pairs. P = 2^(s2 - lse2),
-                        // dS = P (dP - D) (1 - tanh^2)
+                    // fast path, packed pairs: P = 2^(s2 - lse2), dS = P (dP - D) (1 - tanh^2);
+                    // on tiles that cross the band's edges each weight outside
+                    // [vlo, vhi] is replaced by 0 after its exp2
+                    auto fast = [&](auto mask_tag) {
+                        constexpr bool MASK = decltype(mask_tag)::value;
+                        auto keep = [&](int i, int e, float p) {
+                            if constexpr (MASK) {
+                                const int idx = (KV ? ((cb + i + e) & 63) : cb + i + e) + ccol0;
+                                return static_cast<unsigned>(idx - vlo) <= vspan ? p : 0.0f;
+                            } else {
+                                return p;
+                            }
+                        };
                         const float2 one = make_float2(1.f, 1.f), mone = make_float2(-1.f, -1.f);
                         if (P.has_cap) {
                             const float2 us = make_float2(P.u_scale, P.u_scale);
@@ -728,7 +810,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                 const float2 th = mul2(u, q);              // tanh(alpha x / C)
                                 const float2 e2 = fma2(th, cl2, nl2);       // s2 - lse2
                                 const float2 dcap = fma2(mul2(th, th), mone, one);
-                                const float p0 = ex2_approx(e2.x), p1 = ex2_approx(e2.y);
+                                const float p0 = keep(i, 0, ex2_approx(e2.x));
+                                const float p1 = keep(i, 1, ex2_approx(e2.y));
                                 const float2 ds = mul2(mul2(make_float2(p0, p1), add2(y, nd)), dcap);
                                 pp[i / 2] = pack_bf16x2(p0, p1);
                                 pd[i / 2] = pack_bf16x2(ds.x, ds.y);
@@ -744,12 +827,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                 const float2 y = make_float2(__uint_as_float(yv[i]),
                                                              __uint_as_float(yv[i + 1]));
                                 const float2 e2 = fma2(x, sl2, nl2);
-                                const float p0 = ex2_approx(e2.x), p1 = ex2_approx(e2.y);
+                                const float p0 = keep(i, 0, ex2_approx(e2.x));
+                                const float p1 = keep(i, 1, ex2_approx(e2.y));
                                 const float2 ds = mul2(make_float2(p0, p1), add2(y, nd));
                                 pp[i / 2] = pack_bf16x2(p0, p1);
                                 pd[i / 2] = pack_bf16x2(ds.x, ds.y);
                             }
                         }
+                    };
+                    if (poly || !P.has_cap) {
+                        if (interior) fast(BwMask<false>{}); else fast(BwMask<true>{});
                     } else {
                         // general path: per-element mask, exact cap when |u| > 1/4
 #pragma unroll
