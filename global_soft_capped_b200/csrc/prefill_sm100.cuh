@@ -217,9 +217,12 @@ __device__ __forceinline__ void pf_unit(const PfParams& P, const VlTables& V, in
 
 // Row of key `key` (relative to the sequence start) in the K/V tensor maps. A
 // paged cache keeps every 128-key tile inside one block (blocks >= 128 rows).
+// The table column stays inside the sequence's row and the entry inside the
+// cache, whatever the lengths and the table hold.
 __device__ __forceinline__ int pf_key_row(const PfParams& P, const PfUnit& U, int key) {
     if (!P.paged) return U.kbase + key;
-    int b = P.kv_table[static_cast<size_t>(U.seq) * P.kv_max_blocks + (key >> P.kv_block_shift)];
+    const int col = min(key >> P.kv_block_shift, P.kv_max_blocks - 1);
+    int b = P.kv_table[static_cast<size_t>(U.seq) * P.kv_max_blocks + col];
     b = max(0, min(b, P.kv_num_blocks - 1));
     return (b << P.kv_block_shift) + (key & ((1 << P.kv_block_shift) - 1));
 }

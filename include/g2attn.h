@@ -116,8 +116,10 @@ G2ATTN_API int g2attn_prefill_varlen(const void* q, const void* k, const void* v
  *   Requires block_size a power of two >= 128 (every 128-key tile then lies in
  *   one block) and max_blocks_per_seq * block_size >= max_S. Rows of a sequence's
  *   last block beyond S_s must hold finite values (they meet zero weights).
- *   Table entries outside [0, num_blocks) are clamped. out, lse, limits and
- *   errors as g2attn_prefill_varlen.
+ *   Table entries outside [0, num_blocks) are clamped and no table column past
+ *   max_blocks_per_seq is read: malformed lengths or tables give undefined
+ *   results, never an out-of-bounds access. out, lse, limits and errors as
+ *   g2attn_prefill_varlen.
  */
 G2ATTN_API int g2attn_prefill_paged(const void* q, const void* k_blocks, const void* v_blocks,
                          void* out, float* lse, const int* cu_seqlens_q,
