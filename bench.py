@@ -18,8 +18,9 @@ Printed (rank 0, one JSON line): the contract keys, plus
   extra         9B pair (local/global separately), 27B decode (KV GB/s,
                 tokens/s), the 9B ragged varlen prefill, the Gemma 3-shaped
                 variant of the 2B pair (window 1024, no cap) and the gradients
-                of the 27B-shaped pair, dense and as a packed batch of 8
-                sequences (useful backward TFLOP/s)
+                of the 27B-shaped pair (dense and as a packed batch of 8
+                sequences) and of the 2B-shaped pair at d = 256 (useful
+                backward TFLOP/s)
 
 `--impl reference` times the fp64 oracle (the reference arm of this build)
 on the host cores on bounded samples of the same workload.
@@ -519,25 +520,27 @@ def extra_workloads(g2, dev, stream, flush):
     res["9b_varlen_paged_kv"] = rp
     del q, kp, vp, out, lse
 
-    # gradients of the 27B-shaped layer pair (dq, dk, dv; three launches per call)
-    w = WORKLOADS["27b_backward"]
-    q, k, v, dout = (t.to(dev) for t in backward_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std,
-                                                         w.seed))
-    ws = g2.backward_workspace(w.B, w.T, w.H, dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    rb = {}
-    for lay, win in (("local", w.window_local), ("global", 0)):
-        out, lse = g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap, window=win,
-                              stream=stream)
-        f = backward_flops(w.B, w.T, w.S, w.H, w.d, 0, win)
-        med, best = time_launches(
-            lambda: g2.prefill_backward(q, k, v, out, lse, dout, query_scale=w.query_scale,
-                                        softcap=w.softcap, window=win, workspace=ws, dq=dq, dk=dk,
-                                        dv=dv, stream=stream), flush, stream)
-        rb[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
-                   "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
-    res["27b_backward"] = rb
-    del q, k, v, dout, dq, dk, dv, ws, out, lse
+    # gradients of the 27B-shaped (d = 128) and 2B-shaped (d = 256) layer pairs
+    # (dq, dk, dv; three launches per call)
+    for name in ("27b_backward", "2b_backward"):
+        w = WORKLOADS[name]
+        q, k, v, dout = (t.to(dev) for t in backward_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d,
+                                                             w.std, w.seed))
+        ws = g2.backward_workspace(w.B, w.T, w.H, dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        rb = {}
+        for lay, win in (("local", w.window_local), ("global", 0)):
+            out, lse = g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap,
+                                  window=win, stream=stream)
+            f = backward_flops(w.B, w.T, w.S, w.H, w.d, 0, win)
+            med, best = time_launches(
+                lambda: g2.prefill_backward(q, k, v, out, lse, dout, query_scale=w.query_scale,
+                                            softcap=w.softcap, window=win, workspace=ws, dq=dq,
+                                            dk=dk, dv=dv, stream=stream), flush, stream)
+            rb[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
+                       "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
+        res[name] = rb
+        del q, k, v, dout, dq, dk, dv, ws, out, lse
 
     # gradients of a 27B-shaped packed batch (8 sequences of 512-8192 tokens)
     w = WORKLOADS["27b_varlen_backward"]
@@ -642,7 +645,7 @@ def run_single(args, dev):
         fn = lambda: g2.prefill_varlen_backward(q, k, v, out, lse, dout, cq, ck, max(Ts),
                                                 max(Ss), query_scale=w.query_scale,
                                                 softcap=w.softcap, window=win, stream=stream)
-    elif name == "27b_backward":
+    elif name in ("27b_backward", "2b_backward"):
         q, k, v, dout = (t.to(dev) for t in backward_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d,
                                                              w.std, w.seed))
         out, lse = g2.prefill(q, k, v, query_scale=w.query_scale, softcap=w.softcap, window=win,

@@ -338,16 +338,32 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mo, const CUtensorMap& 
     return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
 }
 
+// Tensor maps of the two gradient kernels: the dk/dv kernel keeps 128-key K/V
+// tiles and streams CQ-position q/dout tiles; the dq kernel keeps 64-position
+// q/dout tiles and streams CK-key K/V tiles (both heads of a group per q box).
+struct BwMaps {
+    CUtensorMap q_kv, o_kv, k_kv, v_kv;  // dk/dv kernel
+    CUtensorMap q_q, o_q, k_q, v_q;      // dq kernel
+};
+
+template <int D>
+bool make_bw_maps(BwMaps& m, const void* q, const void* k, const void* v, const void* dout,
+                  long long tq, long long tk, int H, int Hkv) {
+    using C = g2::BwCfg<D>;
+    return make_map(&m.q_kv, q, D, tq, H, C::CQ, 2) && make_map(&m.o_kv, dout, D, tq, H, C::CQ, 2) &&
+           make_map(&m.k_kv, k, D, tk, Hkv, g2::BW_KEYS, 1) &&
+           make_map(&m.v_kv, v, D, tk, Hkv, g2::BW_KEYS, 1) &&
+           make_map(&m.q_q, q, D, tq, H, g2::BW_QPOS, 2) &&
+           make_map(&m.o_q, dout, D, tq, H, g2::BW_QPOS, 2) &&
+           make_map(&m.k_q, k, D, tk, Hkv, C::CK, 1) && make_map(&m.v_q, v, D, tk, Hkv, C::CK, 1);
+}
+
 template <int D>
 int launch_backward(const void* q, const void* k, const void* v, const void* out,
                     const float* lse, const void* dout, g2::BwParams& P, cudaStream_t st) {
-    CUtensorMap mq, mo, mk, mv;
+    BwMaps m;
     const long long tq = static_cast<long long>(P.B) * P.T, tk = static_cast<long long>(P.B) * P.S;
-    if (!make_map(&mq, q, D, tq, P.H, g2::BW_QPOS, 2) ||
-        !make_map(&mo, dout, D, tq, P.H, g2::BW_QPOS, 2) ||
-        !make_map(&mk, k, D, tk, P.Hkv, g2::BW_KEYS, 1) ||
-        !make_map(&mv, v, D, tk, P.Hkv, g2::BW_KEYS, 1))
-        return G2ATTN_ERR_CUDA;
+    if (!make_bw_maps<D>(m, q, k, v, dout, tq, tk, P.H, P.Hkv)) return G2ATTN_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return G2ATTN_ERR_CUDA;
     // -D = -(dout . out) and -lse * log2(e) per (b, h, position)
@@ -363,10 +379,13 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
     const int key_tiles = (P.S + g2::BW_KEYS - 1) / g2::BW_KEYS;
     const int q_tiles = (P.T + g2::BW_QPOS - 1) / g2::BW_QPOS;
     P.row_tiles = key_tiles;
-    int rc = launch_bwd<D, g2::BW_KV>(mq, mo, mk, mv, P, key_tiles * BG, sms, st);
+    const long long kv_units = static_cast<long long>(key_tiles) * BG * g2::BwCfg<D>::DSPLIT_KV;
+    if (kv_units > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    int rc = launch_bwd<D, g2::BW_KV>(m.q_kv, m.o_kv, m.k_kv, m.v_kv, P,
+                                      static_cast<int>(kv_units), sms, st);
     if (rc) return rc;
     P.row_tiles = q_tiles;
-    return launch_bwd<D, g2::BW_Q>(mq, mo, mk, mv, P, q_tiles * BG, sms, st);
+    return launch_bwd<D, g2::BW_Q>(m.q_q, m.o_q, m.k_q, m.v_q, P, q_tiles * BG, sms, st);
 }
 
 // Varlen backward workspace: -lse2 and -D as (H, wmax) fp32 each, then the
@@ -384,12 +403,8 @@ template <int D>
 int launch_backward_varlen(const void* q, const void* k, const void* v, const void* out,
                            const float* lse, const void* dout, int total_q, int total_k,
                            g2::BwParams& P, cudaStream_t st) {
-    CUtensorMap mq, mo, mk, mv;
-    if (!make_map(&mq, q, D, total_q, P.H, g2::BW_QPOS, 2) ||
-        !make_map(&mo, dout, D, total_q, P.H, g2::BW_QPOS, 2) ||
-        !make_map(&mk, k, D, total_k, P.Hkv, g2::BW_KEYS, 1) ||
-        !make_map(&mv, v, D, total_k, P.Hkv, g2::BW_KEYS, 1))
-        return G2ATTN_ERR_CUDA;
+    BwMaps m;
+    if (!make_bw_maps<D>(m, q, k, v, dout, total_q, total_k, P.H, P.Hkv)) return G2ATTN_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return G2ATTN_ERR_CUDA;
     g2::bwd_wq_prefix<<<1, 32, 0, st>>>(P.cu_q, P.num_seqs, total_q, const_cast<int*>(P.wq));
@@ -404,12 +419,14 @@ int launch_backward_varlen(const void* q, const void* k, const void* v, const vo
     if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
     // Units are counted on the device from cu_seqlens; the grids come from
     // upper bounds and surplus units are skipped by the kernels.
-    const long long kv_ub = (static_cast<long long>(total_k) / g2::BW_KEYS + P.num_seqs) * P.Hkv;
+    const long long kv_ub = (static_cast<long long>(total_k) / g2::BW_KEYS + P.num_seqs) * P.Hkv *
+                            g2::BwCfg<D>::DSPLIT_KV;
     const long long q_ub = (static_cast<long long>(total_q) / g2::BW_QPOS + P.num_seqs) * P.Hkv;
     if (kv_ub > INT32_MAX || q_ub > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
-    int rc = launch_bwd<D, g2::BW_KV>(mq, mo, mk, mv, P, static_cast<int>(kv_ub), sms, st);
+    int rc = launch_bwd<D, g2::BW_KV>(m.q_kv, m.o_kv, m.k_kv, m.v_kv, P, static_cast<int>(kv_ub),
+                                      sms, st);
     if (rc) return rc;
-    return launch_bwd<D, g2::BW_Q>(mq, mo, mk, mv, P, static_cast<int>(q_ub), sms, st);
+    return launch_bwd<D, g2::BW_Q>(m.q_q, m.o_q, m.k_q, m.v_q, P, static_cast<int>(q_ub), sms, st);
 }
 
 }  // namespace
@@ -436,7 +453,6 @@ int g2attn_prefill_varlen_backward(const void* q, const void* k, const void* v, 
         return G2ATTN_ERR_INVALID_ARG;
     int rc = check_common(H, Hkv, d, query_scale, softcap, window);
     if (rc) return rc;
-    if (d != 64 && d != 128) return G2ATTN_ERR_UNSUPPORTED;
     if (num_seqs > g2::BwCfg<64>::MAX_SEQ_TABLE) return G2ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
         !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
@@ -483,7 +499,9 @@ int g2attn_prefill_varlen_backward(const void* q, const void* k, const void* v, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 64)
         return launch_backward_varlen<64>(q, k, v, out, lse, dout, total_q, total_k, P, st);
-    return launch_backward_varlen<128>(q, k, v, out, lse, dout, total_q, total_k, P, st);
+    if (d == 128)
+        return launch_backward_varlen<128>(q, k, v, out, lse, dout, total_q, total_k, P, st);
+    return launch_backward_varlen<256>(q, k, v, out, lse, dout, total_q, total_k, P, st);
 }
 
 size_t g2attn_backward_workspace_size(int B, int T, int H) {
@@ -503,7 +521,6 @@ int g2attn_prefill_backward(const void* q, const void* k, const void* v, const v
         return G2ATTN_ERR_INVALID_ARG;
     int rc = check_common(H, Hkv, d, query_scale, softcap, window);
     if (rc) return rc;
-    if (d != 64 && d != 128) return G2ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
         !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return G2ATTN_ERR_MISALIGNED;
@@ -540,7 +557,8 @@ int g2attn_prefill_backward(const void* q, const void* k, const void* v, const v
     P.timeout_ns = wait_limit_ns();
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 64) return launch_backward<64>(q, k, v, out, lse, dout, P, st);
-    return launch_backward<128>(q, k, v, out, lse, dout, P, st);
+    if (d == 128) return launch_backward<128>(q, k, v, out, lse, dout, P, st);
+    return launch_backward<256>(q, k, v, out, lse, dout, P, st);
 }
 
 int g2attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,

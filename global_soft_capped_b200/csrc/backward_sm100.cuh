@@ -1,5 +1,5 @@
 // backward_sm100.cuh -- gradients of the soft-capped local/global attention
-// layer on sm_100a (tcgen05 UMMA + TMA), for head sizes d = 64 and 128.
+// layer on sm_100a (tcgen05 UMMA + TMA), for head sizes d = 64, 128 and 256.
 //
 // Chain rule through the layer (Gemma 2 card, "Method", per-layer attention
 // pseudo-code; derivative of the soft-cap from the "Gemma 2 Guide", Deep Dive
@@ -16,16 +16,18 @@
 //   bwd_prep      D_i and lse_i * log2(e), per (b, h, position), into the
 //                 caller's workspace (positions padded to a multiple of 64)
 //   bwd_sm100<D, BW_KV>  one unit = 128 keys of one KV head: K and V stay in
-//                 shared memory, the 64-position query tiles (both heads of
-//                 the group: 128 rows) stream through. X = K Q^T (S^T) and
+//                 shared memory, the query tiles (CQ positions of both heads
+//                 of the group: 2 CQ rows) stream through. X = K Q^T (S^T) and
 //                 Y = V dout^T (dP^T) land in TMEM with one key per lane, so
 //                 P^T and dS^T are written back as bf16 and used directly as
 //                 the A operand of dv += P^T dout and dk += dS^T q.
 //   bwd_sm100<D, BW_Q>   one unit = 64 query positions x 2 heads: q and dout
-//                 stay, the 128-key tiles stream; X = q K^T, Y = dout V^T,
+//                 stay, the CK-key tiles stream; X = q K^T, Y = dout V^T,
 //                 dq += dS K.
-// TMEM (512 columns): accumulators at 0.., X at 256, Y at 384. KV mode needs
-// 2d + 256 columns, which is why d = 256 is not built here.
+// Column tiles are 128 rows for d <= 128 and 32 rows at d = 256 (BwCfg).
+// TMEM (512 columns): accumulators at 0..255, X at 256, Y at 384. The dk/dv
+// kernel needs 2 d accumulator columns, so at d = 256 each key tile is two
+// units, one per half of the d columns (X and Y are computed in both).
 #pragma once
 
 #include "common.cuh"
@@ -44,12 +46,29 @@ constexpr int BW_X_COL = 256;
 constexpr int BW_Y_COL = 384;
 constexpr uint32_t BW_TMEM_COLS = 512;
 
+// Tile shapes per head size. The resident (row) tiles are always 128 rows:
+// 128 keys (KV mode) or 64 positions x 2 heads (Q mode). The streamed column
+// tiles are CR rows: CQ positions x 2 heads (KV) or CK keys (Q), split into
+// two halves of HW columns, one per column part of the elementwise warps. At
+// d = 256 the column tiles shrink to 32 rows so that two slots still fit
+// next to the 128 KB resident pair, and the dk/dv kernel splits d into two
+// halves (DSPLIT units per key tile) so that its accumulators fit TMEM.
 template <int D>
 struct BwCfg {
-    static_assert(D == 64 || D == 128, "backward kernels are built for d = 64 and 128");
-    static constexpr int TILE_BYTES = 128 * D * 2;         // one 128-row operand tile
-    static constexpr int VEC_BYTES = 2 * 128 * 4;          // -lse2 and -D of 128 query rows
-    static constexpr int SLOT_BYTES = 2 * TILE_BYTES + VEC_BYTES;
+    static_assert(D == 64 || D == 128 || D == 256, "backward kernels: d = 64, 128, 256");
+    static constexpr int CQ = D == 256 ? 16 : BW_QPOS;  // KV column tile: positions per head
+    static constexpr int CK = D == 256 ? 32 : BW_KEYS;  // Q column tile: keys
+    static constexpr int CR = 2 * CQ;                    // column tile rows (both modes)
+    static_assert(CR == CK, "column tiles of both modes have CR rows");
+    static constexpr int HW = CR / 2;                    // columns per half (per warp part)
+    static constexpr int CHUNK = HW < 32 ? HW : 32;      // columns per TMEM round trip
+    static constexpr int DSPLIT_KV = D == 256 ? 2 : 1;   // dk/dv kernel: d-halves per key tile
+    static constexpr int TILE_BYTES = 128 * D * 2;       // one 128-row resident tile
+    static constexpr int CTILE_BYTES = CR * D * 2;       // one streamed column tile
+    static constexpr int VEC_BYTES = 1024;               // -lse2, -D of the tile's query rows
+    static constexpr int VEC_TX = 2 * CR * 4;            //   (bytes copied: CR rows, two arrays)
+    static constexpr int SLOT_BYTES = 2 * CTILE_BYTES + VEC_BYTES;
+    static_assert(SLOT_BYTES % 1024 == 0 && VEC_TX <= VEC_BYTES, "slot layout");
     static constexpr int SMEM_TILES = 2 * TILE_BYTES + 2 * SLOT_BYTES;  // R1, R2, 2 column slots
     static constexpr int MAX_SEQ_TABLE = 1024;                  // varlen: sequences per launch
     // varlen: per-sequence work, sequences ranked by it, unit prefix in rank order
@@ -104,13 +123,14 @@ struct BwMask {
 
 struct BwUnit {
     int g;
+    int dh;           // d-half of the dk/dv columns (d = 256); 0 otherwise
     int T, S, qoff;   // the sequence: queries, keys, position of query 0
     int qbase, kbase; // packed row of its first query / key
     long long wbase;  // workspace column of its position 0 for head 0 ...
     long long wstride;  // ... and the stride between heads
     int row0;     // KV: first key; Q: first query position (row index t within the sequence)
     int rvalid;   // KV: keys in the tile (<= 128); Q: positions in the tile (<= 64)
-    int col0;     // first column tile index (KV: 64-position tiles; Q: 128-key tiles)
+    int col0;     // first column tile index (KV: CQ-position tiles; Q: CK-key tiles)
     int ncols;    // column tiles (0: no visible pair; KV units then store zeros)
 };
 
@@ -129,8 +149,9 @@ __device__ __forceinline__ void bw_seq_rows(const int* cu, int s, int total, int
 // keys: its rows and the column tiles that hold a visible pair. KV: key tiles
 // ascending (the earliest keys see the most queries); Q: query tiles
 // descending (the latest queries see the most keys).
-template <int MODE>
+template <int D, int MODE>
 __device__ __forceinline__ void bw_tile_cols(int rt, int tiles, int window, BwUnit& U) {
+    constexpr int CQ = BwCfg<D>::CQ, CK = BwCfg<D>::CK;
     if (MODE == BW_KV) {
         U.row0 = rt * BW_KEYS;
         U.rvalid = min(BW_KEYS, U.S - U.row0);
@@ -138,8 +159,8 @@ __device__ __forceinline__ void bw_tile_cols(int rt, int tiles, int window, BwUn
         const int t_lo = max(0, U.row0 - U.qoff);
         const int t_hi = window > 0 ? min(U.T - 1, U.row0 + BW_KEYS - 1 + window - 1 - U.qoff)
                                     : U.T - 1;
-        U.col0 = t_lo / BW_QPOS;
-        U.ncols = (t_lo <= t_hi) ? t_hi / BW_QPOS - U.col0 + 1 : 0;
+        U.col0 = t_lo / CQ;
+        U.ncols = (t_lo <= t_hi) ? t_hi / CQ - U.col0 + 1 : 0;
     } else {
         const int qt = tiles - 1 - rt;
         U.row0 = qt * BW_QPOS;
@@ -147,8 +168,8 @@ __device__ __forceinline__ void bw_tile_cols(int rt, int tiles, int window, BwUn
         const int p_min = U.row0 + U.qoff, p_max = p_min + U.rvalid - 1;
         const int j_lo = window > 0 ? max(0, p_min - window + 1) : 0;
         const int j_hi = min(p_max, U.S - 1);
-        U.col0 = j_lo / BW_KEYS;
-        U.ncols = j_hi >= j_lo ? j_hi / BW_KEYS - U.col0 + 1 : 0;
+        U.col0 = j_lo / CK;
+        U.ncols = j_hi >= j_lo ? j_hi / CK - U.col0 + 1 : 0;
     }
 }
 
@@ -159,10 +180,14 @@ __device__ __forceinline__ int bw_row_tiles(int T, int S) {
 
 // Units. Dense: row tiles in the order of bw_tile_cols, then batch, then KV
 // head. Varlen: sequence by sequence, heaviest first (`order`, with the unit
-// prefix `cum` in that order), within a sequence as dense.
-template <int MODE>
+// prefix `cum` in that order), within a sequence as dense. The d-halves of a
+// key tile (dk/dv kernel at d = 256) are consecutive units.
+template <int D, int MODE>
 __device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, const int* order,
                                         int u, BwUnit& U) {
+    constexpr int DS = MODE == BW_KV ? BwCfg<D>::DSPLIT_KV : 1;
+    U.dh = u % DS;
+    u /= DS;
     int rt, tiles;
     if (!P.varlen) {
         const int BG = P.B * P.Hkv;
@@ -193,7 +218,7 @@ __device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, const
         U.wstride = P.wmax;
         tiles = bw_row_tiles<MODE>(U.T, U.S);
     }
-    bw_tile_cols<MODE>(rt, tiles, P.window, U);
+    bw_tile_cols<D, MODE>(rt, tiles, P.window, U);
 }
 
 // -D_i = -(dout_i . out_i) (fp32 sum of bf16 products) and -lse_i * log2(e),
@@ -320,9 +345,9 @@ __device__ __forceinline__ int bw_sched(int r, int c, int G) {
 // (query-side tensors); else 128 rows of head g (key-side tensors).
 template <int D>
 __device__ __forceinline__ void bw_load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
-                                             int row, int head) {
+                                             int row, int head, int rows = 128) {
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * 16384, map, bar, c * 64, row, head);
+    for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * rows * 128, map, bar, c * 64, row, head);
 }
 
 // HALF (= D/2) accumulator columns of this thread's row, times f, as bf16 to
@@ -351,6 +376,55 @@ __device__ __forceinline__ void bw_store_acc(uint32_t taddr, __nv_bfloat16* dst,
     }
 }
 
+// TMEM round trips of N columns (32 lanes x 32 bit): loads of 16 or 32
+// columns (complete with tmem_wait_ld, then bw_fence before use) and stores of
+// 8 or 16.
+template <int N>
+__device__ __forceinline__ void bw_ld_async(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 32, "TMEM load width");
+    if constexpr (N == 32) {
+        tmem_ld32_async(taddr, r);
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+              "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+              "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr)
+            : "memory");
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void bw_fence(uint32_t (&r)[N]) {
+    if constexpr (N == 32) {
+        tmem_reg_fence(r);
+    } else {
+        static_assert(N == 16, "TMEM load width");
+        asm volatile(""
+                     : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                       "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                       "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                     :
+                     : "memory");
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void bw_st(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 8 || N == 16, "TMEM store width");
+    if constexpr (N == 16) {
+        tmem_st16(taddr, r);
+    } else {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                taddr),
+            "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+            : "memory");
+    }
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(BW_THREADS, 1)
     bwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
@@ -358,12 +432,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
               const BwParams P) {
     using C = BwCfg<D>;
     constexpr bool KV = MODE == BW_KV;
+    constexpr int DS = KV ? C::DSPLIT_KV : 1;  // units per row tile (d-halves)
+    constexpr int ACC_N = D / DS;             // accumulator columns per product
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t* sR1 = base;                    // KV: K tile;  Q: q tile
     uint8_t* sR2 = base + C::TILE_BYTES;    // KV: V tile;  Q: dout tile
-    uint8_t* sSlot = base + 2 * C::TILE_BYTES;  // [2] x (C1 tile, C2 tile, lse2[128], D[128])
+    uint8_t* sSlot = base + 2 * C::TILE_BYTES;  // [2] x (C1 tile, C2 tile, lse2[CR], D[CR])
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::SMEM_TILES);
     uint64_t* r_full = bars + 0;
     uint64_t* r_empty = bars + 1;
@@ -416,7 +492,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const int tiles = W.T > 0 ? bw_row_tiles<MODE>(W.T, W.S) : 0;
             int w = 0;
             for (int rt = 0; rt < tiles; ++rt) {
-                bw_tile_cols<MODE>(rt, tiles, P.window, W);
+                bw_tile_cols<D, MODE>(rt, tiles, P.window, W);
                 w += max(W.ncols, 0);
             }
             work[q] = w;
@@ -473,7 +549,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const int G = gridDim.x;
     const int cta = blockIdx.x;
     const uint64_t lim = P.timeout_ns;
-    const int num_units = P.varlen ? min(P.num_units, cum[P.num_seqs]) : P.num_units;
+    const int num_units = P.varlen ? min(P.num_units, cum[P.num_seqs] * DS) : P.num_units;
 
     if (warp == BW_WARP_PRODUCER) {
         // ------------------------------------------------------------ producer
@@ -485,7 +561,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const int u = bw_sched(r, cta, G);
                 if (u >= num_units) continue;
                 BwUnit U;
-                bw_unit<MODE>(P, cum, order, u, U);
+                bw_unit<D, MODE>(P, cum, order, u, U);
                 if (U.ncols == 0) continue;
                 if (uw > 0) {
                     ok = mbar_wait(r_empty, (uw - 1) & 1, abort_flag, lim, SITE_BW_PROD);
@@ -506,26 +582,27 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (!ok) break;
                     uint8_t* slot = sSlot + sl * C::SLOT_BYTES;
                     if (KV) {
-                        const int t0 = (U.col0 + c) * BW_QPOS;
-                        mbar_arrive_expect_tx(&c_full[sl], 2 * C::TILE_BYTES + C::VEC_BYTES);
-                        bw_load_tile<D>(slot, &tmQ, &c_full[sl], U.qbase + t0, 2 * U.g);
-                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmO, &c_full[sl], U.qbase + t0,
-                                        2 * U.g);
-                        // -lse2 and -D of the tile's 128 query rows (head 2g, then 2g+1)
-                        float* vec = reinterpret_cast<float*>(slot + 2 * C::TILE_BYTES);
+                        const int t0 = (U.col0 + c) * C::CQ;
+                        mbar_arrive_expect_tx(&c_full[sl], 2 * C::CTILE_BYTES + C::VEC_TX);
+                        bw_load_tile<D>(slot, &tmQ, &c_full[sl], U.qbase + t0, 2 * U.g, C::CR);
+                        bw_load_tile<D>(slot + C::CTILE_BYTES, &tmO, &c_full[sl], U.qbase + t0,
+                                        2 * U.g, C::CR);
+                        // -lse2 and -D of the tile's CR query rows (head 2g, then 2g+1)
+                        float* vec = reinterpret_cast<float*>(slot + 2 * C::CTILE_BYTES);
 #pragma unroll
                         for (int hl = 0; hl < 2; ++hl) {
                             const size_t off = static_cast<size_t>(U.wbase) +
                                                (2 * U.g + hl) * U.wstride + t0;
-                            bulk_load(vec + hl * 64, P.nlse2 + off, 256, &c_full[sl]);
-                            bulk_load(vec + 128 + hl * 64, P.ndvec + off, 256, &c_full[sl]);
+                            bulk_load(vec + hl * C::CQ, P.nlse2 + off, C::CQ * 4, &c_full[sl]);
+                            bulk_load(vec + C::CR + hl * C::CQ, P.ndvec + off, C::CQ * 4,
+                                      &c_full[sl]);
                         }
                     } else {
-                        const int key0 = (U.col0 + c) * BW_KEYS;
-                        mbar_arrive_expect_tx(&c_full[sl], 2 * C::TILE_BYTES);
-                        bw_load_tile<D>(slot, &tmK, &c_full[sl], U.kbase + key0, U.g);
-                        bw_load_tile<D>(slot + C::TILE_BYTES, &tmV, &c_full[sl], U.kbase + key0,
-                                        U.g);
+                        const int key0 = (U.col0 + c) * C::CK;
+                        mbar_arrive_expect_tx(&c_full[sl], 2 * C::CTILE_BYTES);
+                        bw_load_tile<D>(slot, &tmK, &c_full[sl], U.kbase + key0, U.g, C::CR);
+                        bw_load_tile<D>(slot + C::CTILE_BYTES, &tmV, &c_full[sl], U.kbase + key0,
+                                        U.g, C::CR);
                     }
                     ++ct;
                 }
@@ -544,58 +621,66 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     else if (warp == BW_WARP_MMA) {
         // ------------------------------------------------------------ UMMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_XY = idesc_bf16(128, 64, false);  // one column half
-            constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, true);
+            constexpr int HW = C::HW;
+            constexpr uint32_t IDESC_XY = idesc_bf16(128, HW, false);  // one column half
+            constexpr uint32_t IDESC_ACC = idesc_bf16(128, ACC_N, true);
             constexpr uint32_t HI = sdesc_hi(1024);  // SBO 1024 B (8 rows x 128 B)
-            // K-major operands (contraction over d): 64-column blocks of 16 KB,
-            // k-step of 16 columns = 32 B inside a block
+            // K-major operands (contraction over d): 64-column blocks of rows x
+            // 128 B (resident tiles: 128 rows; column tiles: CR rows), k-step of
+            // 16 columns = 32 B inside a block
             const uint32_t r1_lo = sdesc_lo(smem_u32(sR1), 16);
             const uint32_t r2_lo = sdesc_lo(smem_u32(sR2), 16);
             const uint32_t slot_lo = sdesc_lo(smem_u32(sSlot), 16);
-            // the same column tiles read MN-major (contraction over their 128
-            // rows): LBO = 128 rows x 128 B between 64-column blocks
-            const uint32_t slot_lo_mn = sdesc_lo(smem_u32(sSlot), 128 * 128);
+            // the same column tiles read MN-major (contraction over their CR
+            // rows): LBO = CR rows x 128 B between 64-column blocks
+            constexpr uint32_t CBLOCK = (C::CR * 128) >> 4;
+            const uint32_t slot_lo_mn = sdesc_lo(smem_u32(sSlot), C::CR * 128);
             constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
-            constexpr uint32_t TILE_STEP = C::TILE_BYTES >> 4;
-            constexpr uint32_t HALF_ROWS = (64 * 128) >> 4;  // rows 64.. of a tile
+            constexpr uint32_t CTILE_STEP = C::CTILE_BYTES >> 4;
+            constexpr uint32_t HALF_ROWS = (HW * 128) >> 4;  // rows HW.. of a column tile
             uint32_t ct = 0;
             int uw = 0;
             bool ok = true;
             auto kstep = [](int kk) -> uint32_t {
                 return ((kk * 16) / 64) * (16384 >> 4) + (((kk * 16) % 64) / 16) * 2;
             };
-            // X, Y columns [64h, 64h + 64) of the tile in slot sl: rows 64h.. of
-            // the column tiles (N = 64), contraction over d
+            auto kstep_c = [](int kk) -> uint32_t {
+                return ((kk * 16) / 64) * CBLOCK + (((kk * 16) % 64) / 16) * 2;
+            };
+            // X, Y columns [HW h, HW h + HW) of the tile in slot sl: rows HW h..
+            // of the column tiles (N = HW), contraction over d
             auto issue_xy = [&](int sl, int h) {
                 const uint32_t c1 = slot_lo + sl * SLOT_STEP + h * HALF_ROWS;
-                const uint32_t c2 = c1 + TILE_STEP;
+                const uint32_t c2 = c1 + CTILE_STEP;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + BW_X_COL + 64 * h, r1_lo + kstep(kk), c1 + kstep(kk), HI,
+                    umma_ss_lh(tmem + BW_X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
                                IDESC_XY, kk != 0);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + BW_Y_COL + 64 * h, r2_lo + kstep(kk), c2 + kstep(kk), HI,
+                    umma_ss_lh(tmem + BW_Y_COL + HW * h, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
                                IDESC_XY, kk != 0);
                 umma_commit(&xy_full[h]);
             };
-            // accumulations over the half's 64 rows (K indices 64h..64h+63): A =
-            // the bf16 operand the half's warps wrote at columns 64h + 8(kk%4)
-            auto issue_acc = [&](int sl, int h, bool first) {
-                const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
-                const uint32_t c2_mn = c1_mn + TILE_STEP;
+            // accumulations over the half's HW rows (K indices HW h ..): A = the
+            // bf16 operand the half's warps wrote at columns HW h + 8 k4; B =
+            // the streamed tiles' columns of d-half dh (ACC_N columns)
+            auto issue_acc = [&](int sl, int h, int dh, bool first) {
+                const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP + dh * (ACC_N / 64) * CBLOCK;
+                const uint32_t c2_mn = c1_mn + CTILE_STEP;
+                constexpr int KS = HW / 16;  // K steps per half
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const int kk = 4 * h + k4;
+                for (int k4 = 0; k4 < KS; ++k4) {
+                    const int kk = KS * h + k4;
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
                     const uint32_t bstep = kk * ((16 * 128) >> 4);
-                    const uint32_t zc = 64 * h + 8 * k4;
+                    const uint32_t zc = HW * h + 8 * k4;
                     if (KV) {
                         // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y)
                         umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c2_mn + bstep, HI, IDESC_ACC,
                                    acc);
-                        umma_ts_lh(tmem + D, tmem + BW_Y_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
-                                   acc);
+                        umma_ts_lh(tmem + ACC_N, tmem + BW_Y_COL + zc, c1_mn + bstep, HI,
+                                   IDESC_ACC, acc);
                     } else {
                         // dq += dS K (dS at X)
                         umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
@@ -611,7 +696,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const int u = bw_sched(r, cta, G);
                 if (u >= num_units) continue;
                 BwUnit U;
-                bw_unit<MODE>(P, cum, order, u, U);
+                bw_unit<D, MODE>(P, cum, order, u, U);
                 if (U.ncols == 0) continue;
                 ok = mbar_wait(r_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
@@ -631,7 +716,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         if (!ok) break;
                     }
                     tc_fence_after();
-                    issue_acc(sl, 0, c == 0);
+                    issue_acc(sl, 0, U.dh, c == 0);
                     if (next) {
                         ok = mbar_wait(&c_full[sl ^ 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
                                        SITE_BW_MMA);
@@ -642,7 +727,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     ok = mbar_wait(&z_full[1], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_acc(sl, 1, false);
+                    issue_acc(sl, 1, U.dh, false);
                     umma_commit(&c_empty[sl]);
                     if (next) issue_xy(sl ^ 1, 1);
                     ++ct;
@@ -661,13 +746,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     else {
         // ------------------------------------------------------------ elementwise + epilogue
         // Warps w and w+4 share TMEM lane quadrant w%4 (rows 32(w%4)..+31);
-        // warp w takes columns 0..63 of X and Y, warp w+4 columns 64..127.
-        // KV mode: row = key, column = query row (head 2g + column/64). Q mode:
+        // warp w takes columns 0..HW-1 of X and Y, warp w+4 columns HW..2HW-1.
+        // KV mode: row = key, column = query row (head 2g + column/CQ). Q mode:
         // row = query row (head 2g + row/64), column = key.
+        constexpr int HW = C::HW, CQ = C::CQ, CHUNK = C::CHUNK;
         const int qd = warp & 3, part = warp >> 2;
         const int r = (qd << 5) | lane;
         const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
-        const int col0 = part * 64;
+        const int col0 = part * HW;
         uint32_t ct = 0;
         int uw = 0;
         bool ok = true;
@@ -675,18 +761,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const int u = bw_sched(rr, cta, G);
             if (u >= num_units) continue;
             BwUnit U;
-            bw_unit<MODE>(P, cum, order, u, U);
+            bw_unit<D, MODE>(P, cum, order, u, U);
             if (U.ncols == 0) {
                 // keys that no query sees: zero gradients (KV mode only; every
                 // query sees at least its own key)
                 if (KV && r < U.rvalid) {
                     const size_t row = (static_cast<size_t>(U.kbase) + U.row0 + r) * P.Hkv + U.g;
+                    const size_t c0 = row * D + U.dh * ACC_N + part * (ACC_N / 2);
 #pragma unroll
-                    for (int c = 0; c < D / 2; c += 8) {
-                        *reinterpret_cast<uint4*>(P.dv + row * D + part * (D / 2) + c) =
-                            make_uint4(0u, 0u, 0u, 0u);
-                        *reinterpret_cast<uint4*>(P.dk + row * D + part * (D / 2) + c) =
-                            make_uint4(0u, 0u, 0u, 0u);
+                    for (int c = 0; c < ACC_N / 2; c += 8) {
+                        *reinterpret_cast<uint4*>(P.dv + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(P.dk + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
                     }
                 }
                 continue;
@@ -711,17 +796,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const float* vec =
-                    reinterpret_cast<const float*>(sSlot + sl * C::SLOT_BYTES + 2 * C::TILE_BYTES);
-                const int ccol0 = (U.col0 + c) * (KV ? BW_QPOS : BW_KEYS);  // first t or key
+                    reinterpret_cast<const float*>(sSlot + sl * C::SLOT_BYTES + 2 * C::CTILE_BYTES);
+                const int ccol0 = (U.col0 + c) * (KV ? CQ : C::CK);  // first t or key
                 // Every pair of the tile visible? (then no per-element mask)
                 bool interior;
                 {
                     int j_lo, j_hi, t_lo, t_hi;
                     if (KV) {
                         j_lo = U.row0; j_hi = U.row0 + BW_KEYS - 1;
-                        t_lo = ccol0;  t_hi = ccol0 + BW_QPOS - 1;
+                        t_lo = ccol0;  t_hi = ccol0 + CQ - 1;
                     } else {
-                        j_lo = ccol0;  j_hi = ccol0 + BW_KEYS - 1;
+                        j_lo = ccol0;  j_hi = ccol0 + C::CK - 1;
                         t_lo = U.row0; t_hi = U.row0 + BW_QPOS - 1;
                     }
                     interior = j_hi <= t_lo + U.qoff && t_hi < U.T && j_hi < U.S &&
@@ -749,26 +834,26 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     vspan = static_cast<unsigned>(hi - lo);
                 }
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {  // two chunks of 32 columns
-                    const int cb = col0 + 32 * h2;
-                    uint32_t xv[32], yv[32];
-                    tmem_ld32_async(tmem + lane_addr + BW_X_COL + cb, xv);
-                    tmem_ld32_async(tmem + lane_addr + BW_Y_COL + cb, yv);
+                for (int h2 = 0; h2 < HW / CHUNK; ++h2) {  // chunks of CHUNK columns
+                    const int cb = col0 + CHUNK * h2;
+                    uint32_t xv[CHUNK], yv[CHUNK];
+                    bw_ld_async<CHUNK>(tmem + lane_addr + BW_X_COL + cb, xv);
+                    bw_ld_async<CHUNK>(tmem + lane_addr + BW_Y_COL + cb, yv);
                     tmem_wait_ld();
-                    tmem_reg_fence(xv);
-                    tmem_reg_fence(yv);
+                    bw_fence<CHUNK>(xv);
+                    bw_fence<CHUNK>(yv);
                     // the cap's tanh by series when every |u| of this warp's chunk <= 1/4
                     float amax = 0.f;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(xv[i])));
+                    for (int i = 0; i < CHUNK; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(xv[i])));
                     const bool poly = __all_sync(0xffffffffu, amax <= P.poly_acc_max);
-                    uint32_t pp[16], pd[16];
+                    uint32_t pp[CHUNK / 2], pd[CHUNK / 2];
                     // -lse2 / -D of the column pair i, i+1 (KV: per column, from
                     // the slot; Q: this row's)
                     auto vec_pair = [&](int i, float2& nl2, float2& nd) {
                         if (KV) {
                             nl2 = *reinterpret_cast<const float2*>(vec + cb + i);
-                            nd = *reinterpret_cast<const float2*>(vec + 128 + cb + i);
+                            nd = *reinterpret_cast<const float2*>(vec + C::CR + cb + i);
                         } else {
                             nl2 = make_float2(row_nl2, row_nl2);
                             nd = make_float2(row_nd, row_nd);
@@ -781,7 +866,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         constexpr bool MASK = decltype(mask_tag)::value;
                         auto keep = [&](int i, int e, float p) {
                             if constexpr (MASK) {
-                                const int idx = (KV ? ((cb + i + e) & 63) : cb + i + e) + ccol0;
+                                const int idx = (KV ? ((cb + i + e) & (CQ - 1)) : cb + i + e) + ccol0;
                                 return static_cast<unsigned>(idx - vlo) <= vspan ? p : 0.0f;
                             } else {
                                 return p;
@@ -795,7 +880,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             const float2 c1 = make_float2(-1.0f / 3.0f, -1.0f / 3.0f);
                             const float2 cl2 = make_float2(P.cap_l2, P.cap_l2);
 #pragma unroll
-                            for (int i = 0; i < 32; i += 2) {
+                            for (int i = 0; i < CHUNK; i += 2) {
                                 float2 nl2, nd;
                                 vec_pair(i, nl2, nd);
                                 const float2 x = make_float2(__uint_as_float(xv[i]),
@@ -819,7 +904,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         } else {
                             const float2 sl2 = make_float2(P.scale_l2, P.scale_l2);
 #pragma unroll
-                            for (int i = 0; i < 32; i += 2) {
+                            for (int i = 0; i < CHUNK; i += 2) {
                                 float2 nl2, nd;
                                 vec_pair(i, nl2, nd);
                                 const float2 x = make_float2(__uint_as_float(xv[i]),
@@ -840,7 +925,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     } else {
                         // general path: per-element mask, exact cap when |u| > 1/4
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
+                        for (int i = 0; i < CHUNK; i += 2) {
                             float2 nl2v, ndv;
                             vec_pair(i, nl2v, ndv);
                             float pv[2], dsv[2];
@@ -849,7 +934,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                 const int cc = cb + i + e;  // column 0..127
                                 int t, j;
                                 if (KV) {
-                                    t = ccol0 + (cc & 63);  // head 2g + cc/64
+                                    t = ccol0 + (cc & (CQ - 1));  // head 2g + cc/CQ
                                     j = key_row;
                                 } else {
                                     t = t_row;
@@ -886,16 +971,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             pd[i / 2] = pack_bf16x2(dsv[0], dsv[1]);
                         }
                     }
-                    // bf16 pairs of columns cb .. cb+31 go to TMEM columns
-                    // col0 + 16*h2 .. +15: inside this warp's own X / Y columns,
-                    // already read (chunk 0), never the other warp's (no
-                    // ordering between the two warps of a quadrant is needed)
-                    const uint32_t zc = col0 + 16 * h2;
+                    // bf16 pairs of columns cb .. cb+CHUNK-1 go to TMEM columns
+                    // col0 + (CHUNK/2) h2 ..: inside this warp's own X / Y
+                    // columns, already read (chunk 0), never the other warp's
+                    // (no ordering between the two warps of a quadrant is needed)
+                    const uint32_t zc = col0 + (CHUNK / 2) * h2;
                     if (KV) {
-                        tmem_st16(tmem + lane_addr + BW_X_COL + zc, pp);  // P^T
-                        tmem_st16(tmem + lane_addr + BW_Y_COL + zc, pd);  // dS^T
+                        bw_st<CHUNK / 2>(tmem + lane_addr + BW_X_COL + zc, pp);  // P^T
+                        bw_st<CHUNK / 2>(tmem + lane_addr + BW_Y_COL + zc, pd);  // dS^T
                     } else {
-                        tmem_st16(tmem + lane_addr + BW_X_COL + zc, pd);  // dS
+                        bw_st<CHUNK / 2>(tmem + lane_addr + BW_X_COL + zc, pd);  // dS
                     }
                 }
                 tmem_wait_st();
@@ -910,21 +995,29 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            constexpr int HALF = D / 2;  // accumulator columns per warp
+            constexpr int HALF = ACC_N / 2;           // accumulator columns per warp
+            constexpr int SEG = HALF < 64 ? HALF : 64;  // columns per TMEM round trip
             if (KV) {
                 const bool valid = r < U.rvalid;
                 const size_t row = (static_cast<size_t>(U.kbase) + key_row) * P.Hkv + U.g;
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {  // a = 0: dv (columns 0..), a = 1: dk (columns D..)
+                for (int a = 0; a < 2; ++a) {  // a = 0: dv (columns 0..), a = 1: dk (ACC_N..)
                     const float f = a ? P.query_scale : 1.0f;
-                    __nv_bfloat16* dst = (a ? P.dk : P.dv) + row * D + part * HALF;
-                    bw_store_acc<HALF>(tmem + lane_addr + a * D + part * HALF, dst, f, valid);
+                    __nv_bfloat16* dst =
+                        (a ? P.dk : P.dv) + row * D + U.dh * ACC_N + part * HALF;
+#pragma unroll
+                    for (int sg = 0; sg < HALF / SEG; ++sg)
+                        bw_store_acc<SEG>(tmem + lane_addr + a * ACC_N + part * HALF + SEG * sg,
+                                          dst + SEG * sg, f, valid);
                 }
             } else {
                 const bool valid = pr_row < U.rvalid;
                 const size_t row = (static_cast<size_t>(U.qbase) + t_row) * P.H + 2 * U.g + hl_row;
                 __nv_bfloat16* dst = P.dq + row * D + part * HALF;
-                bw_store_acc<HALF>(tmem + lane_addr + part * HALF, dst, P.query_scale, valid);
+#pragma unroll
+                for (int sg = 0; sg < HALF / SEG; ++sg)
+                    bw_store_acc<SEG>(tmem + lane_addr + part * HALF + SEG * sg, dst + SEG * sg,
+                                      P.query_scale, valid);
             }
             tc_fence_before();
             __syncwarp();

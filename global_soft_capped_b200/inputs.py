@@ -77,6 +77,11 @@ WORKLOADS = {
         "27b_backward", "prefill", H=32, Hkv=16, d=128, window_local=4096,
         query_scale=144.0 ** -0.5, softcap=50.0, std=1.0, seed=6, B=1, T=8192, S=8192,
         note="27B-shaped layer pair, forward outputs and upstream gradients for the backward"),
+    # Training-shaped 2B layer pair for the gradients at d = 256
+    "2b_backward": Workload(
+        "2b_backward", "prefill", H=8, Hkv=4, d=256, window_local=4096, query_scale=1.0 / 16,
+        softcap=50.0, std=1.0, seed=8, B=1, T=8192, S=8192,
+        note="2B-shaped layer pair, forward outputs and upstream gradients for the backward"),
     # Packed training batch of the same 27B shape: 8 self-attention sequences of
     # 512-8192 tokens, dout drawn after q, k, v from the same generator
     "27b_varlen_backward": Workload(

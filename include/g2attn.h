@@ -242,9 +242,9 @@ G2ATTN_API size_t g2attn_backward_workspace_size(int B, int T, int H);
  *   workspace: device memory of at least
  *     g2attn_backward_workspace_size(B, T, H) bytes, 16-byte aligned, owned by
  *     the caller and overwritten.
- * Supported: d = 64 and 128 (the 27B and smaller head sizes). d = 256 returns
- * G2ATTN_ERR_UNSUPPORTED: the fused dk/dv kernel keeps both d-column
- * accumulators and two 128-column work tiles in the 512 TMEM columns of an SM.
+ * Supported: d = 64, 128 and 256. At d = 256 the streamed tiles are 32 rows
+ * and the dk/dv kernel runs each 128-key tile as two units, one per half of
+ * the d columns, so that its accumulators fit the 512 TMEM columns of an SM.
  * Other limits and errors as g2attn_prefill; lse is required; a workspace that
  * is missing or too small returns G2ATTN_ERR_WORKSPACE. Three kernels run on
  * `stream`: a pass computing D and lse*log2(e), the dk/dv kernel (K, V tiles
@@ -275,7 +275,7 @@ G2ATTN_API size_t g2attn_varlen_backward_workspace_size(int num_seqs, int total_
  *     total_q, H) bytes, 16-byte aligned, overwritten.
  * Sequence rows derived from cu_seqlens are clamped into [0, total_q) and
  * [0, total_k): malformed offsets give undefined results but no access
- * outside the tensors. Supported: d = 64 and 128; num_seqs <= 1024.
+ * outside the tensors. Supported: d = 64, 128 and 256; num_seqs <= 1024.
  * Other errors as g2attn_prefill_backward. Four kernels run on `stream`: the
  * padded-prefix and D passes, the dk/dv kernel and the dq kernel.
  * Source: as g2attn_prefill_backward; the packing is this library's.

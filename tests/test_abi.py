@@ -169,7 +169,7 @@ def backward_args(**kw):
     (dict(dk=None), g2.G2ATTN_ERR_INVALID_ARG),
     (dict(q_offset=1), g2.G2ATTN_ERR_INVALID_ARG),
     (dict(softcap=-1.0), g2.G2ATTN_ERR_INVALID_ARG),
-    (dict(d=256), g2.G2ATTN_ERR_UNSUPPORTED),               # TMEM budget of the dk/dv kernel
+    (dict(d=96), g2.G2ATTN_ERR_UNSUPPORTED),
     (dict(H=6), g2.G2ATTN_ERR_UNSUPPORTED),
     (dict(workspace=None), g2.G2ATTN_ERR_WORKSPACE),
     (dict(workspace_bytes=1024), g2.G2ATTN_ERR_WORKSPACE),
@@ -204,7 +204,7 @@ def varlen_backward_args(**kw):
     (dict(max_T=129), g2.G2ATTN_ERR_INVALID_ARG),             # above max_S
     (dict(max_S=257), g2.G2ATTN_ERR_INVALID_ARG),             # above total_k
     (dict(window=-2), g2.G2ATTN_ERR_INVALID_ARG),
-    (dict(d=256), g2.G2ATTN_ERR_UNSUPPORTED),
+    (dict(d=32), g2.G2ATTN_ERR_UNSUPPORTED),
     (dict(Hkv=3), g2.G2ATTN_ERR_UNSUPPORTED),
     (dict(num_seqs=1025), g2.G2ATTN_ERR_UNSUPPORTED),         # the kernels' sequence table
     (dict(workspace_bytes=64), g2.G2ATTN_ERR_WORKSPACE),

@@ -61,6 +61,13 @@ CASES = [
     (1, 1, 129, 2, 1, 128, 128, 0, 50.0, 128 ** -0.5),        # a single query
     (1, 64, 1000, 2, 1, 64, 936, 32, 50.0, 0.125),            # keys no query sees: zero grads
     (1, 300, 300, 2, 1, 128, 0, 129, 50.0, 128 ** -0.5),      # window across a tile edge
+    # d = 256: 32-row column tiles, the dk/dv kernel in two d-halves
+    (1, 200, 300, 4, 2, 256, 100, 70, 50.0, 1 / 16),          # ragged, window, chunked
+    (2, 130, 130, 2, 1, 256, 0, 0, 50.0, 1 / 16),             # batch, ragged tail
+    (1, 77, 500, 2, 1, 256, 423, 0, 0.0, 1 / 16),             # no cap
+    (1, 256, 256, 2, 1, 256, 0, 64, 5.0, 1.0),                # logits past the cap
+    (1, 64, 1000, 2, 1, 256, 936, 32, 50.0, 1 / 16),          # keys no query sees: zero grads
+    (1, 1, 33, 2, 1, 256, 32, 0, 50.0, 1 / 16),               # a single query
 ]
 
 
@@ -87,20 +94,33 @@ def test_27b_shaped_backward(layer):
 
 
 @pytest.mark.parametrize("layer", ["local", "global"])
-def test_full_size_value_gradient_invariant(layer):
-    """At the full 27B-shaped size (T = S = 8192): the softmax weights of each
+def test_2b_shaped_backward(layer):
+    """2B head layout (H=8, Hkv=4, d=256, query_scale 1/16) at T = S = 1024."""
+    W = 256 if layer == "local" else 0
+    (q, k, v, dout), grads = _run(1, 1024, 1024, 8, 4, 256, 0, W, 50.0, 1 / 16, seed=5)
+    ref = oracle.attn_bwd(q, k, v, dout, query_scale=1 / 16, softcap=50.0, window=W)
+    _check(grads, ref)
+
+
+@pytest.mark.parametrize("shape", ["27b", "2b"])
+@pytest.mark.parametrize("layer", ["local", "global"])
+def test_full_size_value_gradient_invariant(layer, shape):
+    """At full size (T = S = 8192, 27B and 2B head layouts): the softmax weights of each
     row sum to one, so the value gradients of KV head g add up to the upstream
     gradients of all rows of its two query heads. Also: two runs agree bitwise
     (no atomics anywhere)."""
     W = 4096 if layer == "local" else 0
-    B, T, S, H, Hkv, d = 1, 8192, 8192, 32, 16, 128
+    if shape == "27b":
+        B, T, S, H, Hkv, d, alpha = 1, 8192, 8192, 32, 16, 128, 144 ** -0.5
+    else:
+        B, T, S, H, Hkv, d, alpha = 1, 8192, 8192, 8, 4, 256, 1 / 16
     q, k, v = (t.cuda() for t in prefill_inputs(B, T, S, H, Hkv, d, 1.0, 3))
     dout = _dout(B, T, H, d, 4).cuda()
-    out, lse = g2.prefill(q, k, v, query_scale=144 ** -0.5, softcap=50.0, window=W)
+    out, lse = g2.prefill(q, k, v, query_scale=alpha, softcap=50.0, window=W)
     ws = g2.backward_workspace(B, T, H)
-    dq, dk, dv = g2.prefill_backward(q, k, v, out, lse, dout, query_scale=144 ** -0.5,
+    dq, dk, dv = g2.prefill_backward(q, k, v, out, lse, dout, query_scale=alpha,
                                      softcap=50.0, window=W, workspace=ws)
-    dq2, dk2, dv2 = g2.prefill_backward(q, k, v, out, lse, dout, query_scale=144 ** -0.5,
+    dq2, dk2, dv2 = g2.prefill_backward(q, k, v, out, lse, dout, query_scale=alpha,
                                         softcap=50.0, window=W, workspace=ws)
     torch.cuda.synchronize()
     assert g2.g2attn_get_device_error() == g2.G2ATTN_OK

@@ -74,6 +74,8 @@ FIXED = [
     ([(333, 333), (17, 250), (128, 128)], 2, 1, 64, 0, 50.0),
     ([(333, 333), (17, 250), (128, 128)], 6, 3, 64, 65, 0.0),
     ([(700, 700)], 2, 1, 128, 257, 50.0),
+    ([(200, 300), (0, 77), (1, 1), (64, 64), (129, 400)], 4, 2, 256, 100, 50.0),
+    ([(333, 333), (17, 250), (33, 33)], 2, 1, 256, 0, 0.0),
 ]
 
 
@@ -84,7 +86,8 @@ def test_varlen_backward_fixed(case):
     _close(grads, ref, case)
 
 
-RANDOM = [c for c in _varlen_cases(30, 31337) if c[3] in (64, 128)][:8]
+RANDOM = ([c for c in _varlen_cases(30, 31337) if c[3] in (64, 128)][:8] +
+          [c for c in _varlen_cases(30, 2718) if c[3] == 256][:4])
 
 
 @pytest.mark.parametrize("case", RANDOM, ids=[str(i) for i in range(len(RANDOM))])
@@ -94,10 +97,11 @@ def test_varlen_backward_random(case):
     _close(grads, ref, case)
 
 
-def test_single_sequence_matches_dense_bitwise():
+@pytest.mark.parametrize("d", [128, 256])
+def test_single_sequence_matches_dense_bitwise(d):
     """One packed sequence runs the same units in the same order as the dense
     call with B = 1 and q_offset = S - T, so the gradients agree bit for bit."""
-    T, S, H, Hkv, d = 300, 520, 4, 2, 128
+    T, S, H, Hkv = 300, 520, 4, 2
     Ts, Ss, cq, ck, q, k, v = varlen_inputs(0, 0, 0, H, Hkv, d, 1.0, 5, seq_lens=[(T, S)])
     g = torch.Generator().manual_seed(6)
     dout = torch.randn(q.shape, generator=g).to(torch.bfloat16).cuda()

@@ -91,7 +91,8 @@ def test_random_varlen(case):
     check(out, ro, lse, rl, what=str(case))
 
 
-BACKWARD = [c for c in _dense_cases(40, 4242) if c[5] in (64, 128)][:8]
+BACKWARD = ([c for c in _dense_cases(40, 4242) if c[5] in (64, 128)][:8] +
+            [c for c in _dense_cases(40, 9898) if c[5] == 256][:6])
 
 
 @pytest.mark.parametrize("case", BACKWARD, ids=[str(i) for i in range(len(BACKWARD))])
