@@ -662,6 +662,26 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                IDESC_XY, kk != 0);
                 umma_commit(&xy_full[h]);
             };
+            // Both halves of the tile in slot sl as one UMMA pair (N = CR): with
+            // 32-row column tiles (d = 256) an N = 16 half re-reads the whole
+            // 128-row resident A tile per UMMA, which makes shared-memory
+            // bandwidth the limit; one N = 32 UMMA reads it once per tile.
+            auto issue_xy_tile = [&](int sl) {
+                constexpr uint32_t IDESC_XYT = idesc_bf16(128, C::CR, false);
+                const uint32_t c1 = slot_lo + sl * SLOT_STEP;
+                const uint32_t c2 = c1 + CTILE_STEP;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_lh(tmem + BW_X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                               IDESC_XYT, kk != 0);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_lh(tmem + BW_Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                               IDESC_XYT, kk != 0);
+                umma_commit(&xy_full[0]);
+                umma_commit(&xy_full[1]);
+            };
+            constexpr bool TILE_XY = HW < 32;
             // accumulations over the half's HW rows (K indices HW h ..): A = the
             // bf16 operand the half's warps wrote at columns HW h + 8 k4; B =
             // the streamed tiles' columns of d-half dh (ACC_N columns)
@@ -691,7 +711,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             // Issue order per tile c (slot sl): XY_0(c) XY_1(c) | z_0 | ACC_0(c)
             // XY_0(c+1) | z_1 | ACC_1(c) XY_1(c+1). A half's X / Y overwrite
             // that half's P / dS only after the accumulation reading them was
-            // issued; UMMAs of one thread execute in issue order.
+            // issued; UMMAs of one thread execute in issue order. With whole-
+            // tile X / Y (TILE_XY): XY(c) | z_0 | ACC_0(c) | z_1 | ACC_1(c) XY(c+1).
             for (int r = 0; ok && r * G < num_units; ++r) {
                 const int u = bw_sched(r, cta, G);
                 if (u >= num_units) continue;
@@ -704,8 +725,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
                 tc_fence_after();
-                issue_xy(ct & 1, 0);
-                issue_xy(ct & 1, 1);
+                if constexpr (TILE_XY) {
+                    issue_xy_tile(ct & 1);
+                } else {
+                    issue_xy(ct & 1, 0);
+                    issue_xy(ct & 1, 1);
+                }
                 for (int c = 0; c < U.ncols; ++c) {
                     const int sl = ct & 1;
                     const bool next = c + 1 < U.ncols;
@@ -717,7 +742,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     }
                     tc_fence_after();
                     issue_acc(sl, 0, U.dh, c == 0);
-                    if (next) {
+                    if (next && !TILE_XY) {
                         ok = mbar_wait(&c_full[sl ^ 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
                                        SITE_BW_MMA);
                         if (!ok) break;
@@ -729,7 +754,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     tc_fence_after();
                     issue_acc(sl, 1, U.dh, false);
                     umma_commit(&c_empty[sl]);
-                    if (next) issue_xy(sl ^ 1, 1);
+                    if (next) {
+                        if constexpr (TILE_XY) {
+                            ok = mbar_wait(&c_full[sl ^ 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
+                                           SITE_BW_MMA);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_xy_tile(sl ^ 1);
+                        } else {
+                            issue_xy(sl ^ 1, 1);
+                        }
+                    }
                     ++ct;
                 }
                 if (!ok) break;
