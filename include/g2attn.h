@@ -1,6 +1,6 @@
 /*
- * g2attn.h -- libg2attn: Gemma 2 soft-capped local/global attention forward
- * for NVIDIA B200 (sm_100a).
+ * g2attn.h -- libg2attn: Gemma 2 soft-capped local/global attention (forward,
+ * decode and gradients) for NVIDIA B200 (sm_100a).
  *
  * The operation (Gemma 2 card, "Method", per-layer attention pseudo-code; the
  * soft-cap formula is the "Gemma 2 Guide", section 1): for every query row i
@@ -54,7 +54,7 @@ typedef enum {
     G2ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
     G2ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
     G2ATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting (see g2attn_get_device_error) */
-    G2ATTN_ERR_WORKSPACE = 6       /* decode workspace NULL or smaller than required */
+    G2ATTN_ERR_WORKSPACE = 6       /* a workspace NULL or smaller than required */
 } g2attn_status;
 
 /*
