@@ -340,9 +340,10 @@ __device__ __forceinline__ int bw_sched(int r, int c, int G) {
     return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-// 128-row tile of a (rows, heads, d) tensor into shared memory: D/64 boxes of
-// 64 d-columns (128-byte swizzle). `two_heads`: 64 positions x heads 2g, 2g+1
-// (query-side tensors); else 128 rows of head g (key-side tensors).
+// A `rows`-row tile of a (rows, heads, d) tensor into shared memory: D/64
+// boxes of 64 d-columns (128-byte swizzle), `rows` x 128 B apart. The tensor
+// map's box gives the rows: query-side maps take rows/2 positions of heads 2g
+// and 2g+1, key-side maps `rows` keys of head g.
 template <int D>
 __device__ __forceinline__ void bw_load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
                                              int row, int head, int rows = 128) {
@@ -445,8 +446,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* r_empty = bars + 1;
     uint64_t* c_full = bars + 2;    // [2]
     uint64_t* c_empty = bars + 4;   // [2]
-    // Column halves h = 0, 1 (columns 0..63 / 64..127 of X and Y, the column
-    // parts of the elementwise warps) run as a two-stage pipeline:
+    // Column halves h = 0, 1 (columns HW h .. HW h + HW - 1 of X and Y, the
+    // column parts of the elementwise warps) run as a two-stage pipeline:
     uint64_t* xy_full = bars + 6;   // [2] X and Y of half h of the current tile are in TMEM
     uint64_t* z_full = bars + 8;    // [2] P / dS of half h written back (4 warp arrivals)
     uint64_t* acc_done = bars + 10; // last accumulation of the unit completed
