@@ -4,6 +4,7 @@ checks run without a GPU: no compute call is made)."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -213,3 +214,23 @@ def varlen_backward_args(**kw):
 ])
 def test_varlen_backward_rejects_before_launch(lib, kw, status):
     assert g2.g2attn_prefill_varlen_backward(*varlen_backward_args(**kw)) == status
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/g2attn.h compiles as C99 (no C++ in the interface), and a C
+    program that calls every declared entry point links against the library
+    (the program is built, not run)."""
+    names = declared_symbols()
+    calls = "\n".join(f"    (void)&{n};" for n in names)
+    src = tmp_path / "use.c"
+    src.write_text('#include "g2attn.h"\nint main(void) {\n' + calls + "\n    return 0;\n}\n")
+    lib_dir = os.path.dirname(g2.LIB_PATH)
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                          str(src), "-L", lib_dir, "-lg2attn", "-o", str(tmp_path / "use")],
+                         capture_output=True, text=True)
+    if res.returncode != 0 and "cannot find -lg2attn" in res.stderr:
+        # the library is named libg2attn.so in-tree; link by path instead
+        res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I",
+                              os.path.join(ROOT, "include"), str(src), g2.LIB_PATH,
+                              "-o", str(tmp_path / "use")], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
