@@ -234,3 +234,15 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
                               os.path.join(ROOT, "include"), str(src), g2.LIB_PATH,
                               "-o", str(tmp_path / "use")], capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_binding_argument_counts_match_header(lib):
+    """Every ctypes prototype has as many arguments as the header declares
+    (a miscounted marshalling list would shift every later argument)."""
+    text = open(HEADER).read()
+    decls = re.findall(r"G2ATTN_API\s+[\w\s\*]*?\b(g2attn_\w+)\s*\(([^)]*)\)\s*;", text)
+    assert sorted(n for n, _ in decls) == sorted(g2.EXPORTS)
+    for name, params in decls:
+        params = " ".join(params.split())
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(getattr(lib, name).argtypes) == n, name
