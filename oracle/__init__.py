@@ -14,6 +14,7 @@ Functions (each follows the Gemma 2 card's per-layer attention pseudo-code,
 * :func:`decode`      one query per sequence at position L-1 of its cache
 * :func:`varlen`      packed sequences, each a dense layer with q_offset = S_i - T_i
 * :func:`attn_bwd`    gradients of the dense layer (dq, dk, dv) for an upstream dout
+* :func:`attn_bwd_sampled`  the same gradients at chosen query rows and chosen keys
 
 Parity of every function is pinned by ``tests/test_oracle_pins.py`` (the
 gradients by ``tests/test_oracle_backward_pins.py``).
@@ -62,6 +63,9 @@ def _load():
         lib.g2ref_row_detail.restype = ctypes.c_int
         lib.g2ref_attn_bwd.argtypes = [P] * 7 + [I64] * 7 + [D, D, I64]
         lib.g2ref_attn_bwd.restype = ctypes.c_int
+        lib.g2ref_attn_bwd_sampled.argtypes = [P] * 5 + [I64, P, I64] + [P] * 3 + [I64] * 7 + [
+            D, D, I64]
+        lib.g2ref_attn_bwd_sampled.restype = ctypes.c_int
         lib.g2ref_set_threads.argtypes = [ctypes.c_int]
         lib.g2ref_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -157,6 +161,36 @@ def attn_bwd(q, k, v, dout, q_offset=0, query_scale=1.0, softcap=50.0, window=0)
                                 float(softcap), int(window))
     if rc != 0:
         raise ValueError("g2ref_attn_bwd rejected its arguments")
+    return dq, dk, dv
+
+
+def attn_bwd_sampled(q, k, v, dout, qrows, keys, q_offset=0, query_scale=1.0, softcap=50.0,
+                     window=0):
+    """Gradients of :func:`attn` at chosen places, for layers too large for
+    :func:`attn_bwd`.
+
+    ``qrows`` is (nq, 3) of (b, i, h) and ``keys`` (nk, 3) of (b, j, g), g a
+    KV head. Returns (dq (nq,d), dk (nk,d), dv (nk,d)) float64: dq[b,i,h,:],
+    and dk[b,j,g,:], dv[b,j,g,:] summed over every row of the group's heads
+    that sees key j. Same chain rule as :func:`attn_bwd`; the weights a key
+    needs come from the statistics (lse, D) of the rows that see it.
+    """
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, T, H, d = qb.shape
+    S, Hkv = kb.shape[1], kb.shape[2]
+    assert kb.shape == (B, S, Hkv, d) and vb.shape == kb.shape and gb.shape == qb.shape
+    qrows = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64).reshape(-1, 3))
+    keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64).reshape(-1, 3))
+    nq, nk = qrows.shape[0], keys.shape[0]
+    dq = np.empty((nq, d), np.float64)
+    dk = np.empty((nk, d), np.float64)
+    dv = np.empty((nk, d), np.float64)
+    rc = _load().g2ref_attn_bwd_sampled(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(qrows), nq,
+                                        _ptr(keys), nk, _ptr(dq), _ptr(dk), _ptr(dv), B, T, S, H,
+                                        Hkv, d, int(q_offset), float(query_scale),
+                                        float(softcap), int(window))
+    if rc != 0:
+        raise ValueError("g2ref_attn_bwd_sampled rejected its arguments")
     return dq, dk, dv
 
 

@@ -258,6 +258,154 @@ int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     return err ? -1 : 0;
 }
 
+/* Gradients at chosen query rows and chosen keys (see g2ref.h), for layers
+ * too large for g2ref_attn_bwd. The same chain rule as above, in two passes:
+ * first every row that a chosen key can reach gets its softmax statistics
+ * (lse and D = sum_j w_j dw_j, by one_row and the same dw loop); then each
+ * chosen key sums its terms over those rows, each weight recovered from the
+ * row's lse as w = exp(s - lse). dq rows are formed exactly as above. */
+int g2ref_attn_bwd_sampled(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const uint16_t* dout, const int64_t* qrows, int64_t nq,
+                           const int64_t* keys, int64_t nk, double* dq, double* dk, double* dv,
+                           int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                           int64_t q_offset, double query_scale, double softcap,
+                           int64_t window) {
+    if (check_args(B, T, S, H, Hkv, d, q_offset, softcap, window)) return -1;
+    const int64_t group = H / Hkv;
+    for (int64_t r = 0; r < nq; ++r) {
+        const int64_t b = qrows[3 * r], i = qrows[3 * r + 1], h = qrows[3 * r + 2];
+        if (b < 0 || b >= B || i < 0 || i >= T || h < 0 || h >= H) return -1;
+    }
+    for (int64_t r = 0; r < nk; ++r) {
+        const int64_t b = keys[3 * r], j = keys[3 * r + 1], g = keys[3 * r + 2];
+        if (b < 0 || b >= B || j < 0 || j >= S || g < 0 || g >= Hkv) return -1;
+    }
+    /* which (b, g) have a chosen key: only their rows need statistics */
+    unsigned char* need = (unsigned char*)calloc((size_t)(B * Hkv), 1);
+    double* row_lse = (double*)malloc(sizeof(double) * (size_t)(B * T * H));
+    double* row_D = (double*)malloc(sizeof(double) * (size_t)(B * T * H));
+    if (!need || !row_lse || !row_D) {
+        free(need);
+        free(row_lse);
+        free(row_D);
+        return -1;
+    }
+    for (int64_t r = 0; r < nk; ++r) need[keys[3 * r] * Hkv + keys[3 * r + 2]] = 1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* qs = (double*)malloc(sizeof(double) * (size_t)d);
+        double* s = (double*)malloc(sizeof(double) * (size_t)S);
+        double* w = (double*)malloc(sizeof(double) * (size_t)S);
+        double* x = (double*)malloc(sizeof(double) * (size_t)S);
+        if (!qs || !s || !w || !x) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            /* pass 1a: dq of the chosen rows (the row loop of g2ref_attn_bwd) */
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nq; ++r) {
+                const int64_t b = qrows[3 * r], i = qrows[3 * r + 1], h = qrows[3 * r + 2];
+                const int64_t g = h / group;
+                one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale, softcap,
+                        window, qs, s, w, NULL, NULL);
+                const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
+                double D = 0.0;
+                for (int64_t j = 0; j < S; ++j) {
+                    x[j] = 0.0;
+                    if (w[j] == 0.0) continue;
+                    const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
+                    double dw = 0.0;
+                    for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
+                    x[j] = dw;
+                    D += w[j] * dw;
+                }
+                double* dqrow = dq + r * d;
+                for (int64_t c = 0; c < d; ++c) dqrow[c] = 0.0;
+                for (int64_t j = 0; j < S; ++j) {
+                    if (w[j] == 0.0) continue;
+                    const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
+                    double dx = w[j] * (x[j] - D);
+                    if (softcap > 0.0) {
+                        double xl = 0.0;
+                        for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
+                        const double t = tanh(xl / softcap);
+                        dx *= 1.0 - t * t;
+                    }
+                    for (int64_t c = 0; c < d; ++c) dqrow[c] += query_scale * dx * widen(krow[c]);
+                }
+            }
+            /* pass 1b: lse and D of every row of a (b, g) that has a chosen key */
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t r = 0; r < B * T * H; ++r) {
+                const int64_t b = r / (T * H);
+                const int64_t i = (r / H) % T;
+                const int64_t h = r % H;
+                const int64_t g = h / group;
+                if (!need[b * Hkv + g]) continue;
+                double lse;
+                one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale, softcap,
+                        window, qs, s, w, NULL, &lse);
+                const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
+                double D = 0.0;
+                for (int64_t j = 0; j < S; ++j) {
+                    if (w[j] == 0.0) continue;
+                    const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
+                    double dw = 0.0;
+                    for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
+                    D += w[j] * dw;
+                }
+                row_lse[(b * H + h) * T + i] = lse;
+                row_D[(b * H + h) * T + i] = D;
+            }
+            /* pass 2: dk and dv of each chosen key, summed over the rows of
+             * both heads of its group that see it */
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nk; ++r) {
+                const int64_t b = keys[3 * r], j = keys[3 * r + 1], g = keys[3 * r + 2];
+                const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
+                const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
+                double* dkrow = dk + r * d;
+                double* dvrow = dv + r * d;
+                for (int64_t c = 0; c < d; ++c) dkrow[c] = dvrow[c] = 0.0;
+                for (int64_t h = g * group; h < (g + 1) * group; ++h) {
+                    for (int64_t i = 0; i < T; ++i) {
+                        if (!visible(i + q_offset, j, window)) continue;
+                        const uint16_t* qrow = q + ((b * T + i) * H + h) * d;
+                        const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
+                        for (int64_t c = 0; c < d; ++c) qs[c] = query_scale * widen(qrow[c]);
+                        /* x = (query_scale q) . k, the capped logit and its weight */
+                        double xl = 0.0;
+                        for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
+                        double sl = xl, cap_grad = 1.0;
+                        if (softcap > 0.0) {
+                            const double t = tanh(xl / softcap);
+                            sl = softcap * t;
+                            cap_grad = 1.0 - t * t;
+                        }
+                        const double wl = exp(sl - row_lse[(b * H + h) * T + i]);
+                        double dw = 0.0;
+                        for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
+                        const double dx = wl * (dw - row_D[(b * H + h) * T + i]) * cap_grad;
+                        for (int64_t c = 0; c < d; ++c) {
+                            dkrow[c] += dx * qs[c];
+                            dvrow[c] += wl * widen(dorow[c]);
+                        }
+                    }
+                }
+            }
+        }
+        free(qs);
+        free(s);
+        free(w);
+        free(x);
+    }
+    free(need);
+    free(row_lse);
+    free(row_D);
+    return err ? -1 : 0;
+}
+
 void g2ref_set_threads(int n) {
 #ifdef _OPENMP
     if (n > 0) omp_set_num_threads(n);

@@ -69,6 +69,21 @@ int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                    int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
                    int64_t q_offset, double query_scale, double softcap, int64_t window);
 
+/* The same gradients at chosen places, for layers whose full gradients are
+ * too costly in fp64: qrows holds nq triples (b, i, h) and keys nk triples
+ * (b, j, g) (g a KV head). dq (nq, d) gets dq[b,i,h,:]; dk and dv (nk, d) get
+ * dk[b,j,g,:] and dv[b,j,g,:], each summed over every row of the group's
+ * heads that sees key j. The softmax statistics of those rows (lse and
+ * D = sum_j w_j dw_j) are computed first, and each weight is then
+ * w_j = exp(s_j - lse). Returns -1 on an argument error or an index outside
+ * the tensors. */
+int g2ref_attn_bwd_sampled(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const uint16_t* dout, const int64_t* qrows, int64_t nq,
+                           const int64_t* keys, int64_t nk, double* dq, double* dk, double* dv,
+                           int64_t B, int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
+                           int64_t q_offset, double query_scale, double softcap,
+                           int64_t window);
+
 /* Threads used by the OpenMP loops (0 leaves the runtime default). */
 void g2ref_set_threads(int n);
 int g2ref_max_threads(void);

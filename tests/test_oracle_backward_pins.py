@@ -175,3 +175,69 @@ def test_saturated_cap_stops_query_and_key_gradients():
     dq, dk, dv = oracle.attn_bwd(q, k, v, dout, query_scale=400.0, softcap=1.0, window=0)
     assert np.abs(dv).max() > 1.0
     assert np.abs(dq).max() < 1e-5 and np.abs(dk).max() < 1e-5
+
+
+def _edge_places(B, T, S, H, Hkv, q_offset, window, rng, n_random=6):
+    """Query rows and keys at both ends, around the diagonal and the window
+    edge, plus random ones."""
+    rows = set()
+    for i in {0, 1, T // 2, T - 2, T - 1} | set(int(x) for x in rng.integers(0, T, n_random)):
+        if 0 <= i < T:
+            rows.add((int(rng.integers(0, B)), i, int(rng.integers(0, H))))
+    keys = set()
+    js = {0, 1, q_offset, q_offset + 1, S - 2, S - 1} | set(int(x) for x in rng.integers(0, S, n_random))
+    if window:
+        js |= {q_offset + window - 1 - T // 2, S - window, S - window + 1}
+    for j in js:
+        if 0 <= j < S:
+            keys.add((int(rng.integers(0, B)), j, int(rng.integers(0, Hkv))))
+    return sorted(rows), sorted(keys)
+
+
+@pytest.mark.parametrize("cap,window,q_offset,H,Hkv", [
+    (50.0, 0, 0, 4, 2), (2.0, 6, 3, 4, 2), (0.0, 5, 9, 2, 1), (4.0, 1, 2, 8, 4)])
+def test_sampled_gradients_match_autograd(cap, window, q_offset, H, Hkv):
+    """attn_bwd_sampled at chosen rows and keys equals fp64 autograd of the
+    plain PyTorch forward above, entry by entry."""
+    B, T, S, d = 2, 21, 30, 16
+    q, k, v, dout = _inputs(B, T, S, H, Hkv, d, std=2.0, seed=11)
+    scale = 0.45
+    rows, keys = _edge_places(B, T, S, H, Hkv, q_offset, window, np.random.default_rng(1))
+    dq, dk, dv = oracle.attn_bwd_sampled(q, k, v, dout, rows, keys, q_offset=q_offset,
+                                         query_scale=scale, softcap=cap, window=window)
+    Q = q.to(torch.float64).requires_grad_()
+    K = k.to(torch.float64).requires_grad_()
+    V = v.to(torch.float64).requires_grad_()
+    out = _torch_forward(Q, K, V, q_offset, scale, cap, window)
+    (out * dout.to(torch.float64)).sum().backward()
+    ref_q = np.stack([Q.grad[b, i, h].numpy() for b, i, h in rows])
+    ref_k = np.stack([K.grad[b, j, g].numpy() for b, j, g in keys])
+    ref_v = np.stack([V.grad[b, j, g].numpy() for b, j, g in keys])
+    np.testing.assert_allclose(dq, ref_q, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, ref_k, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, ref_v, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("cap,window,q_offset", [(50.0, 0, 0), (50.0, 9, 12), (0.0, 4, 3)])
+def test_sampled_gradients_equal_full_gradients(cap, window, q_offset):
+    """Every row and every key through attn_bwd_sampled equals attn_bwd (the
+    finite-difference and autograd pinned routine) to rounding."""
+    B, T, S, H, Hkv, d = 2, 33, 45, 4, 2, 8
+    q, k, v, dout = _inputs(B, T, S, H, Hkv, d, std=1.5, seed=12)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, q_offset=q_offset, query_scale=0.6,
+                                 softcap=cap, window=window)
+    rows = [(b, i, h) for b in range(B) for i in range(T) for h in range(H)]
+    keys = [(b, j, g) for b in range(B) for j in range(S) for g in range(Hkv)]
+    sq, sk, sv = oracle.attn_bwd_sampled(q, k, v, dout, rows, keys, q_offset=q_offset,
+                                         query_scale=0.6, softcap=cap, window=window)
+    np.testing.assert_allclose(sq, dq.reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sk, dk.reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sv, dv.reshape(-1, d), rtol=0, atol=1e-12)
+
+
+def test_sampled_gradients_reject_out_of_range_places():
+    q, k, v, dout = _inputs(1, 4, 6, 2, 1, 8, std=1.0, seed=2)
+    with pytest.raises(ValueError):
+        oracle.attn_bwd_sampled(q, k, v, dout, [(0, 4, 0)], [(0, 0, 0)])
+    with pytest.raises(ValueError):
+        oracle.attn_bwd_sampled(q, k, v, dout, [(0, 0, 0)], [(0, 0, 1)])

@@ -40,6 +40,18 @@ MUTANTS = {
         "dqrow[c] += query_scale * dx * widen(krow[c]);", "dqrow[c] += dx * widen(krow[c]);"),
     "backward: dv without the weight": (
         "dvrow[c] += w[j] * widen(dorow[c]);", "dvrow[c] += widen(dorow[c]);"),
+    # gradients at chosen rows and keys
+    "sampled backward: key terms without the row's D": (
+        "const double dx = wl * (dw - row_D[(b * H + h) * T + i]) * cap_grad;",
+        "const double dx = wl * dw * cap_grad;"),
+    "sampled backward: weight from the uncapped logit": (
+        "const double wl = exp(sl - row_lse", "const double wl = exp(xl - row_lse"),
+    "sampled backward: key seen one row late": (
+        "if (!visible(i + q_offset, j, window)) continue;",
+        "if (!visible(i + q_offset + 1, j, window)) continue;"),
+    "sampled backward: one head of the group only": (
+        "for (int64_t h = g * group; h < (g + 1) * group; ++h) {\n                    for (int64_t i = 0; i < T; ++i) {\n                        if (!visible",
+        "for (int64_t h = g * group; h < g * group + 1; ++h) {\n                    for (int64_t i = 0; i < T; ++i) {\n                        if (!visible"),
 }
 
 
