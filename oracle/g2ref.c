@@ -44,6 +44,16 @@ static int visible(int64_t p, int64_t j, int64_t window) {
     return 1;
 }
 
+/* The KV head that query head h shares: the card's "every two query heads
+ * share one" read as consecutive heads (h / group). */
+static int64_t kv_head(int64_t h, int64_t H, int64_t Hkv) { return h / (H / Hkv); }
+
+/* queries = queries * query_scale (the card's pseudo-code scales the query
+ * row before the dot products). */
+static void scaled_query(const uint16_t* qrow, int64_t d, double query_scale, double* qs) {
+    for (int64_t c = 0; c < d; ++c) qs[c] = query_scale * widen(qrow[c]);
+}
+
 /* Capped logit of key j for the (already scaled) query qs.
  * Soft-cap formula: "Gemma 2 Guide", section 1, cap_val * tanh(logits / cap_val),
  * with cap_val = 50 for attention; the card applies it to every logit before
@@ -62,13 +72,9 @@ static void one_row(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     int64_t T, int64_t S, int64_t H, int64_t Hkv, int64_t d,
                     int64_t q_offset, double query_scale, double softcap, int64_t window,
                     double* qs, double* s, double* w, double* out_row, double* lse) {
-    const int64_t group = H / Hkv;
-    const int64_t g = h / group;
+    const int64_t g = kv_head(h, H, Hkv);
     const int64_t p = i + q_offset;
-    const uint16_t* qrow = q + ((b * T + i) * H + h) * d;
-
-    /* queries = queries * query_scale */
-    for (int64_t c = 0; c < d; ++c) qs[c] = query_scale * widen(qrow[c]);
+    scaled_query(q + ((b * T + i) * H + h) * d, d, query_scale, qs);
 
     /* logits -> soft-cap -> where(mask, logits, -inf) */
     for (int64_t j = 0; j < S; ++j) {
@@ -180,6 +186,57 @@ int g2ref_row_detail(const uint16_t* q, const uint16_t* k,
     return 0;
 }
 
+/* Backward of one query row (b, i, h) whose forward (qs, w) one_row has just
+ * formed: dw_j = dout . v_j, D = sum_j w_j dw_j, then for every visible key
+ * ds_j = w_j (dw_j - D) and dx_j = ds_j (1 - tanh^2(x_j / C)). Adds the row's
+ * dq (dqrow), and its terms of dk and dv (rows of the (b, g) slices, when
+ * given). Returns D. x holds S doubles of scratch. */
+static double row_backward(const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                           int64_t b, int64_t i, int64_t h, int64_t T, int64_t S, int64_t H,
+                           int64_t Hkv, int64_t d, double query_scale, double softcap,
+                           const double* qs, const double* w, double* x, double* dqrow,
+                           double* dk, double* dv) {
+    const int64_t g = kv_head(h, H, Hkv);
+    const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
+    /* dw_j = dout . v_j, and D = sum_j w_j dw_j */
+    double D = 0.0;
+    for (int64_t j = 0; j < S; ++j) {
+        x[j] = 0.0;
+        if (w[j] == 0.0) continue;
+        const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
+        double dw = 0.0;
+        for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
+        x[j] = dw; /* holds dw_j until ds_j is formed */
+        D += w[j] * dw;
+    }
+    if (!dqrow && !dk && !dv) return D;
+    for (int64_t j = 0; j < S; ++j) {
+        if (w[j] == 0.0) continue;
+        const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
+        /* softmax: ds_j = w_j (dw_j - D) */
+        double dx = w[j] * (x[j] - D);
+        /* cap: d(C tanh(x/C))/dx = 1 - tanh^2(x/C), with x the scaled logit */
+        if (softcap > 0.0) {
+            double xl = 0.0;
+            for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
+            const double t = tanh(xl / softcap);
+            dx *= 1.0 - t * t;
+        }
+        /* x = (query_scale q) . k */
+        if (dqrow)
+            for (int64_t c = 0; c < d; ++c) dqrow[c] += query_scale * dx * widen(krow[c]);
+        if (dk) {
+            double* dkrow = dk + ((b * S + j) * Hkv + g) * d;
+            for (int64_t c = 0; c < d; ++c) dkrow[c] += dx * qs[c];
+        }
+        if (dv) {
+            double* dvrow = dv + ((b * S + j) * Hkv + g) * d;
+            for (int64_t c = 0; c < d; ++c) dvrow[c] += w[j] * widen(dorow[c]);
+        }
+    }
+    return D;
+}
+
 /* Gradients (see g2ref.h). Each (b, g) owns dk[b,:,g,:] and dv[b,:,g,:] and
  * the dq rows of its heads, so the parallel loop runs over (b, g). */
 int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -198,8 +255,7 @@ int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         double* s = (double*)malloc(sizeof(double) * (size_t)S);
         double* w = (double*)malloc(sizeof(double) * (size_t)S);
         double* x = (double*)malloc(sizeof(double) * (size_t)S);
-        double* out_row = (double*)malloc(sizeof(double) * (size_t)d);
-        if (!qs || !s || !w || !x || !out_row) {
+        if (!qs || !s || !w || !x) {
 #pragma omp atomic write
             err = 1;
         } else {
@@ -210,41 +266,9 @@ int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     for (int64_t i = 0; i < T; ++i) {
                         /* forward of this row: s, w (and qs = query_scale * q) */
                         one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale,
-                                softcap, window, qs, s, w, out_row, NULL);
-                        const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
-                        /* dw_j = dout . v_j, and D = sum_j w_j dw_j */
-                        double D = 0.0;
-                        for (int64_t j = 0; j < S; ++j) {
-                            x[j] = 0.0;
-                            if (w[j] == 0.0) continue;
-                            const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
-                            double dw = 0.0;
-                            for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
-                            x[j] = dw; /* holds dw_j until ds_j is formed */
-                            D += w[j] * dw;
-                        }
-                        double* dqrow = dq + ((b * T + i) * H + h) * d;
-                        for (int64_t j = 0; j < S; ++j) {
-                            if (w[j] == 0.0) continue;
-                            const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
-                            /* softmax: ds_j = w_j (dw_j - D) */
-                            double dx = w[j] * (x[j] - D);
-                            /* cap: d(C tanh(x/C))/dx = 1 - tanh^2(x/C), with x the scaled logit */
-                            if (softcap > 0.0) {
-                                double xl = 0.0;
-                                for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
-                                const double t = tanh(xl / softcap);
-                                dx *= 1.0 - t * t;
-                            }
-                            /* x = (query_scale q) . k */
-                            double* dkrow = dk + ((b * S + j) * Hkv + g) * d;
-                            double* dvrow = dv + ((b * S + j) * Hkv + g) * d;
-                            for (int64_t c = 0; c < d; ++c) {
-                                dqrow[c] += query_scale * dx * widen(krow[c]);
-                                dkrow[c] += dx * qs[c];
-                                dvrow[c] += w[j] * widen(dorow[c]);
-                            }
-                        }
+                                softcap, window, qs, s, w, NULL, NULL);
+                        row_backward(k, v, dout, b, i, h, T, S, H, Hkv, d, query_scale,
+                                     softcap, qs, w, x, dq + ((b * T + i) * H + h) * d, dk, dv);
                     }
                 }
             }
@@ -253,7 +277,6 @@ int g2ref_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         free(s);
         free(w);
         free(x);
-        free(out_row);
     }
     return err ? -1 : 0;
 }
@@ -302,38 +325,16 @@ int g2ref_attn_bwd_sampled(const uint16_t* q, const uint16_t* k, const uint16_t*
 #pragma omp atomic write
             err = 1;
         } else {
-            /* pass 1a: dq of the chosen rows (the row loop of g2ref_attn_bwd) */
+            /* pass 1a: dq of the chosen rows, as in g2ref_attn_bwd */
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < nq; ++r) {
                 const int64_t b = qrows[3 * r], i = qrows[3 * r + 1], h = qrows[3 * r + 2];
-                const int64_t g = h / group;
                 one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale, softcap,
                         window, qs, s, w, NULL, NULL);
-                const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
-                double D = 0.0;
-                for (int64_t j = 0; j < S; ++j) {
-                    x[j] = 0.0;
-                    if (w[j] == 0.0) continue;
-                    const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
-                    double dw = 0.0;
-                    for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
-                    x[j] = dw;
-                    D += w[j] * dw;
-                }
                 double* dqrow = dq + r * d;
                 for (int64_t c = 0; c < d; ++c) dqrow[c] = 0.0;
-                for (int64_t j = 0; j < S; ++j) {
-                    if (w[j] == 0.0) continue;
-                    const uint16_t* krow = k + ((b * S + j) * Hkv + g) * d;
-                    double dx = w[j] * (x[j] - D);
-                    if (softcap > 0.0) {
-                        double xl = 0.0;
-                        for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
-                        const double t = tanh(xl / softcap);
-                        dx *= 1.0 - t * t;
-                    }
-                    for (int64_t c = 0; c < d; ++c) dqrow[c] += query_scale * dx * widen(krow[c]);
-                }
+                row_backward(k, v, dout, b, i, h, T, S, H, Hkv, d, query_scale, softcap, qs, w,
+                             x, dqrow, NULL, NULL);
             }
             /* pass 1b: lse and D of every row of a (b, g) that has a chosen key */
 #pragma omp for schedule(dynamic, 4)
@@ -341,22 +342,14 @@ int g2ref_attn_bwd_sampled(const uint16_t* q, const uint16_t* k, const uint16_t*
                 const int64_t b = r / (T * H);
                 const int64_t i = (r / H) % T;
                 const int64_t h = r % H;
-                const int64_t g = h / group;
-                if (!need[b * Hkv + g]) continue;
+                if (!need[b * Hkv + kv_head(h, H, Hkv)]) continue;
                 double lse;
                 one_row(q, k, v, b, i, h, T, S, H, Hkv, d, q_offset, query_scale, softcap,
                         window, qs, s, w, NULL, &lse);
-                const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
-                double D = 0.0;
-                for (int64_t j = 0; j < S; ++j) {
-                    if (w[j] == 0.0) continue;
-                    const uint16_t* vj = v + ((b * S + j) * Hkv + g) * d;
-                    double dw = 0.0;
-                    for (int64_t c = 0; c < d; ++c) dw += widen(dorow[c]) * widen(vj[c]);
-                    D += w[j] * dw;
-                }
                 row_lse[(b * H + h) * T + i] = lse;
-                row_D[(b * H + h) * T + i] = D;
+                row_D[(b * H + h) * T + i] = row_backward(k, v, dout, b, i, h, T, S, H, Hkv, d,
+                                                          query_scale, softcap, qs, w, x, NULL,
+                                                          NULL, NULL);
             }
             /* pass 2: dk and dv of each chosen key, summed over the rows of
              * both heads of its group that see it */
@@ -371,17 +364,16 @@ int g2ref_attn_bwd_sampled(const uint16_t* q, const uint16_t* k, const uint16_t*
                 for (int64_t h = g * group; h < (g + 1) * group; ++h) {
                     for (int64_t i = 0; i < T; ++i) {
                         if (!visible(i + q_offset, j, window)) continue;
-                        const uint16_t* qrow = q + ((b * T + i) * H + h) * d;
                         const uint16_t* dorow = dout + ((b * T + i) * H + h) * d;
-                        for (int64_t c = 0; c < d; ++c) qs[c] = query_scale * widen(qrow[c]);
+                        scaled_query(q + ((b * T + i) * H + h) * d, d, query_scale, qs);
                         /* x = (query_scale q) . k, the capped logit and its weight */
                         double xl = 0.0;
                         for (int64_t c = 0; c < d; ++c) xl += qs[c] * widen(krow[c]);
                         double sl = xl, cap_grad = 1.0;
                         if (softcap > 0.0) {
-                            const double t = tanh(xl / softcap);
-                            sl = softcap * t;
-                            cap_grad = 1.0 - t * t;
+                            const double th = tanh(xl / softcap);
+                            sl = softcap * th;
+                            cap_grad = 1.0 - th * th;
                         }
                         const double wl = exp(sl - row_lse[(b * H + h) * T + i]);
                         double dw = 0.0;

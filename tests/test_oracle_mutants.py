@@ -23,7 +23,7 @@ MUTANTS = {
     "cap of the raw logit without the inner divide": ("softcap * tanh(x / softcap)", "softcap * tanh(x)"),
     "softmax exponent with the wrong sign": ("exp(s[j] - m)", "exp(m - s[j])"),
     "query scale dropped": ("qs[c] = query_scale * widen(qrow[c]);", "qs[c] = widen(qrow[c]);"),
-    "wrong GQA head mapping": ("const int64_t g = h / group;", "const int64_t g = h % Hkv;"),
+    "wrong GQA head mapping": ("{ return h / (H / Hkv); }", "{ return h % Hkv; }"),
     "lse without the max": ("*lse = m + log(l);", "*lse = log(l);"),
     "values mixed from the mirrored key": ("const uint16_t* vrow = v + ((b * S + j) * Hkv + g) * d;",
                                            "const uint16_t* vrow = v + ((b * S + (S - 1 - j)) * Hkv + g) * d;"),
@@ -44,6 +44,7 @@ MUTANTS = {
     "sampled backward: key terms without the row's D": (
         "const double dx = wl * (dw - row_D[(b * H + h) * T + i]) * cap_grad;",
         "const double dx = wl * dw * cap_grad;"),
+    "sampled backward: cap derivative dropped": ("cap_grad = 1.0 - th * th;", "cap_grad = 1.0;"),
     "sampled backward: weight from the uncapped logit": (
         "const double wl = exp(sl - row_lse", "const double wl = exp(xl - row_lse"),
     "sampled backward: key seen one row late": (
