@@ -35,6 +35,7 @@ G2ATTN_ERR_MISALIGNED = 3
 G2ATTN_ERR_CUDA = 4
 G2ATTN_ERR_DEVICE_TIMEOUT = 5
 G2ATTN_ERR_WORKSPACE = 6
+G2ATTN_ERR_CACHE_LEN = 7
 
 EXPORTS = (
     "g2attn_prefill",

@@ -297,20 +297,53 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};  // context the address belongs to
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (ids are never reused within a process),
+// or 0 when there is no current context or the driver lacks the call.
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 // Device address of g_noalloc_scratch on the current device. The host-side
-// name of the array is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// name of the array is only a stand-in, so the address is looked up with the
+// device current, once per device and context: after cudaDeviceReset the
+// device gets a new context, the library's module is loaded again and the
+// array may sit elsewhere, so a changed context id triggers a new lookup.
 int noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return G2ATTN_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    const unsigned long long ctx = current_ctx_id();
+    if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
             return G2ATTN_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
+        // the lookup makes the device's context current if none was
+        g_noalloc_ctx[dev] = ctx != 0 ? ctx : current_ctx_id();
     }
     *out = g_noalloc_ptr[dev];
     return G2ATTN_OK;
@@ -793,6 +826,7 @@ const char* g2attn_status_string(int status) {
         case G2ATTN_ERR_CUDA: return "CUDA call failed";
         case G2ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case G2ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case G2ATTN_ERR_CACHE_LEN: return "decode sequence longer than max_cache_len";
         default: return "unknown status";
     }
 }
@@ -806,7 +840,7 @@ int g2attn_get_device_error(void) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g2::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
         return G2ATTN_ERR_CUDA;
-    return G2ATTN_ERR_DEVICE_TIMEOUT;
+    return (v & g2::DEVERR_TIMEOUT) ? G2ATTN_ERR_DEVICE_TIMEOUT : G2ATTN_ERR_CACHE_LEN;
 }
 
 int g2attn_selftest_wait_timeout(int timeout_us) {

@@ -14,10 +14,14 @@
 namespace g2 {
 
 // ---------------------------------------------------------------------------
-// Sticky device error word. Bit 0: a bounded wait gave up. The upper 16 bits
-// keep the code of the first wait site that gave up (diagnostics only).
+// Sticky device error word. Bit 0: a bounded wait gave up. Bit 1
+// (DEVERR_CACHE_LEN): a decode sequence needed more splits than the caller's
+// max_cache_len planned for. The upper 16 bits keep the code of the first
+// wait site that gave up (diagnostics only).
 // ---------------------------------------------------------------------------
 __device__ unsigned int g_device_error = 0;
+constexpr unsigned int DEVERR_TIMEOUT = 1u;
+constexpr unsigned int DEVERR_CACHE_LEN = 2u;
 
 enum WaitSite : unsigned int {
     SITE_SELFTEST = 1,

@@ -96,8 +96,12 @@ __device__ __forceinline__ void dec_range(const DecParams& P, const DecLayoutPar
     if (LAYOUT == DEC_RING) lo = max(lo, L - (LP.ring_mask + 1));
     hi = L;
     // more splits than planned only when the caller's max_cache_len undercounts:
-    // drop the excess (wrong result, but never a read past the workspace)
-    nsplit = min((hi - lo + P.chunk - 1) / P.chunk, P.max_splits);
+    // drop the excess (wrong result, but never a read past the workspace) and
+    // report the broken precondition in the sticky device word
+    const int need = (hi - lo + P.chunk - 1) / P.chunk;
+    nsplit = min(need, P.max_splits);
+    if (need > P.max_splits && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        atomicOr(&g_device_error, DEVERR_CACHE_LEN);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {

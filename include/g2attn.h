@@ -54,7 +54,9 @@ typedef enum {
     G2ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
     G2ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
     G2ATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting (see g2attn_get_device_error) */
-    G2ATTN_ERR_WORKSPACE = 6       /* a workspace NULL or smaller than required */
+    G2ATTN_ERR_WORKSPACE = 6,      /* a workspace NULL or smaller than required */
+    G2ATTN_ERR_CACHE_LEN = 7       /* a decode sequence saw more keys than max_cache_len
+                                      planned for (see g2attn_get_device_error) */
 } g2attn_status;
 
 /*
@@ -145,6 +147,10 @@ G2ATTN_API size_t g2attn_decode_workspace_size(int num_seqs, int H, int d, int m
  *   out (num_seqs, H, d) bf16; lse (num_seqs, H) fp32.
  *   workspace: device memory of at least g2attn_decode_workspace_size(...)
  *   bytes, 16-byte aligned, owned by the caller; no initial contents needed.
+ *   A sequence longer than max_cache_len (which the host cannot see) keeps
+ *   only the splits the plan has room for: its output is wrong, nothing
+ *   outside the buffers is touched, and g2attn_get_device_error reports
+ *   G2ATTN_ERR_CACHE_LEN (all decode calls).
  * Source: the Guide's serving notes (local layers only need the last 4,096
  * cached tokens, "Interleaved Local Sliding Window and Global Attention").
  */
@@ -209,7 +215,9 @@ G2ATTN_API int g2attn_decode_paged(const void* q, const void* k_blocks, const vo
  *     24 MiB (25165824 bytes).
  *   - The first call on each device looks up the scratch array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before any stream capture.
+ *     first call before any stream capture. The address is cached per device
+ *     and context: the first call after a cudaDeviceReset looks it up again
+ *     (a reset gives the device a new context, in which the array may move).
  *   - Every call on a device shares the one scratch array and leaves its
  *     contents behind (nothing in it needs clearing: the kernels write every
  *     partial before reading it). Calls that overlap on the GPU -- on
@@ -292,10 +300,15 @@ G2ATTN_API int g2attn_prefill_varlen_backward(const void* q, const void* k, cons
 G2ATTN_API const char* g2attn_status_string(int status);
 
 /*
- * Sticky device-side error word of the current device: nonzero after a
- * kernel gave up on a bounded wait (G2ATTN_ERR_DEVICE_TIMEOUT). Reading it
- * synchronizes the device and clears it. Returns G2ATTN_OK when clear,
- * G2ATTN_ERR_DEVICE_TIMEOUT when set, G2ATTN_ERR_CUDA if it cannot be read.
+ * Sticky device-side error word of the current device. It is set when a
+ * kernel gave up on a bounded wait, and when a decode call (any cache layout)
+ * met a sequence whose visible keys need more splits than its max_cache_len
+ * planned for: that call still returned G2ATTN_OK and stayed inside its
+ * buffers, but dropped the keys past the plan, so its output for that
+ * sequence is wrong. Reading the word synchronizes the device and clears it.
+ * Returns G2ATTN_OK when clear, G2ATTN_ERR_DEVICE_TIMEOUT when a wait gave up
+ * (this takes precedence), G2ATTN_ERR_CACHE_LEN when only the decode
+ * precondition was broken, G2ATTN_ERR_CUDA if the word cannot be read.
  */
 G2ATTN_API int g2attn_get_device_error(void);
 

@@ -11,12 +11,16 @@ TOL_MAX_ABS = 2e-2
 TOL_REL_L2 = 5e-3
 TOL_LSE = 1e-3
 
+# Errors of the comparisons a test asks to have reported (record=True); the
+# test session prints them in its summary (tests/conftest.py).
+RECORDS = []
+
 
 def to_np(t):
     return t.detach().to(torch.float64).cpu().numpy() if isinstance(t, torch.Tensor) else t
 
 
-def check(out, ref_out, lse=None, ref_lse=None, what=""):
+def check(out, ref_out, lse=None, ref_lse=None, what="", record=False):
     o, r = to_np(out), np.asarray(ref_out, dtype=np.float64)
     assert o.shape == r.shape, (what, o.shape, r.shape)
     assert np.all(np.isfinite(o)), f"{what}: non-finite output"
@@ -33,6 +37,9 @@ def check(out, ref_out, lse=None, ref_lse=None, what=""):
         assert np.all(np.isfinite(l)), f"{what}: non-finite lse"
         lse_err = float(np.abs(l - rl).max())
         assert lse_err <= TOL_LSE, f"{msg} lse_err={lse_err:.3e}"
+    if record:
+        RECORDS.append(f"{what}: {o.size} values, max_abs {max_abs:.3e}, rel_l2 {rel:.3e}"
+                       + (f", lse max {lse_err:.3e}" if lse_err is not None else ""))
     return max_abs, rel, lse_err
 
 

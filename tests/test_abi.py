@@ -39,8 +39,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    names = {g2.g2attn_status_string(i) for i in range(7)}
-    assert len(names) == 7
+    names = {g2.g2attn_status_string(i) for i in range(8)}
+    assert len(names) == 8
     assert g2.g2attn_status_string(99) == "unknown status"
 
 

@@ -68,3 +68,21 @@ def test_decode_is_last_row_of_prefill():
     torch.cuda.synchronize()
     check(out[0], po[0, -1].double().cpu().numpy(), lse[0],
           pl[0, :, -1].double().cpu().numpy(), "decode vs prefill last row")
+
+
+def test_cache_longer_than_max_cache_len_is_reported():
+    """max_cache_len plans the splits; a sequence longer than it keeps only the
+    splits the plan has room for. The call still returns OK (the host cannot
+    see the lengths), stays inside its buffers, and the sticky device word
+    reports G2ATTN_ERR_CACHE_LEN once. Sequences within the plan are right."""
+    lengths, cu, q, k, v = decode_inputs(0, 0, 0, 4, 2, 64, seed=48, lengths=[90, 3000])
+    assert g2.g2attn_get_device_error() == g2.G2ATTN_OK
+    out, lse = g2.decode(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), 100, query_scale=0.125)
+    torch.cuda.synchronize()
+    assert g2.g2attn_get_device_error() == g2.G2ATTN_ERR_CACHE_LEN
+    assert g2.g2attn_get_device_error() == g2.G2ATTN_OK  # reading clears it
+    ro, rl = oracle.decode(q, k, v, cu, query_scale=0.125, seqs=[0])
+    check(out[:1], ro, lse[:1], rl, "sequence within the plan")
+    # the same call with an honest max_cache_len leaves the word clear
+    g2.decode(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lengths), query_scale=0.125)
+    assert g2.g2attn_get_device_error() == g2.G2ATTN_OK

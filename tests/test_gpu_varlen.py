@@ -50,7 +50,10 @@ def test_varlen_shapes_full(case):
 @pytest.mark.parametrize("layer", ["local", "global"])
 def test_9b_varlen_sampled(layer):
     """The benchmark's packed workload (16 sequences plus a chunked-prefill
-    tail): every row finite; sampled rows of every sequence against the oracle."""
+    tail): every row finite; sampled rows of every sequence (both ends, the
+    middle, 64- and 128-row tile edges, the window edge, one random row)
+    against the oracle. The whole tensors are compared in
+    tests/test_gpu_contract_full.py."""
     w = WORKLOADS["9b_varlen"]
     window = w.window_local if layer == "local" else 0
     Ts, Ss, cq, ck, q, k, v = varlen_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv, w.d,
@@ -63,7 +66,11 @@ def test_9b_varlen_sampled(layer):
     go, gl, ro_all, rl_all = [], [], [], []
     for s, (t, sl) in enumerate(zip(Ts, Ss)):
         q0, k0 = int(cq[s]), int(ck[s])
-        pos = sorted({0, t - 1, t // 2, min(t - 1, 64), int(rng.integers(0, t))})
+        qo = sl - t
+        pos = {0, t - 1, t // 2, int(rng.integers(0, t)), 63, 64, 65, 127, 128, 129}
+        if window:  # rows whose absolute position sits around the window edge
+            pos |= {window - 2 - qo, window - 1 - qo, window - qo, window + 1 - qo}
+        pos = sorted(p for p in pos if 0 <= p < t)
         rows = [(0, i, h) for i in pos for h in range(w.H)]
         ro, rl = oracle.attn_rows(q[q0:q0 + t][None], k[k0:k0 + sl][None], v[k0:k0 + sl][None],
                                   rows, q_offset=sl - t, query_scale=w.query_scale,

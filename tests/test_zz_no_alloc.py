@@ -4,8 +4,10 @@ front, a plug-in handed only input and output pointers, code that must avoid
 cudaMalloc's implicit device synchronisation). It keeps its split-KV partials
 in the library's static 24 MiB scratch instead of a caller workspace.
 
-Checked through the C ABI against g2attn_decode on two calls in a row (the
-second call reuses the scratch the first one left behind). This file is named
+Checked through the C ABI on two calls in a row (the second call reuses the
+scratch the first one left behind): bit for bit against g2attn_decode, which
+runs the same kernels with the same split plan on a caller workspace, and
+against the fp64 oracle within the library's tolerance. This file is named
 so pytest collects it last, and it passes alone in a fresh process too.
 """
 import ctypes
@@ -14,6 +16,7 @@ import pytest
 import torch
 
 import global_soft_capped_b200 as g2
+import oracle
 from global_soft_capped_b200.inputs import WORKLOADS, decode_inputs
 from parity import check
 
@@ -28,9 +31,9 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     w = WORKLOADS["27b_decode"]
-    lengths, cu, q, k, v = decode_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv, w.d, w.std,
-                                         w.seed)
-    q, k, v, cu = q.cuda(), k.cuda(), v.cuda(), cu.cuda()
+    lengths, cu, q_h, k_h, v_h = decode_inputs(w.num_seqs, w.len_lo, w.len_hi, w.H, w.Hkv, w.d,
+                                               w.std, w.seed)
+    q, k, v, cu = q_h.cuda(), k_h.cuda(), v_h.cuda(), cu.cuda()
     n, H, d = q.shape
     L = max(lengths)
     assert g2.g2attn_decode_workspace_size(n, H, d, L) <= 24 << 20
@@ -50,8 +53,11 @@ def test_noalloc_decode_matches_workspace_decode_twice():
                                       window, stream)
         assert st == g2.G2ATTN_OK, f"call {call}: {g2.g2attn_status_string(st)}"
         torch.cuda.synchronize()
-        check(out, ref_out.double().cpu().numpy(), lse, ref_lse.double().cpu().numpy(),
-              f"noalloc call {call}")
+        assert torch.equal(out, ref_out), f"call {call}: out differs from g2attn_decode"
+        assert torch.equal(lse, ref_lse), f"call {call}: lse differs from g2attn_decode"
+        ro, rl = oracle.decode(q_h, k_h, v_h, cu.cpu(), query_scale=w.query_scale,
+                               softcap=w.softcap, window=window)
+        check(out, ro, lse, rl, f"noalloc call {call} against the oracle")
     assert g2.g2attn_get_device_error() == g2.G2ATTN_OK
 
 
