@@ -1,32 +1,37 @@
 #!/usr/bin/env python
 """Benchmark of libg2attn on B200: useful attention TFLOP/s (prefill) and KV GB/s (decode).
 
-One step = one pass of the prefill hot path over the 2B-shaped layer pair
-(B=1, T=S=8192, H=8, Hkv=4, d=256, query_scale 1/16, softcap 50): the local
-layer (window 4096) and the global layer, both through the C ABI. Useful FLOPs
-count 4*d per visible (query, key, head) triple only. Inputs live in HBM; the
-L2 is flushed (a 512 MiB write) between timed steps, outside the timed events.
+One step = one pass of the prefill hot path over the 9B-shaped batched layer
+pair (B=2, T=S=8192, H=16, Hkv=8, d=256, query_scale 1/16, softcap 50), the
+largest single-GPU workload: the local layer (window 4096) and the global
+layer, both through the C ABI. Useful FLOPs count 4*d per visible (query,
+key, head) triple only. Inputs live in HBM; the L2 is flushed (a 512 MiB
+write) between timed steps, outside the timed events.
 
 Printed (rank 0, one JSON line): the contract keys, plus
   roofline      dominant kernel (prefill_fwd_sm100<256,2>, the CTA-pair kernel
                 that d = 256 runs on) vs measured bf16 peak
-  cpu_baseline  the fp64 oracle on the host cores on a bounded row sample
+  cpu_baseline  the fp64 oracle on the host cores: a bounded row sample of the
+                step's workload, one thread on the tiny pair, the 27B decode
+                (KV GB/s, tokens/s), the host's CPU model and core counts
   e2e           the same metric with pinned-host inputs and outputs copied
                 inside the timed region
   clocks        nvidia-smi samples taken during the timed region
   layers        per-layer times of the step
-  extra         9B pair (local/global separately), 27B decode (KV GB/s,
-                tokens/s), the 9B ragged varlen prefill, the Gemma 3-shaped
-                variant of the 2B pair (window 1024, no cap) and the gradients
-                of the 27B-shaped pair (dense and as a packed batch of 8
-                sequences) and of the 2B-shaped pair at d = 256 (useful
-                backward TFLOP/s)
+  extra         2B pair, 27B decode (KV GB/s, tokens/s; linear, ring and paged
+                caches), the 9B ragged varlen prefill (packed and paged K/V),
+                the Gemma 3-shaped variant of the 2B pair (window 1024, no cap)
+                and the gradients of the 27B-shaped pair (dense and as a packed
+                batch of 8 sequences) and of the 2B-shaped pair at d = 256
+                (useful backward TFLOP/s)
 
 `--impl reference` times the fp64 oracle (the reference arm of this build)
 on the host cores on bounded samples of the same workload.
 Multi-GPU (torchrun): every rank runs its own replica (the units are
 independent; there is no data-path collective); value = total useful FLOPs
-of all ranks / max-over-ranks device time ("scaling": "weak").
+of all ranks / max-over-ranks device time ("scaling": "weak"). `--gpus N`
+must equal the launcher's WORLD_SIZE (1 without torchrun); otherwise the run
+stops with an error instead of printing a line for another N.
 """
 from __future__ import annotations
 
@@ -50,7 +55,7 @@ from global_soft_capped_b200.inputs import (  # noqa: E402
     varlen_inputs)
 
 METRIC = "useful attention TFLOP/s (prefill) and KV GB/s (decode) vs B200 roofline"
-WORKLOAD = "2b"
+WORKLOAD = "9b"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -82,6 +87,22 @@ def varlen_flops(Ts, Ss, H, d, window):
 def decode_kv_bytes(lengths, Hkv, d, window):
     rows = sum(min(L, window) if window > 0 else L for L in lengths)
     return rows * Hkv * d * 2 * 2  # K and V, bf16
+
+
+def headline_config(world):
+    """The `config` object of the bench line (identical in both arms)."""
+    w = WORKLOADS[WORKLOAD]
+    return {"workload": f"{WORKLOAD}_prefill_pair", "B": w.B, "T": w.T, "S": w.S, "H": w.H,
+            "Hkv": w.Hkv, "d": w.d, "window_local": w.window_local,
+            "query_scale": w.query_scale, "softcap": w.softcap,
+            "global_batch": w.B * world, "seq_len": w.T,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs (256 MiB) larger than L2; also flushed between steps by a 512 MiB "
+                  "write outside the timed events"}
+
+
+def step_flops_of(w):
+    return sum(prefill_flops(w.B, w.T, w.S, w.H, w.d, 0, win) for win in (w.window_local, 0))
 
 
 def peaks():
@@ -243,25 +264,22 @@ def run_ours(args, rank, world, dev):
     pk, pk_kind = peaks()
     avg_loc, avg_glo = sum(loc) / nsteps, sum(glo) / nsteps
     ach = (flops["local"] + flops["global"]) / ((avg_loc + avg_glo) * 1e-3) / 1e12
+    compulsory = 2 * (q.numel() + k.numel() + v.numel() + q.numel())
     roof = {"kernel": f"prefill_fwd_sm100<256,{KERNEL_CG}>", "bound": "tensor", "achieved": round(ach, 2),
             "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
             "peak_kind": f"{pk_kind} bf16 dense (burst; kernel timed alone)",
-            "traffic": ncu_traffic(f"prefill_fwd_sm100<256,{KERNEL_CG}>/2b_pair", 1.0),
+            "traffic": ncu_traffic(f"prefill_fwd_sm100<256,{KERNEL_CG}>/{WORKLOAD}_pair", 1.0),
             "traffic_unit": "bytes per launch (mean of the local and global launch)",
-            "algorithmic": "4*d*H*B per visible (query,key) pair; 0.4811 TFLOP per step "
-                           "(two launches); compulsory bytes Q+K+V+O = 100663296 per launch"}
+            "algorithmic": f"4*d*H*B per visible (query,key) pair; {step_flops / 1e12:.4f} TFLOP "
+                           f"per step (two launches); compulsory bytes Q+K+V+O = {compulsory} "
+                           f"per launch"}
 
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": nsteps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded iid N(0,1) bf16)",
-        "config": {"workload": "2b_prefill_pair", "B": w.B, "T": w.T, "S": w.S, "H": w.H,
-                   "Hkv": w.Hkv, "d": w.d, "window_local": w.window_local,
-                   "query_scale": w.query_scale, "softcap": w.softcap,
-                   "global_batch": w.B * world, "seq_len": w.T,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between steps by a 512 MiB write outside the timed events"},
+        "config": headline_config(world),
         "gpu_launches": 2 * nsteps,
         "wall_s_timed_region": round(t_wall, 3),
         "roofline": roof,
@@ -365,8 +383,8 @@ def time_launches(fn, flush, stream, reps=10, warm=3):
 def extra_workloads(g2, dev, stream, flush):
     pk, _ = peaks()
     res = {}
-    # 9B batched pair, local and global reported separately
-    w = WORKLOADS["9b"]
+    # 2B pair, local and global reported separately
+    w = WORKLOADS["2b"]
     q, k, v = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed))
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
@@ -378,7 +396,7 @@ def extra_workloads(g2, dev, stream, flush):
                                                      lse=lse, stream=stream), flush, stream)
         r9[lay] = {"ms": round(med, 4), "tflops": round(f / (med * 1e-3) / 1e12, 2),
                    "frac_bf16_peak": round(f / (med * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}
-    res["9b_prefill"] = r9
+    res["2b_prefill"] = r9
     del q, k, v, out, lse
 
     # Gemma 3-shaped variant of the 2B pair: window 1024, no soft-cap
@@ -569,61 +587,133 @@ def extra_workloads(g2, dev, stream, flush):
 # ---------------------------------------------------------------------------
 # CPU baseline / reference arm: the fp64 oracle on the host cores
 # ---------------------------------------------------------------------------
-def oracle_sample_rate(target_s=20.0, seed=0):
-    """Useful TFLOP/s of the oracle on a bounded sample of the 2B pair: query
-    rows spread over positions and heads of both layers; useful FLOPs of a
-    row = 4*d*(visible keys of that row)."""
+def host_info():
+    """CPU model and core counts of the host the oracle runs on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "os_cpu_count": os.cpu_count(),
+            "affinity_cpus": len(os.sched_getaffinity(0))}
+
+
+def _oracle_rows(oracle, q, k, v, w, nrows, rng):
+    """The oracle on nrows query rows of each layer of workload w, spread
+    uniformly over batch, positions and heads. Returns (seconds, useful FLOPs);
+    the useful FLOPs of a row are 4*d*(visible keys of that row)."""
+    t0 = time.perf_counter()
+    useful = 0.0
+    for win in (w.window_local, 0):
+        b = rng.integers(0, w.B, nrows)
+        pos = rng.integers(0, w.T, nrows)
+        heads = rng.integers(0, w.H, nrows)
+        rows = np.stack([b, pos, heads], 1).astype(np.int64)
+        oracle.attn_rows(q, k, v, rows, query_scale=w.query_scale, softcap=w.softcap, window=win)
+        vis = np.minimum(pos + 1, win) if win else pos + 1
+        useful += float(np.sum(4.0 * w.d * vis))
+    return time.perf_counter() - t0, useful
+
+
+def _oracle_calibrate(oracle, q, k, v, w, target_s, rng):
+    """Rows per layer for one sample of about target_s seconds."""
+    threads = oracle.max_threads()
+    n = max(threads, 8)
+    dt, _ = _oracle_rows(oracle, q, k, v, w, n, rng)
+    return int(max(threads, min(200000, n * target_s / max(dt, 1e-3))))
+
+
+def cpu_baseline(target_s=15.0):
+    """The fp64 oracle, as it stands, on the host cores (all the process may
+    use): a bounded row sample of the step's workload (its value), one thread
+    on the whole tiny pair, and the whole 27B decode in the GPU's units."""
     import oracle
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    threads = oracle.max_threads()
     w = WORKLOADS[WORKLOAD]
     q, k, v = prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed)
-    rng = np.random.default_rng(seed)
-    threads = oracle.max_threads()
+    rng = np.random.default_rng(0)
+    n = _oracle_calibrate(oracle, q, k, v, w, target_s, rng)
+    dt, useful = _oracle_rows(oracle, q, k, v, w, n, rng)
+    res = {"kind": "oracle", "cores": threads, "value": useful / dt / 1e12, "unit": "TFLOP/s",
+           "sample": f"{2 * n} query rows (half local, half global) of the {WORKLOAD} pair, "
+                     f"uniform batch, positions and heads",
+           "seconds": round(dt, 2), "host": host_info()}
 
-    def run(nrows):
+    # one thread, the whole tiny pair (B=1, T=S=256, H=4, Hkv=2, d=64)
+    wt = WORKLOADS["tiny"]
+    qt, kt, vt = prefill_inputs(wt.B, wt.T, wt.S, wt.H, wt.Hkv, wt.d, wt.std, wt.seed)
+    oracle.set_threads(1)
+    tiny = {"threads": oracle.max_threads()}
+    tiny_useful = tiny_s = 0.0
+    for lay, win in (("local", wt.window_local), ("global", 0)):
         t0 = time.perf_counter()
-        useful = 0.0
-        for win in (w.window_local, 0):
-            pos = rng.integers(0, w.T, nrows)
-            heads = rng.integers(0, w.H, nrows)
-            rows = np.stack([np.zeros(nrows, np.int64), pos, heads], 1)
-            oracle.attn_rows(q, k, v, rows, query_scale=w.query_scale, softcap=w.softcap,
-                             window=win)
-            vis = np.minimum(pos + 1, win) if win else pos + 1
-            useful += float(np.sum(4.0 * w.d * vis))
-        return time.perf_counter() - t0, useful
+        oracle.attn(qt, kt, vt, query_scale=wt.query_scale, softcap=wt.softcap, window=win)
+        tiny[f"{lay}_s"] = round(time.perf_counter() - t0, 4)
+        tiny_s += tiny[f"{lay}_s"]
+        tiny_useful += prefill_flops(wt.B, wt.T, wt.S, wt.H, wt.d, 0, win)
+    tiny["gflops_per_s"] = round(tiny_useful / max(tiny_s, 1e-9) / 1e9, 3)
+    oracle.set_threads(threads)
+    res["tiny_pair_1_thread"] = tiny
 
-    n = max(threads, 8)
-    dt, _ = run(n)
-    n = int(max(threads, min(200000, n * target_s / max(dt, 1e-3))))
-    dt, useful = run(n)
-    return useful / dt / 1e12, {"kind": "oracle", "cores": threads,
-                                "sample": f"{2 * n} query rows (half local, half global) of the "
-                                          f"2B pair, uniform positions and heads",
-                                "seconds": round(dt, 2)}
+    # the whole 27B decode (64 sequences), all threads, per layer
+    wd = WORKLOADS["27b_decode"]
+    lengths, cu, qd, kc, vc = decode_inputs(wd.num_seqs, wd.len_lo, wd.len_hi, wd.H, wd.Hkv,
+                                            wd.d, wd.std, wd.seed)
+    dec = {"sequences": len(lengths)}
+    for lay, win in (("local", wd.window_local), ("global", 0)):
+        t0 = time.perf_counter()
+        oracle.decode(qd, kc, vc, cu, query_scale=wd.query_scale, softcap=wd.softcap, window=win)
+        t = time.perf_counter() - t0
+        nbytes = decode_kv_bytes(lengths, wd.Hkv, wd.d, win)
+        dec[lay] = {"s": round(t, 3), "kv_GBps": round(nbytes / t / 1e9, 3),
+                    "tokens_per_s": round(len(lengths) / t, 2)}
+    res["27b_decode"] = dec
+    return res
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on the host cores, each step a
+    bounded row sample of the step's workload (the same sample size every
+    step), sized so that warm-up and timed steps end within a few minutes."""
     if rank != 0:
         return None
-    rates = []
-    info = None
-    for i in range(args.warmup + args.steps):
-        rate, info = oracle_sample_rate(target_s=max(2.0, 60.0 / (args.warmup + args.steps)),
-                                        seed=i)
-        if i >= args.warmup:
-            rates.append(rate)
-    value = statistics.median(rates)
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    threads = oracle.max_threads()
     w = WORKLOADS[WORKLOAD]
-    useful_step = sum(prefill_flops(w.B, w.T, w.S, w.H, w.d, 0, win) for win in (w.window_local, 0))
-    info = dict(info, value=value, unit="TFLOP/s")
+    q, k, v = prefill_inputs(w.B, w.T, w.S, w.H, w.Hkv, w.d, w.std, w.seed)
+    rng = np.random.default_rng(0)
+    total = args.warmup + args.steps
+    per_step_s = min(10.0, max(0.05, 150.0 / max(total, 1)))
+    n = _oracle_calibrate(oracle, q, k, v, w, per_step_s, rng)
+    times, useful = [], 0.0
+    for i in range(total):
+        dt, u = _oracle_rows(oracle, q, k, v, w, n, rng)
+        if i >= args.warmup:
+            times.append(dt)
+            useful += u
+    value = useful / sum(times) / 1e12
+    ms_per_step = 1e3 * sum(times) / len(times)
+    sample = (f"{2 * n} query rows per step (half local, half global) of the {WORKLOAD} pair, "
+              f"uniform batch, positions and heads")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": useful_step / (value * 1e12) * 1e3, "higher_is_better": True,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded iid N(0,1) bf16)",
-            "config": {"workload": "2b_prefill_pair", "B": w.B, "T": w.T, "S": w.S, "H": w.H,
-                       "Hkv": w.Hkv, "d": w.d, "window_local": w.window_local},
-            "cpu_baseline": info,
+            "config": headline_config(world),
+            "step": "one bounded sample of the workload (ms_per_step is the sample's time); "
+                    "the whole two-layer step would take projected_ms_per_full_step",
+            "projected_ms_per_full_step": step_flops_of(w) / (value * 1e12) * 1e3,
+            "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": sample,
+                             "value": value, "unit": "TFLOP/s", "host": host_info()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -709,6 +799,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        # one rank per GPU: N GPUs need N ranks (torchrun --nproc-per-node N)
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE is {world}; launch "
+                         f"{args.gpus} ranks with torchrun --nproc-per-node {args.gpus}\n")
+        sys.exit(2)
 
     if args.impl == "reference":
         if world > 1 and rank != 0:
@@ -726,8 +821,7 @@ def main():
     # the oracle's thread pool is created before any GPU work (never forked after it)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, info = oracle_sample_rate()
-        cpu = dict(info, value=rate, unit="TFLOP/s")
+        cpu = cpu_baseline()
     res = run_ours(args, rank, world, dev)
     if rank == 0:
         if cpu is not None:

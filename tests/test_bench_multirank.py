@@ -72,3 +72,19 @@ def test_reference_arm_prints_on_rank_zero_only():
                          capture_output=True, text=True, timeout=300)
     assert res.returncode == 0, res.stderr[-2000:]
     assert res.stdout.strip() == ""
+
+
+def test_gpus_must_match_the_world_size():
+    """--gpus N without N ranks (or N ranks with another --gpus) stops with an
+    error before any work, instead of printing a line for the wrong N."""
+    for gpus, env_world in ((2, None), (1, "2")):
+        env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+        env.pop("WORLD_SIZE", None)
+        if env_world:
+            env.update(RANK="0", LOCAL_RANK="0", WORLD_SIZE=env_world)
+        res = subprocess.run([sys.executable, "bench.py", "--gpus", str(gpus), "--steps", "1",
+                              "--warmup", "3"], cwd=ROOT, env=env, capture_output=True,
+                             text=True, timeout=300)
+        assert res.returncode != 0, (gpus, env_world)
+        assert res.stdout.strip() == ""
+        assert "WORLD_SIZE" in res.stderr
