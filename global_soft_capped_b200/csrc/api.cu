@@ -501,6 +501,9 @@ int g2attn_prefill_varlen_backward(const void* q, const void* k, const void* v, 
     P.dq = static_cast<__nv_bfloat16*>(dq);
     P.dk = static_cast<__nv_bfloat16*>(dk);
     P.dv = static_cast<__nv_bfloat16*>(dv);
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.k = static_cast<const __nv_bfloat16*>(k);
+    P.v = static_cast<const __nv_bfloat16*>(v);
     P.B = 1;
     P.T = max_T;
     P.S = max_S;
@@ -566,6 +569,9 @@ int g2attn_prefill_backward(const void* q, const void* k, const void* v, const v
     P.dq = static_cast<__nv_bfloat16*>(dq);
     P.dk = static_cast<__nv_bfloat16*>(dk);
     P.dv = static_cast<__nv_bfloat16*>(dv);
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.k = static_cast<const __nv_bfloat16*>(k);
+    P.v = static_cast<const __nv_bfloat16*>(v);
     P.B = B;
     P.T = T;
     P.S = S;

@@ -24,10 +24,14 @@
 //   bwd_sm100<D, BW_Q>   one unit = 64 query positions x 2 heads: q and dout
 //                 stay, the CK-key tiles stream; X = q K^T, Y = dout V^T,
 //                 dq += dS K.
-// Column tiles are 128 rows for d <= 128 and 32 rows at d = 256 (BwCfg).
-// TMEM (512 columns): accumulators at 0..255, X at 256, Y at 384. The dk/dv
-// kernel needs 2 d accumulator columns, so at d = 256 each key tile is two
-// units, one per half of the d columns (X and Y are computed in both).
+// Column tiles are 128 rows for d <= 128 and 64 rows at d = 256 (BwCfg).
+// TMEM (512 columns), d <= 128: accumulators at 0..255, X at 256, Y at 384.
+// d = 256: one 256-column accumulator at 0, one resident operand held in TMEM
+// at 256..383 (read by the UMMAs as their A operand, so its bytes never cross
+// shared memory again), X at 384 and Y at 448. The dk/dv kernel then runs
+// each key tile as two units, a dv unit (X only: K in TMEM; dv += P^T dout)
+// and a dk unit (X with K in shared memory, Y with V in TMEM; dk += dS^T q);
+// the dq kernel keeps q in TMEM and dout in shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -56,20 +60,29 @@ constexpr uint32_t BW_TMEM_COLS = 512;
 template <int D>
 struct BwCfg {
     static_assert(D == 64 || D == 128 || D == 256, "backward kernels: d = 64, 128, 256");
-    static constexpr int CQ = D == 256 ? 16 : BW_QPOS;  // KV column tile: positions per head
-    static constexpr int CK = D == 256 ? 32 : BW_KEYS;  // Q column tile: keys
+    // d = 256: one resident operand in TMEM instead of shared memory (see the
+    // file header), which leaves room for 64-row column tiles
+    static constexpr bool A_TMEM = D == 256;
+    static constexpr int CQ = D == 256 ? 32 : BW_QPOS;  // KV column tile: positions per head
+    static constexpr int CK = D == 256 ? 64 : BW_KEYS;  // Q column tile: keys
     static constexpr int CR = 2 * CQ;                    // column tile rows (both modes)
     static_assert(CR == CK, "column tiles of both modes have CR rows");
     static constexpr int HW = CR / 2;                    // columns per half (per warp part)
     static constexpr int CHUNK = HW < 32 ? HW : 32;      // columns per TMEM round trip
-    static constexpr int DSPLIT_KV = D == 256 ? 2 : 1;   // dk/dv kernel: d-halves per key tile
+    static constexpr int DSPLIT_KV = D == 256 ? 2 : 1;   // dk/dv kernel: units per key tile
+    static constexpr int RES_TILES = A_TMEM ? 1 : 2;     // resident tiles in shared memory
     static constexpr int TILE_BYTES = 128 * D * 2;       // one 128-row resident tile
     static constexpr int CTILE_BYTES = CR * D * 2;       // one streamed column tile
     static constexpr int VEC_BYTES = 1024;               // -lse2, -D of the tile's query rows
     static constexpr int VEC_TX = 2 * CR * 4;            //   (bytes copied: CR rows, two arrays)
     static constexpr int SLOT_BYTES = 2 * CTILE_BYTES + VEC_BYTES;
     static_assert(SLOT_BYTES % 1024 == 0 && VEC_TX <= VEC_BYTES, "slot layout");
-    static constexpr int SMEM_TILES = 2 * TILE_BYTES + 2 * SLOT_BYTES;  // R1, R2, 2 column slots
+    static constexpr int SMEM_TILES = RES_TILES * TILE_BYTES + 2 * SLOT_BYTES;  // R1 (R2), 2 slots
+    // TMEM columns: accumulators at 0, the resident A operand (d = 256), X, Y
+    static constexpr uint32_t A_COL = 256;
+    static constexpr uint32_t X_COL = A_TMEM ? 384 : BW_X_COL;
+    static constexpr uint32_t Y_COL = A_TMEM ? 448 : BW_Y_COL;
+    static_assert(!A_TMEM || (X_COL + CR <= Y_COL && Y_COL + CR <= BW_TMEM_COLS), "TMEM columns");
     static constexpr int MAX_SEQ_TABLE = 1024;                  // varlen: sequences per launch
     // varlen: per-sequence work, sequences ranked by it, unit prefix in rank order
     static constexpr int VL_BYTES = 4 * (3 * MAX_SEQ_TABLE + 1);
@@ -81,6 +94,11 @@ struct BwParams {
     __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
+    // inputs, read directly by the elementwise warps when a resident tile
+    // goes to TMEM (d = 256)
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
     // -lse * log2(e) and -D = -(dout . out) per (head, query position), with
     // each sequence's positions padded to whole 64-position tiles (-inf / 0):
     // dense (B, H, Tp); varlen (H, Wmax), sequence s at columns wq[s] ..
@@ -123,7 +141,7 @@ struct BwMask {
 
 struct BwUnit {
     int g;
-    int dh;           // d-half of the dk/dv columns (d = 256); 0 otherwise
+    int dh;           // dk/dv kernel at d = 256: 0 = dv unit, 1 = dk unit; 0 otherwise
     int T, S, qoff;   // the sequence: queries, keys, position of query 0
     int qbase, kbase; // packed row of its first query / key
     long long wbase;  // workspace column of its position 0 for head 0 ...
@@ -433,14 +451,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
               const BwParams P) {
     using C = BwCfg<D>;
     constexpr bool KV = MODE == BW_KV;
-    constexpr int DS = KV ? C::DSPLIT_KV : 1;  // units per row tile (d-halves)
-    constexpr int ACC_N = D / DS;             // accumulator columns per product
+    constexpr int DS = KV ? C::DSPLIT_KV : 1;  // units per row tile
+    constexpr bool AT = C::A_TMEM;
+    constexpr int ACC_N = D;                   // accumulator columns per product
+    constexpr uint32_t X_COL = C::X_COL, Y_COL = C::Y_COL, A_COL = C::A_COL;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t* sR1 = base;                    // KV: K tile;  Q: q tile
-    uint8_t* sR2 = base + C::TILE_BYTES;    // KV: V tile;  Q: dout tile
-    uint8_t* sSlot = base + 2 * C::TILE_BYTES;  // [2] x (C1 tile, C2 tile, lse2[CR], D[CR])
+    // d <= 128: R1 = K (KV) or q (Q), R2 = V or dout. d = 256: R1 = K (KV, dk
+    // units) or dout (Q); the other operand is in TMEM.
+    uint8_t* sR1 = base;
+    uint8_t* sR2 = base + C::TILE_BYTES;
+    uint8_t* sSlot = base + C::RES_TILES * C::TILE_BYTES;  // [2] x (C1, C2, lse2[CR], D[CR])
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::SMEM_TILES);
     uint64_t* r_full = bars + 0;
     uint64_t* r_empty = bars + 1;
@@ -453,7 +475,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* acc_done = bars + 10; // last accumulation of the unit completed
     uint64_t* acc_free = bars + 11; // epilogue read the accumulators (8 warp arrivals)
     uint64_t* drain = bars + 12;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
+    uint64_t* ra_full = bars + 13;  // d = 256: the unit's TMEM-resident operand written (8 warps)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     // varlen tables: cum[num_seqs + 1] (unit prefix in rank order), order[], work[]
     int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
@@ -476,6 +499,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         mbar_init(acc_done, 1);
         mbar_init(acc_free, BW_EW_THREADS / 32);
         mbar_init(drain, 1);
+        mbar_init(ra_full, BW_EW_THREADS / 32);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -568,13 +592,27 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     ok = mbar_wait(r_empty, (uw - 1) & 1, abort_flag, lim, SITE_BW_PROD);
                     if (!ok) break;
                 }
-                mbar_arrive_expect_tx(r_full, 2 * C::TILE_BYTES);
-                if (KV) {
-                    bw_load_tile<D>(sR1, &tmK, r_full, U.kbase + U.row0, U.g);
-                    bw_load_tile<D>(sR2, &tmV, r_full, U.kbase + U.row0, U.g);
+                if constexpr (AT) {
+                    // one resident tile in shared memory: K for a dk unit,
+                    // dout for the dq kernel; a dv unit has none
+                    if (KV && U.dh == 0) {
+                        mbar_arrive(r_full);
+                    } else {
+                        mbar_arrive_expect_tx(r_full, C::TILE_BYTES);
+                        if (KV)
+                            bw_load_tile<D>(sR1, &tmK, r_full, U.kbase + U.row0, U.g);
+                        else
+                            bw_load_tile<D>(sR1, &tmO, r_full, U.qbase + U.row0, 2 * U.g);
+                    }
                 } else {
-                    bw_load_tile<D>(sR1, &tmQ, r_full, U.qbase + U.row0, 2 * U.g);
-                    bw_load_tile<D>(sR2, &tmO, r_full, U.qbase + U.row0, 2 * U.g);
+                    mbar_arrive_expect_tx(r_full, 2 * C::TILE_BYTES);
+                    if (KV) {
+                        bw_load_tile<D>(sR1, &tmK, r_full, U.kbase + U.row0, U.g);
+                        bw_load_tile<D>(sR2, &tmV, r_full, U.kbase + U.row0, U.g);
+                    } else {
+                        bw_load_tile<D>(sR1, &tmQ, r_full, U.qbase + U.row0, 2 * U.g);
+                        bw_load_tile<D>(sR2, &tmO, r_full, U.qbase + U.row0, 2 * U.g);
+                    }
                 }
                 for (int c = 0; c < U.ncols; ++c) {
                     const int sl = ct & 1;
@@ -650,17 +688,43 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             };
             // X, Y columns [HW h, HW h + HW) of the tile in slot sl: rows HW h..
             // of the column tiles (N = HW), contraction over d
-            auto issue_xy = [&](int sl, int h) {
+            auto issue_xy = [&](int sl, int h, int kind) {
                 const uint32_t c1 = slot_lo + sl * SLOT_STEP + h * HALF_ROWS;
                 const uint32_t c2 = c1 + CTILE_STEP;
+                if constexpr (AT) {
+                    // d = 256, A operands: KV dv unit X: K in TMEM; KV dk unit
+                    // X: K in R1, Y: V in TMEM; Q: X: q in TMEM, Y: dout in R1
+                    const bool x_tmem = !KV || kind == 0;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + BW_X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
-                               IDESC_XY, kk != 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        if (x_tmem)
+                            umma_ts_lh(tmem + X_COL + HW * h, tmem + A_COL + 8 * kk,
+                                       c1 + kstep_c(kk), HI, IDESC_XY, kk != 0);
+                        else
+                            umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk),
+                                       HI, IDESC_XY, kk != 0);
+                    }
+                    if (!KV || kind == 1) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + BW_Y_COL + HW * h, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
-                               IDESC_XY, kk != 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            if (KV)
+                                umma_ts_lh(tmem + Y_COL + HW * h, tmem + A_COL + 8 * kk,
+                                           c2 + kstep_c(kk), HI, IDESC_XY, kk != 0);
+                            else
+                                umma_ss_lh(tmem + Y_COL + HW * h, r1_lo + kstep(kk),
+                                           c2 + kstep_c(kk), HI, IDESC_XY, kk != 0);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                                   IDESC_XY, kk != 0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss_lh(tmem + Y_COL + HW * h, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                                   IDESC_XY, kk != 0);
+                }
                 umma_commit(&xy_full[h]);
             };
             // Both halves of the tile in slot sl as one UMMA pair (N = CR): with
@@ -673,21 +737,22 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const uint32_t c2 = c1 + CTILE_STEP;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + BW_X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                    umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
                                IDESC_XYT, kk != 0);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + BW_Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                    umma_ss_lh(tmem + Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
                                IDESC_XYT, kk != 0);
                 umma_commit(&xy_full[0]);
                 umma_commit(&xy_full[1]);
             };
             constexpr bool TILE_XY = HW < 32;
+            static_assert(!(TILE_XY && AT), "whole-tile X / Y only with both resident tiles in shared memory");
             // accumulations over the half's HW rows (K indices HW h ..): A = the
             // bf16 operand the half's warps wrote at columns HW h + 8 k4; B =
-            // the streamed tiles' columns of d-half dh (ACC_N columns)
-            auto issue_acc = [&](int sl, int h, int dh, bool first) {
-                const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP + dh * (ACC_N / 64) * CBLOCK;
+            // the streamed tile read MN-major (all D columns)
+            auto issue_acc = [&](int sl, int h, int kind, bool first) {
+                const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
                 const uint32_t c2_mn = c1_mn + CTILE_STEP;
                 constexpr int KS = HW / 16;  // K steps per half
 #pragma unroll
@@ -697,14 +762,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     const uint32_t bstep = kk * ((16 * 128) >> 4);
                     const uint32_t zc = HW * h + 8 * k4;
                     if (KV) {
-                        // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y)
-                        umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c2_mn + bstep, HI, IDESC_ACC,
-                                   acc);
-                        umma_ts_lh(tmem + ACC_N, tmem + BW_Y_COL + zc, c1_mn + bstep, HI,
-                                   IDESC_ACC, acc);
+                        // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y); at
+                        // d = 256 the dv unit does the first, the dk unit the second
+                        if (!AT || kind == 0)
+                            umma_ts_lh(tmem + 0, tmem + X_COL + zc, c2_mn + bstep, HI, IDESC_ACC,
+                                       acc);
+                        if (!AT || kind == 1)
+                            umma_ts_lh(tmem + (AT ? 0 : ACC_N), tmem + Y_COL + zc, c1_mn + bstep,
+                                       HI, IDESC_ACC, acc);
                     } else {
                         // dq += dS K (dS at X)
-                        umma_ts_lh(tmem + 0, tmem + BW_X_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
+                        umma_ts_lh(tmem + 0, tmem + X_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
                                    acc);
                     }
                 }
@@ -722,6 +790,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (U.ncols == 0) continue;
                 ok = mbar_wait(r_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
+                if constexpr (AT) {  // the elementwise warps wrote the TMEM-resident operand
+                    ok = mbar_wait(ra_full, uw & 1, abort_flag, lim, SITE_BW_MMA);
+                    if (!ok) break;
+                }
                 tc_fence_after();
                 ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
@@ -729,8 +801,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if constexpr (TILE_XY) {
                     issue_xy_tile(ct & 1);
                 } else {
-                    issue_xy(ct & 1, 0);
-                    issue_xy(ct & 1, 1);
+                    issue_xy(ct & 1, 0, U.dh);
+                    issue_xy(ct & 1, 1, U.dh);
                 }
                 for (int c = 0; c < U.ncols; ++c) {
                     const int sl = ct & 1;
@@ -748,7 +820,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                        SITE_BW_MMA);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_xy(sl ^ 1, 0);
+                        issue_xy(sl ^ 1, 0, U.dh);
                     }
                     ok = mbar_wait(&z_full[1], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
                     if (!ok) break;
@@ -763,7 +835,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             tc_fence_after();
                             issue_xy_tile(sl ^ 1);
                         } else {
-                            issue_xy(sl ^ 1, 1);
+                            issue_xy(sl ^ 1, 1, U.dh);
                         }
                     }
                     ++ct;
@@ -803,11 +875,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 // query sees at least its own key)
                 if (KV && r < U.rvalid) {
                     const size_t row = (static_cast<size_t>(U.kbase) + U.row0 + r) * P.Hkv + U.g;
-                    const size_t c0 = row * D + U.dh * ACC_N + part * (ACC_N / 2);
+                    const size_t c0 = row * D + part * (D / 2);
 #pragma unroll
-                    for (int c = 0; c < ACC_N / 2; c += 8) {
-                        *reinterpret_cast<uint4*>(P.dv + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
-                        *reinterpret_cast<uint4*>(P.dk + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
+                    for (int c = 0; c < D / 2; c += 8) {
+                        if (!AT || U.dh == 0)
+                            *reinterpret_cast<uint4*>(P.dv + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
+                        if (!AT || U.dh == 1)
+                            *reinterpret_cast<uint4*>(P.dk + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
                     }
                 }
                 continue;
@@ -823,6 +897,40 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 row_nd = P.ndvec[off];
             }
             const int key_row = U.row0 + r;  // KV mode
+            if constexpr (AT) {
+                // This thread's row of the unit's TMEM-resident operand (KV dv
+                // unit: K, dk unit: V; Q: q), its part's half of the d columns
+                // as bf16 pairs at TMEM columns A_COL + 64 part ..; rows past
+                // the sequence are zeros. The previous unit's UMMAs, which read
+                // these columns, completed before its epilogue (acc_done).
+                const __nv_bfloat16* src = nullptr;
+                if (KV) {
+                    if (key_row < U.S)
+                        src = (U.dh == 0 ? P.k : P.v) +
+                              ((static_cast<size_t>(U.kbase) + key_row) * P.Hkv + U.g) * D;
+                } else if (t_row < U.T) {
+                    src = P.q + ((static_cast<size_t>(U.qbase) + t_row) * P.H + 2 * U.g + hl_row) * D;
+                }
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {  // 2 x 32 columns = 128 d values
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                        if (src)
+                            x = __ldg(reinterpret_cast<const uint4*>(src + part * (D / 2) + 64 * hc) + i);
+                        w[4 * i] = x.x;
+                        w[4 * i + 1] = x.y;
+                        w[4 * i + 2] = x.z;
+                        w[4 * i + 3] = x.w;
+                    }
+                    tmem_st32(tmem + lane_addr + A_COL + 64 * part + 32 * hc, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ra_full);
+            }
             for (int c = 0; c < U.ncols; ++c) {
                 const int sl = ct & 1;
                 ok = mbar_wait(&xy_full[part], ct & 1, abort_flag, lim, SITE_BW_EW);
@@ -873,8 +981,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 for (int h2 = 0; h2 < HW / CHUNK; ++h2) {  // chunks of CHUNK columns
                     const int cb = col0 + CHUNK * h2;
                     uint32_t xv[CHUNK], yv[CHUNK];
-                    bw_ld_async<CHUNK>(tmem + lane_addr + BW_X_COL + cb, xv);
-                    bw_ld_async<CHUNK>(tmem + lane_addr + BW_Y_COL + cb, yv);
+                    // d = 256 dv unit: P only (no Y; dS is not formed)
+                    const bool want_y = !(AT && KV && U.dh == 0);
+                    bw_ld_async<CHUNK>(tmem + lane_addr + X_COL + cb, xv);
+                    if (want_y) {
+                        bw_ld_async<CHUNK>(tmem + lane_addr + Y_COL + cb, yv);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < CHUNK; ++i) yv[i] = 0u;
+                    }
                     tmem_wait_ld();
                     bw_fence<CHUNK>(xv);
                     bw_fence<CHUNK>(yv);
@@ -1013,10 +1128,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     // (no ordering between the two warps of a quadrant is needed)
                     const uint32_t zc = col0 + (CHUNK / 2) * h2;
                     if (KV) {
-                        bw_st<CHUNK / 2>(tmem + lane_addr + BW_X_COL + zc, pp);  // P^T
-                        bw_st<CHUNK / 2>(tmem + lane_addr + BW_Y_COL + zc, pd);  // dS^T
+                        // d = 256: the dv unit needs P^T only, the dk unit dS^T only
+                        if (!AT || U.dh == 0)
+                            bw_st<CHUNK / 2>(tmem + lane_addr + X_COL + zc, pp);  // P^T
+                        if (!AT || U.dh == 1)
+                            bw_st<CHUNK / 2>(tmem + lane_addr + Y_COL + zc, pd);  // dS^T
                     } else {
-                        bw_st<CHUNK / 2>(tmem + lane_addr + BW_X_COL + zc, pd);  // dS
+                        bw_st<CHUNK / 2>(tmem + lane_addr + X_COL + zc, pd);  // dS
                     }
                 }
                 tmem_wait_st();
@@ -1038,12 +1156,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const size_t row = (static_cast<size_t>(U.kbase) + key_row) * P.Hkv + U.g;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {  // a = 0: dv (columns 0..), a = 1: dk (ACC_N..)
+                    // d = 256: one accumulator at column 0, dv or dk by unit
+                    if (AT && a != U.dh) continue;
                     const float f = a ? P.query_scale : 1.0f;
-                    __nv_bfloat16* dst =
-                        (a ? P.dk : P.dv) + row * D + U.dh * ACC_N + part * HALF;
+                    const uint32_t acol = AT ? 0u : static_cast<uint32_t>(a * ACC_N);
+                    __nv_bfloat16* dst = (a ? P.dk : P.dv) + row * D + part * HALF;
 #pragma unroll
                     for (int sg = 0; sg < HALF / SEG; ++sg)
-                        bw_store_acc<SEG>(tmem + lane_addr + a * ACC_N + part * HALF + SEG * sg,
+                        bw_store_acc<SEG>(tmem + lane_addr + acol + part * HALF + SEG * sg,
                                           dst + SEG * sg, f, valid);
                 }
             } else {
