@@ -93,6 +93,9 @@ void fill_cap(float query_scale, float softcap, float& k_exp, float& cap_l2, flo
 }
 
 void fill_poly(float query_scale, float softcap, g2::PfParams& P) {
+    // fixed softmax shift when the cap bounds every logit tightly enough
+    P.fixed_ref_on = softcap > 0.f && softcap * kLog2e <= g2::PF_FIXED_REF_MAX;
+    P.fixed_ref = P.fixed_ref_on ? softcap * kLog2e - 64.0f : 0.f;
     P.u_scale = softcap > 0.f ? query_scale / softcap : 0.f;
     const float a = fabsf(query_scale);
     P.poly_acc_max = (softcap > 0.f && a > 0.f) ? g2::PF_POLY_U_MAX * softcap / a : INFINITY;

@@ -42,6 +42,7 @@ constexpr int PF_THREADS = PF_SOFTMAX_THREADS + 64;  // + producer warp + UMMA w
 constexpr int PF_BM = 128;   // MMA rows per tile (64 positions x 2 heads)
 constexpr int PF_QPOS = 64;  // query positions per tile
 constexpr int PF_BN = 128;   // keys per KV tile
+constexpr int PF_PHC = PF_BN / PF_NSPLIT;  // keys (S columns) per softmax column part
 constexpr int PF_TMEM_COLS = 512;
 constexpr int PF_S_COL0 = 256;  // S buffers at TMEM columns 256 and 384; O at 0
 constexpr float PF_RESCALE_LOG2 = 8.0f;
@@ -52,6 +53,9 @@ constexpr float kTanhC1 = -1.0f / 3.0f;
 constexpr float kTanhC2 = 2.0f / 15.0f;
 constexpr float kTanhC3 = -17.0f / 315.0f;
 constexpr float PF_POLY_U_MAX = 0.25f;  // |x / C| bound of the series path
+// Largest C log2(e) for which the fixed softmax shift keeps every weight a
+// normal float: 2^(-2 C log2(e) + 64) >= 2^-126.
+constexpr float PF_FIXED_REF_MAX = 95.0f;
 
 // CG = 1: one CTA per unit of 64 query positions. CG = 2 (d = 256 only): a CTA
 // pair per unit of 128 positions, 64 per CTA; each CTA stages half of every
@@ -106,6 +110,13 @@ struct PfParams {
     float u_scale;  // alpha/C             (cap on)
     float poly_acc_max;  // largest |q.k| for which |alpha q.k / C| <= PF_POLY_U_MAX
     int has_cap;
+    // Fixed softmax shift (cap on, C log2(e) <= PF_FIXED_REF_MAX): every capped
+    // logit lies in [-C log2(e), C log2(e)], so p = 2^(s2 - fixed_ref) with
+    // fixed_ref = C log2(e) - 64 stays in [2^(-2 C log2(e) + 64), 2^64]: normal
+    // in fp32 and bf16, and sums over up to 2^31 keys stay finite. The
+    // softmax is invariant to the shift, so no running max is needed.
+    int fixed_ref_on;
+    float fixed_ref;
     int out_align32;  // out is 32-byte aligned: the epilogue stores 32 bytes at a time
     unsigned long long timeout_ns;
 };
@@ -225,6 +236,43 @@ __device__ __forceinline__ int pf_key_row(const PfParams& P, const PfUnit& U, in
     int b = P.kv_table[static_cast<size_t>(U.seq) * P.kv_max_blocks + col];
     b = max(0, min(b, P.kv_num_blocks - 1));
     return (b << P.kv_block_shift) + (key & ((1 << P.kv_block_shift) - 1));
+}
+
+// Output rows of one warp (32 rows, one per lane, EC bf16 columns each as
+// EC/2 packed words) stored so that every store instruction writes whole row
+// segments: the 16-byte chunks are transposed within groups of NCH = EC/8
+// lanes by an XOR-shuffle butterfly (log2 NCH stages, half the chunks moving
+// in each), after which lane g*NCH + c holds chunk c of rows g*NCH + i in slot
+// i. row_ptr(i) gives the destination of warp row i, or nullptr to skip it.
+template <int EC, typename RowPtr>
+__device__ __forceinline__ void pf_store_rows(uint32_t (&w)[EC / 2], int lane, RowPtr row_ptr) {
+    constexpr int NCH = EC / 8;
+    static_assert(NCH == 4 || NCH == 8, "row segments of 64 or 128 bytes");
+#pragma unroll
+    for (int k = NCH / 2; k >= 1; k >>= 1) {
+        const bool upper = (lane & k) != 0;
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+            if (j & k) continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t send = upper ? w[4 * j + e] : w[4 * (j | k) + e];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, k);
+                if (upper)
+                    w[4 * j + e] = recv;
+                else
+                    w[4 * (j | k) + e] = recv;
+            }
+        }
+    }
+    const int grp = lane / NCH, ch = lane % NCH;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        __nv_bfloat16* dst = row_ptr(grp * NCH + i);
+        if (dst != nullptr)
+            *reinterpret_cast<uint4*>(dst + 8 * ch) =
+                make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
 }
 
 // Static persistent schedule: round r gives CTA c unit r*G + c (even rounds)
@@ -556,7 +604,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     const uint32_t v_lo = slot_lo0_v + slot * SLOT_STEP;
 #pragma unroll
                     for (int kk = 0; kk < C::VROWS / 16; ++kk) {
-                        const uint32_t a = p_tmem + (s * C::VROWS + kk * 16) / 2;
+                        // key kc of the tile: its P pair in the column part kc/HC,
+                        // at column part*HC + (kc % HC)/2
+                        const int kc = s * C::VROWS + kk * 16;
+                        const uint32_t a = p_tmem + (kc / PF_PHC) * PF_PHC + (kc % PF_PHC) / 2;
                         const uint32_t acc = (first && s == 0 && kk == 0) ? 0u : 1u;
                         if constexpr (PAIR)
                             umma_ts_lh_pair(tmem, a, v_lo + kk * ((16 * 128) >> 4), HI, IDESC_O, acc);
@@ -610,7 +661,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        constexpr int HC = PF_BN / PF_NSPLIT;           // key columns per part
+        constexpr int HC = PF_PHC;                      // key columns per part
         static_assert(HC % 32 == 0 && (D / PF_NSPLIT) % 16 == 0, "softmax split");
         constexpr int OC = D / PF_NSPLIT;               // O columns per part
         constexpr int EC = OC >= 64 ? 64 : OC;          // O columns per TMEM round trip
@@ -670,17 +721,31 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int j0 = (U.kt0 + jj) * PF_BN;  // key position of column 0
                 const bool boundary =
                     (j0 + PF_BN - 1 > U.p_min) || (P.window > 0 && j0 < U.p_max - P.window + 1);
-                // raw accumulator range of this warp's columns
-                float mxa[4], mna[4];
+                // Raw accumulator range of this warp's columns (the running max
+                // needs the tile max; with the fixed shift only max |x| is
+                // needed, for the series check).
+                float amx, amn;
+                if (P.fixed_ref_on) {
+                    float ma[4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) mxa[k] = mna[k] = s[k];
+                    for (int k = 0; k < 4; ++k) ma[k] = fabsf(s[k]);
 #pragma unroll
-                for (int i = 4; i < HC; i += 2) {
-                    mxa[(i >> 1) & 3] = fmax3f(mxa[(i >> 1) & 3], s[i], s[i + 1]);
-                    mna[(i >> 1) & 3] = fmin3f(mna[(i >> 1) & 3], s[i], s[i + 1]);
+                    for (int i = 4; i < HC; i += 2)
+                        ma[(i >> 1) & 3] = fmax3f(ma[(i >> 1) & 3], fabsf(s[i]), fabsf(s[i + 1]));
+                    amx = fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3]));
+                    amn = -amx;
+                } else {
+                    float mxa[4], mna[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mxa[k] = mna[k] = s[k];
+#pragma unroll
+                    for (int i = 4; i < HC; i += 2) {
+                        mxa[(i >> 1) & 3] = fmax3f(mxa[(i >> 1) & 3], s[i], s[i + 1]);
+                        mna[(i >> 1) & 3] = fmin3f(mna[(i >> 1) & 3], s[i], s[i + 1]);
+                    }
+                    amx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+                    amn = fminf(fminf(mna[0], mna[1]), fminf(mna[2], mna[3]));
                 }
-                const float amx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
-                const float amn = fminf(fminf(mna[0], mna[1]), fminf(mna[2], mna[3]));
                 // Fast path: no mask in this tile, cap on, |x/C| <= 1/4 for the
                 // whole warp. The capped map is monotonic in x, so the tile max
                 // is the map of the extreme accumulators and s2 - m fuses into
@@ -689,10 +754,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const bool fast = __all_sync(
                     0xffffffffu, !boundary && (!P.has_cap ||
                                                fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max));
-                float mt;
+                float mt = 0.f;
                 if (fast) {
-                    mt = P.has_cap ? fmaxf(series_s2(amx), series_s2(amn))
-                                   : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
+                    if (!P.fixed_ref_on)
+                        mt = P.has_cap ? fmaxf(series_s2(amx), series_s2(amn))
+                                       : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
                 } else {
                     // general path: capped logits in log2 units, then the mask
                     if (P.has_cap) {
@@ -719,51 +785,58 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         for (int i = 0; i < HC; ++i)
                             if (i > hi || i < lo) s[i] = -INFINITY;
                     }
-                    float mx[4];
+                    if (!P.fixed_ref_on) {
+                        float mx[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mx[k] = s[k];
+                        for (int k = 0; k < 4; ++k) mx[k] = s[k];
 #pragma unroll
-                    for (int i = 4; i < HC; i += 2)
-                        mx[(i >> 1) & 3] = fmax3f(mx[(i >> 1) & 3], s[i], s[i + 1]);
-                    mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                        for (int i = 4; i < HC; i += 2)
+                            mx[(i >> 1) & 3] = fmax3f(mx[(i >> 1) & 3], s[i], s[i + 1]);
+                        mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    }
                 }
-                // row max over all parts
-                xmax[(buf * PF_NSPLIT + part) * 128 + r] = mt;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&xbar[qd * 2 + buf]);  // release for the warp
-                ok = mbar_wait(&xbar[qd * 2 + buf], (gt >> 1) & 1, abort_flag, lim,
-                               SITE_SM_PAIR);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-#pragma unroll
-                for (int k = 0; k < PF_NSPLIT; ++k)
-                    mt = fmaxf(mt, xmax[(buf * PF_NSPLIT + k) * 128 + r]);
-                const float m_new = fmaxf(m_ref, mt);
-                const bool need = (m_ref != -INFINITY) && (m_new > m_ref + PF_RESCALE_LOG2);
-                if (__any_sync(0xffffffffu, need)) {
-                    // O holds PV(0..gt-1) relative to m_ref: scale this part to m_new.
-                    ok = mbar_wait(&o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, abort_flag,
-                                         lim, SITE_SM_O_DONE);
+                if (P.fixed_ref_on) {
+                    // fixed shift: no running max, no exchange, no rescaling
+                    m_ref = P.fixed_ref;
+                } else {
+                    // row max over all parts
+                    xmax[(buf * PF_NSPLIT + part) * 128 + r] = mt;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&xbar[qd * 2 + buf]);  // release for the warp
+                    ok = mbar_wait(&xbar[qd * 2 + buf], (gt >> 1) & 1, abort_flag, lim,
+                                   SITE_SM_PAIR);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
-                    tc_fence_after();
-                    const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
-                    const uint32_t o_addr = tmem + lane_addr + part * OC;
-#pragma unroll 1
-                    for (int c = 0; c < OC / 32; ++c) {  // 32 columns per TMEM round trip
-                        uint32_t v[32];
-                        tmem_ld32(o_addr + c * 32, v);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-                        tmem_st32(o_addr + c * 32, v);
+                    for (int k = 0; k < PF_NSPLIT; ++k)
+                        mt = fmaxf(mt, xmax[(buf * PF_NSPLIT + k) * 128 + r]);
+                    const float m_new = fmaxf(m_ref, mt);
+                    const bool need = (m_ref != -INFINITY) && (m_new > m_ref + PF_RESCALE_LOG2);
+                    if (__any_sync(0xffffffffu, need)) {
+                        // O holds PV(0..gt-1) relative to m_ref: scale this part to m_new.
+                        ok = mbar_wait(&o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, abort_flag,
+                                             lim, SITE_SM_O_DONE);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
+                        const uint32_t o_addr = tmem + lane_addr + part * OC;
+#pragma unroll 1
+                        for (int c = 0; c < OC / 32; ++c) {  // 32 columns per TMEM round trip
+                            uint32_t v[32];
+                            tmem_ld32(o_addr + c * 32, v);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+                            tmem_st32(o_addr + c * 32, v);
+                        }
+                        tmem_wait_st();
+                        l *= f;
+                        lr *= f;
+                        if (need) m_ref = m_new;
                     }
-                    tmem_wait_st();
-                    l *= f;
-                    lr *= f;
-                    if (need) m_ref = m_new;
-                }
-                if (m_ref == -INFINITY) m_ref = mt;
+                    if (m_ref == -INFINITY) m_ref = mt;
+                }  // running max
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
                 // The PV product sees bf16(p); normalising O by the sum of the
                 // same rounded weights makes them sum to one exactly, so their
@@ -811,12 +884,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                                                                   __uint_as_float(pk[i] & 0xFFFF0000u)));
                     }
                 }
+                // P of this part's HC keys as bf16 pairs: HC/2 columns at the
+                // start of its own S columns, which it has already read (the
+                // other part's S columns may still be unread)
 #pragma unroll
-                for (int c = 0; c < HC / 32; ++c) {  // bf16 pairs: HC/2 columns
+                for (int c = 0; c < HC / 32; ++c) {
                     uint32_t pc[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pc[i] = pk[16 * c + i];
-                    tmem_st16(s_addr + part * (HC / 2) + 16 * c, pc);
+                    tmem_st16(s_addr + part * HC + 16 * c, pc);
                 }
                 const float2 lsum = add2(ls[0], ls[1]);
                 const float2 lrsum = add2(lrs[0], lrs[1]);
@@ -858,40 +934,31 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const bool valid = pr < U.tvalid;
             const int h = 2 * U.g + hl;
             const float inv_l = 1.0f / lr;
-            const size_t orow = static_cast<size_t>(U.qbase + U.t0 + pr) * P.H + h;
-            __nv_bfloat16* optr = P.out + orow * D + part * OC;
             const uint32_t o_addr = tmem + lane_addr + part * OC;
+            // destination of warp row rw (TMEM lane 32 qd + rw) for O columns part*OC + col
+            auto row_ptr = [&](int rw, int col) -> __nv_bfloat16* {
+                const int rr = (qd << 5) | rw;
+                const int prr = rr & 63;
+                if (prr >= U.tvalid) return nullptr;
+                return P.out + (static_cast<size_t>(U.qbase + U.t0 + prr) * P.H + 2 * U.g +
+                                (rr >> 6)) * D + part * OC + col;
+            };
 #pragma unroll 1
             for (int c = 0; c < OC / EC; ++c) {  // EC columns per TMEM round trip
                 uint32_t v[EC / 32][32];
 #pragma unroll
                 for (int j = 0; j < EC / 32; ++j) tmem_ld32_async(o_addr + c * EC + 32 * j, v[j]);
                 tmem_wait_ld();
+                uint32_t w[EC / 2];
 #pragma unroll
                 for (int j = 0; j < EC / 32; ++j) {
                     tmem_reg_fence(v[j]);
-                    uint32_t pkk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        pkk[i] = pack_bf16x2(__uint_as_float(v[j][2 * i]) * inv_l,
-                                             __uint_as_float(v[j][2 * i + 1]) * inv_l);
-                    if (valid) {
-                        __nv_bfloat16* dst = optr + c * EC + 32 * j;
-                        if (P.out_align32) {  // two 32-byte stores: one full sector each
-#pragma unroll
-                            for (int q8 = 0; q8 < 2; ++q8)
-                                st_global_v8(dst + 16 * q8, pkk[8 * q8], pkk[8 * q8 + 1],
-                                             pkk[8 * q8 + 2], pkk[8 * q8 + 3], pkk[8 * q8 + 4],
-                                             pkk[8 * q8 + 5], pkk[8 * q8 + 6], pkk[8 * q8 + 7]);
-                        } else {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4)
-                                d4[q4] = make_uint4(pkk[4 * q4], pkk[4 * q4 + 1], pkk[4 * q4 + 2],
-                                                    pkk[4 * q4 + 3]);
-                        }
-                    }
+                        w[16 * j + i] = pack_bf16x2(__uint_as_float(v[j][2 * i]) * inv_l,
+                                                    __uint_as_float(v[j][2 * i + 1]) * inv_l);
                 }
+                pf_store_rows<EC>(w, lane, [&](int rw) { return row_ptr(rw, c * EC); });
             }
             if (valid && part == 0 && P.lse != nullptr) {
                 const float lse = (m_ref + log2f(l)) * 0.69314718055994531f;
