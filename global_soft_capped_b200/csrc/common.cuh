@@ -42,6 +42,8 @@ enum WaitSite : unsigned int {
     SITE_BW_MMA_Z = 16,     // backward issuer: P / dS written back
     SITE_BW_MMA_ACC = 17,   // backward issuer: accumulators read out
     SITE_BW_EW_ACC = 18,    // backward elementwise: accumulation finished
+    SITE_EPI_O_DONE = 19,   // forward epilogue: the unit's last PV completed
+    SITE_EPI_STATS = 20,    // forward epilogue: row statistics handed over
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -6,17 +6,24 @@
 // window on local layers, softmax over keys, grouped mix of the values);
 // cap formula from the "Gemma 2 Guide", section 1.
 //
-// Design (one persistent CTA per SM, 320 threads, warp-specialised):
-//   warps 0..7  softmax + epilogue: warps w and w+4 share MMA rows 32*(w%4)..+31
-//               (the TMEM lanes of their sub-partition); part w/4 takes key
-//               columns 64*part..+63 of every S tile and O columns
-//               part*D/2..+D/2-1. The parts exchange their partial row maxima
-//               through shared memory once per tile (a bounded mbarrier wait),
-//               so both use the same running max.
+// Design (one persistent CTA per SM, 512 threads, warp-specialised):
+//   warps 0..7  softmax: warps w and w+4 share MMA rows 32*(w%4)..+31 (the
+//               TMEM lanes of their sub-partition); part w/4 takes key columns
+//               64*part..+63 of every S tile and O columns part*D/2..+D/2-1
+//               when O is rescaled. With a running max the parts exchange
+//               their partial row maxima through shared memory once per tile
+//               (a bounded mbarrier wait), so both use the same one. At the end
+//               of a unit they hand the row sums to the epilogue warps and go
+//               on with the next unit.
 //   warp 8      TMA producer: Q tile once per work unit, then K/V tiles into a
 //               ring of shared-memory slots (128-byte swizzle).
 //   warp 9      UMMA issuer (one thread): S = Q K^T into TMEM (two S buffers),
 //               O += P V with P read from TMEM; owns the TMEM allocation.
+//   warps 12..15 epilogue, one per TMEM lane quadrant: once a unit's last PV
+//               has completed, O / l -> bf16 rows and the log-sum-exp, while
+//               the softmax warps already work on the next unit; the next
+//               unit's first PV waits until O has been read. (Warps 10 and 11
+//               only keep the warpgroups aligned.)
 // A work unit is (sequence, KV head g, 64 query positions); its 128 MMA rows
 // are the two query heads 2g, 2g+1 that share KV head g (row = head_local*64 +
 // position), so each K/V tile feeds both heads. Only KV tiles that intersect
@@ -38,7 +45,9 @@ constexpr int PF_NSPLIT = 2;     // softmax warps per TMEM lane quadrant
 constexpr int PF_SOFTMAX_THREADS = 128 * PF_NSPLIT;
 constexpr int PF_WARP_PRODUCER = 4 * PF_NSPLIT;
 constexpr int PF_WARP_MMA = PF_WARP_PRODUCER + 1;
-constexpr int PF_THREADS = PF_SOFTMAX_THREADS + 64;  // + producer warp + UMMA warp
+constexpr int PF_WARP_EPI = PF_WARP_PRODUCER + 4;   // warps 12..15
+constexpr int PF_EPI_WARPS = 4;
+constexpr int PF_THREADS = PF_SOFTMAX_THREADS + 256;  // + producer, issuer, 2 idle, 4 epilogue
 constexpr int PF_BM = 128;   // MMA rows per tile (64 positions x 2 heads)
 constexpr int PF_QPOS = 64;  // query positions per tile
 constexpr int PF_BN = 128;   // keys per KV tile
@@ -76,7 +85,10 @@ struct PfCfg {
     static constexpr int MAX_SEQ_TABLE = 1024;  // varlen: sequences per launch
     static constexpr int VL_BYTES = 4 * (3 * MAX_SEQ_TABLE + 1);
     static constexpr int SMEM_TILES = Q_BYTES + NSLOT * SLOT_BYTES;
-    static constexpr int CTRL_BYTES = 1024 + 2 * PF_NSPLIT * 128 * 4 + PF_NSPLIT * 128 * 2 * 4;
+    // barriers, partial row maxima [2][NSPLIT][128], row statistics handed to
+    // the epilogue by unit parity: sums [2][NSPLIT][128][2], maxima [2][128]
+    static constexpr int CTRL_BYTES =
+        1024 + 2 * PF_NSPLIT * 128 * 4 + 2 * PF_NSPLIT * 128 * 2 * 4 + 2 * 128 * 4;
     static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + CTRL_BYTES + VL_BYTES;
     static_assert(KCOLS % 64 == 0 && KCOLS <= D && VROWS % 16 == 0 && VROWS <= PF_BN,
                   "tile shapes");
@@ -301,17 +313,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint64_t* o_done = bars + 6;   // [2]: PV(t) completes phase t/2 of o_done[t%2]
     uint64_t* o_free = bars + 8;
     uint64_t* drain = bars + 9;
-    uint64_t* slot_full = bars + 10;              // [NSLOT]
-    uint64_t* slot_empty = bars + 10 + C::NSLOT;  // [NSLOT]
-    // softmax warp pairs: max exchange per tile parity [4][2], sum exchange [4]
-    uint64_t* xbar = bars + 10 + 2 * C::NSLOT;
-    uint64_t* sbar = xbar + 8;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sbar + 4);
+    // the last PV of a unit completed (one phase per unit): the epilogue warps
+    // wait on it first, so that their o_done wait is never more than one
+    // phase behind (o_done completes a phase per tile)
+    uint64_t* o_last = bars + 10;
+    uint64_t* slot_full = bars + 11;              // [NSLOT]
+    uint64_t* slot_empty = bars + 11 + C::NSLOT;  // [NSLOT]
+    // softmax warp pairs: max exchange per tile parity [4][2]
+    uint64_t* xbar = bars + 11 + 2 * C::NSLOT;
+    // row statistics of a unit handed to the epilogue warps, by unit parity [2]
+    uint64_t* stat_full = xbar + 8;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(stat_full + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     // partial row maxima of the column parts, by tile parity: [2][NSPLIT][128]
     float* xmax = reinterpret_cast<float*>(base + C::SMEM_TILES + 1024);
-    // partial (l, lr) row sums of the parts at the end of a unit: [NSPLIT][128][2]
+    // partial (l, lr) row sums of the parts at the end of a unit, by unit
+    // parity: [2][NSPLIT][128][2]; the row's reference max: [2][128]
     float* xsum = xmax + 2 * PF_NSPLIT * 128;
+    float* xref = xsum + 2 * PF_NSPLIT * 128 * 2;
     VlTables vt;
     vt.work = reinterpret_cast<int*>(base + C::SMEM_TILES + C::CTRL_BYTES);
     vt.order = vt.work + C::MAX_SEQ_TABLE;
@@ -328,13 +347,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             mbar_init(&p_full[i], CG * PF_SOFTMAX_THREADS / 32);
             mbar_init(&o_done[i], 1);
         }
-        // softmax-side barriers take one arrival per warp (elected lane, after
-        // __syncwarp orders the whole warp's prior writes before it); a pair
-        // counts the warps of both CTAs on the even CTA's p_full and o_free
-        mbar_init(o_free, CG * PF_SOFTMAX_THREADS / 32);
+        // softmax- and epilogue-side barriers take one arrival per warp
+        // (elected lane, after __syncwarp orders the whole warp's prior
+        // writes before it); a pair counts the warps of both CTAs on the even
+        // CTA's p_full and o_free
+        mbar_init(o_free, CG * PF_EPI_WARPS);
         for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], PF_NSPLIT);
-        for (int i = 0; i < 4; ++i) mbar_init(&sbar[i], PF_NSPLIT);
+        for (int i = 0; i < 2; ++i) mbar_init(&stat_full[i], PF_SOFTMAX_THREADS / 32);
         mbar_init(drain, 1);
+        mbar_init(o_last, 1);
         for (int i = 0; i < C::NSLOT; ++i) {
             mbar_init(&slot_full[i], 1);
             mbar_init(&slot_empty[i], 1);
@@ -649,6 +670,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     tc_fence_after();
                     ok = issue_pv(gt, jj == 0);
                 }
+                if (!ok) break;
+                commit(o_last);  // the unit's last PV issued
                 tile += U.nkt;
                 ++unit_it;
             }
@@ -659,8 +682,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             mbar_wait_drain(drain, 0, lim);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ softmax + epilogue
+    } else if (warp < PF_WARP_PRODUCER) {
+        // ------------------------------------------------------------ softmax
         constexpr int HC = PF_PHC;                      // key columns per part
         static_assert(HC % 32 == 0 && (D / PF_NSPLIT) % 16 == 0, "softmax split");
         constexpr int OC = D / PF_NSPLIT;               // O columns per part
@@ -909,42 +932,71 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
             }
             if (!ok) break;
-            // ---- epilogue: O / lr -> bf16, lse
+            // ---- hand the row statistics to the epilogue warps
+            const int sb = unit_it & 1;
+            xsum[((sb * PF_NSPLIT + part) * 128 + r) * 2 + 0] = l;
+            xsum[((sb * PF_NSPLIT + part) * 128 + r) * 2 + 1] = lr;
+            if (part == 0) xref[sb * 128 + r] = m_ref;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&stat_full[sb]);
+            tile += U.nkt;
+            ++unit_it;
+        }
+    } else if (warp >= PF_WARP_EPI) {
+        // ------------------------------------------------------------ epilogue
+        // O / lr -> bf16 and lse of each unit, one row (TMEM lane) per thread,
+        // all D columns. lr sums the bf16-rounded weights that PV used, so the
+        // weights of a row sum to one exactly; l (fp32 weights) gives the lse.
+        constexpr int EC = 64;                          // O columns per TMEM round trip
+        static_assert(D % EC == 0, "epilogue chunks");
+        const int qd = warp & 3;                        // TMEM lane quadrant
+        const int r = (qd << 5) | lane;                 // MMA row == TMEM lane
+        const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
+        const int hl = r >> 6;                          // head within the pair
+        const int pr = r & 63;                          // position within the tile
+        uint32_t tile = 0;
+        int unit_it = 0;
+        bool ok = true;
+        for (int rr = 0; ok && rr * G < num_units; ++rr) {
+            const int u = pf_sched(rr, cta, G);
+            if (u >= num_units) continue;
+            PfUnit U;
+            pf_unit<CG>(P, vt, u, U, rank);
             // PV(gl) completing implies every earlier UMMA of this CTA completed.
+            // o_last first (at most one unit ahead: the next unit's first PV
+            // waits for this epilogue), then the unit's last o_done phase, so
+            // that its arrival has landed before this CTA can leave.
             const uint32_t gl = tile + U.nkt - 1;
-            ok = mbar_wait(&o_done[gl & 1], (gl >> 1) & 1, abort_flag, lim, SITE_SM_O_DONE);
+            const int sb = unit_it & 1;
+            ok = mbar_wait(o_last, unit_it & 1, abort_flag, lim, SITE_EPI_O_DONE);
+            if (ok)
+                ok = mbar_wait(&o_done[gl & 1], (gl >> 1) & 1, abort_flag, lim,
+                               SITE_EPI_O_DONE);
+            if (ok)
+                ok = mbar_wait(&stat_full[sb], (unit_it >> 1) & 1, abort_flag, lim,
+                               SITE_EPI_STATS);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            // combine the parts' sums
-            xsum[(part * 128 + r) * 2 + 0] = l;
-            xsum[(part * 128 + r) * 2 + 1] = lr;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sbar[qd]);
-            ok = mbar_wait(&sbar[qd], unit_it & 1, abort_flag, lim, SITE_SM_PAIR);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            l = 0.f;
-            lr = 0.f;
+            float l = 0.f, lr = 0.f;
 #pragma unroll
             for (int k = 0; k < PF_NSPLIT; ++k) {
-                l += xsum[(k * 128 + r) * 2 + 0];
-                lr += xsum[(k * 128 + r) * 2 + 1];
+                l += xsum[((sb * PF_NSPLIT + k) * 128 + r) * 2 + 0];
+                lr += xsum[((sb * PF_NSPLIT + k) * 128 + r) * 2 + 1];
             }
-            const bool valid = pr < U.tvalid;
-            const int h = 2 * U.g + hl;
+            const float m_ref = xref[sb * 128 + r];
             const float inv_l = 1.0f / lr;
-            const uint32_t o_addr = tmem + lane_addr + part * OC;
-            // destination of warp row rw (TMEM lane 32 qd + rw) for O columns part*OC + col
+            const uint32_t o_addr = tmem + lane_addr;
+            // destination of warp row rw (TMEM lane 32 qd + rw), O column col
             auto row_ptr = [&](int rw, int col) -> __nv_bfloat16* {
-                const int rr = (qd << 5) | rw;
-                const int prr = rr & 63;
+                const int rq = (qd << 5) | rw;
+                const int prr = rq & 63;
                 if (prr >= U.tvalid) return nullptr;
                 return P.out + (static_cast<size_t>(U.qbase + U.t0 + prr) * P.H + 2 * U.g +
-                                (rr >> 6)) * D + part * OC + col;
+                                (rq >> 6)) * D + col;
             };
 #pragma unroll 1
-            for (int c = 0; c < OC / EC; ++c) {  // EC columns per TMEM round trip
+            for (int c = 0; c < D / EC; ++c) {
                 uint32_t v[EC / 32][32];
 #pragma unroll
                 for (int j = 0; j < EC / 32; ++j) tmem_ld32_async(o_addr + c * EC + 32 * j, v[j]);
@@ -960,7 +1012,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
                 pf_store_rows<EC>(w, lane, [&](int rw) { return row_ptr(rw, c * EC); });
             }
-            if (valid && part == 0 && P.lse != nullptr) {
+            if (pr < U.tvalid && P.lse != nullptr) {
+                const int h = 2 * U.g + hl;
                 const float lse = (m_ref + log2f(l)) * 0.69314718055994531f;
                 size_t li;
                 if (P.varlen)

@@ -250,9 +250,11 @@ G2ATTN_API size_t g2attn_backward_workspace_size(int B, int T, int H);
  *   workspace: device memory of at least
  *     g2attn_backward_workspace_size(B, T, H) bytes, 16-byte aligned, owned by
  *     the caller and overwritten.
- * Supported: d = 64, 128 and 256. At d = 256 the streamed tiles are 32 rows
- * and the dk/dv kernel runs each 128-key tile as two units, one per half of
- * the d columns, so that its accumulators fit the 512 TMEM columns of an SM.
+ * Supported: d = 64, 128 and 256. At d = 256 one of the two resident tiles of
+ * each gradient kernel is held in tensor memory (it is read by the UMMAs as
+ * their A operand), the streamed tiles are 64 rows, and the dk/dv kernel runs
+ * each 128-key tile as two units, one accumulating dv and one dk, so that an
+ * accumulator fits the 512 TMEM columns of an SM next to X and Y.
  * Other limits and errors as g2attn_prefill; lse is required; a workspace that
  * is missing or too small returns G2ATTN_ERR_WORKSPACE. Three kernels run on
  * `stream`: a pass computing D and lse*log2(e), the dk/dv kernel (K, V tiles
