@@ -727,27 +727,54 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
                 umma_commit(&xy_full[h]);
             };
-            // Both halves of the tile in slot sl as one UMMA pair (N = CR): with
-            // 32-row column tiles (d = 256) an N = 16 half re-reads the whole
-            // 128-row resident A tile per UMMA, which makes shared-memory
-            // bandwidth the limit; one N = 32 UMMA reads it once per tile.
-            auto issue_xy_tile = [&](int sl) {
+            // Both halves of the tile in slot sl as one UMMA pair (N = CR): fewer,
+            // wider UMMAs, and a resident A tile in shared memory is read once
+            // per tile instead of once per half.
+            auto issue_xy_tile = [&](int sl, int kind) {
                 constexpr uint32_t IDESC_XYT = idesc_bf16(128, C::CR, false);
                 const uint32_t c1 = slot_lo + sl * SLOT_STEP;
                 const uint32_t c2 = c1 + CTILE_STEP;
+                if constexpr (AT) {  // A operands as in issue_xy
+                    const bool x_tmem = !KV || kind == 0;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
-                               IDESC_XYT, kk != 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        if (x_tmem)
+                            umma_ts_lh(tmem + X_COL, tmem + A_COL + 8 * kk, c1 + kstep_c(kk), HI,
+                                       IDESC_XYT, kk != 0);
+                        else
+                            umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                                       IDESC_XYT, kk != 0);
+                    }
+                    if (!KV || kind == 1) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_lh(tmem + Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
-                               IDESC_XYT, kk != 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            if (KV)
+                                umma_ts_lh(tmem + Y_COL, tmem + A_COL + 8 * kk, c2 + kstep_c(kk),
+                                           HI, IDESC_XYT, kk != 0);
+                            else
+                                umma_ss_lh(tmem + Y_COL, r1_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                                           IDESC_XYT, kk != 0);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                                   IDESC_XYT, kk != 0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss_lh(tmem + Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                                   IDESC_XYT, kk != 0);
+                }
                 umma_commit(&xy_full[0]);
                 umma_commit(&xy_full[1]);
             };
-            constexpr bool TILE_XY = HW < 32;
-            static_assert(!(TILE_XY && AT), "whole-tile X / Y only with both resident tiles in shared memory");
+            // Whole-tile X / Y at d = 256 (N = 64): one thread issues a
+            // tcgen05.mma about every 67 cycles however small it is, so N = 32
+            // halves (16 cycles of math each at M = 128) leave the tensor pipe
+            // mostly idle; at d <= 128 the N = 64 halves and their overlap with
+            // the elementwise warps measured faster.
+            constexpr bool TILE_XY = HW < 32 || AT;
             // accumulations over the half's HW rows (K indices HW h ..): A = the
             // bf16 operand the half's warps wrote at columns HW h + 8 k4; B =
             // the streamed tile read MN-major (all D columns)
@@ -799,7 +826,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 if constexpr (TILE_XY) {
-                    issue_xy_tile(ct & 1);
+                    issue_xy_tile(ct & 1, U.dh);
                 } else {
                     issue_xy(ct & 1, 0, U.dh);
                     issue_xy(ct & 1, 1, U.dh);
@@ -833,7 +860,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                            SITE_BW_MMA);
                             if (!ok) break;
                             tc_fence_after();
-                            issue_xy_tile(sl ^ 1);
+                            issue_xy_tile(sl ^ 1, U.dh);
                         } else {
                             issue_xy(sl ^ 1, 1, U.dh);
                         }

@@ -693,7 +693,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int part = warp >> 2;                     // column part of this warp
         const int r = (qd << 5) | lane;                 // MMA row == TMEM lane
         const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
-        const int hl = r >> 6;                          // head within the pair
         const int pr = r & 63;                          // position within the tile
         const int col0 = part * HC;                     // first S column of this warp
         // s2 = x * (b0 + b1 x^2 + b2 x^4 + b3 x^6) with b_k = alpha*log2(e)*c_k*(alpha/C)^(2k):
