@@ -40,10 +40,11 @@ namespace g2 {
 
 constexpr int BW_KV = 0;
 constexpr int BW_Q = 1;
-constexpr int BW_THREADS = 320;          // 8 elementwise warps, producer, UMMA issuer
+constexpr int BW_THREADS = 352;          // 8 elementwise warps, producer, 2 UMMA issuers
 constexpr int BW_EW_THREADS = 256;
 constexpr int BW_WARP_PRODUCER = 8;
-constexpr int BW_WARP_MMA = 9;
+constexpr int BW_WARP_MMA = 9;           // issuer 0: X and the accumulation reading X; TMEM owner
+constexpr int BW_WARP_MMA2 = 10;         // issuer 1 (d = 256): Y and the accumulation reading Y
 constexpr int BW_QPOS = 64;              // query positions per column/row tile (x 2 heads)
 constexpr int BW_KEYS = 128;             // keys per tile
 constexpr int BW_X_COL = 256;
@@ -71,6 +72,10 @@ struct BwCfg {
     static constexpr int CHUNK = HW < 32 ? HW : 32;      // columns per TMEM round trip
     static constexpr int DSPLIT_KV = D == 256 ? 2 : 1;   // dk/dv kernel: units per key tile
     static constexpr int RES_TILES = A_TMEM ? 1 : 2;     // resident tiles in shared memory
+    // UMMA issuing threads: two at d = 256 (measured 7-8% faster); at d <= 128
+    // a second issuer measured 4-6% slower than one issuing everything in the
+    // X / Y / accumulation order of the column-half pipeline
+    static constexpr int ISSUERS = A_TMEM ? 2 : 1;
     static constexpr int TILE_BYTES = 128 * D * 2;       // one 128-row resident tile
     static constexpr int CTILE_BYTES = CR * D * 2;       // one streamed column tile
     static constexpr int VEC_BYTES = 1024;               // -lse2, -D of the tile's query rows
@@ -487,18 +492,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(r_full, 1);
-        mbar_init(r_empty, 1);
+        mbar_init(r_empty, C::ISSUERS);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&c_full[i], 1);
-            mbar_init(&c_empty[i], 1);
+            mbar_init(&c_empty[i], C::ISSUERS);
         }
         for (int h = 0; h < 2; ++h) {
-            mbar_init(&xy_full[h], 1);
+            mbar_init(&xy_full[h], C::ISSUERS);
             mbar_init(&z_full[h], BW_EW_THREADS / 64);
         }
-        mbar_init(acc_done, 1);
+        mbar_init(acc_done, C::ISSUERS);
         mbar_init(acc_free, BW_EW_THREADS / 32);
-        mbar_init(drain, 1);
+        mbar_init(drain, C::ISSUERS);
         mbar_init(ra_full, BW_EW_THREADS / 32);
         *abort_flag = 0;
         fence_mbar_init();
@@ -657,8 +662,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
         __syncwarp();
     }
-    else if (warp == BW_WARP_MMA) {
-        // ------------------------------------------------------------ UMMA issuer
+    else if (warp == BW_WARP_MMA || (C::ISSUERS == 2 && warp == BW_WARP_MMA2)) {
+        // ------------------------------------------------------------ UMMA issuers
+        // One thread issues a tcgen05.mma about every 67 cycles, less than the
+        // math of the N = 64 UMMAs at d = 256, so there two threads in
+        // different warps share the issue: issuer 0 X and the accumulation
+        // that reads X (dv, or dq), issuer 1 Y and the accumulation that reads
+        // Y (dk). Neither writes what the other's UMMAs read, and each keeps
+        // its own order (X(c+1) after the accumulation over X(c)'s P, Y(c+1)
+        // after the one over Y(c)'s dS). Both take every wait; the barriers
+        // their commits complete count both. At d <= 128 issuer 0 issues all.
+        const int role = warp - BW_WARP_MMA;
+        const bool do_x = role == 0;
+        const bool do_y = C::ISSUERS == 2 ? role == 1 : role == 0;
         if (lane == 0) {
             constexpr int HW = C::HW;
             constexpr uint32_t IDESC_XY = idesc_bf16(128, HW, false);  // one column half
@@ -697,6 +713,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     const bool x_tmem = !KV || kind == 0;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
+                        if (!do_x) break;
                         if (x_tmem)
                             umma_ts_lh(tmem + X_COL + HW * h, tmem + A_COL + 8 * kk,
                                        c1 + kstep_c(kk), HI, IDESC_XY, kk != 0);
@@ -704,7 +721,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk),
                                        HI, IDESC_XY, kk != 0);
                     }
-                    if (!KV || kind == 1) {
+                    if (do_y && (!KV || kind == 1)) {
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             if (KV)
@@ -716,14 +733,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         }
                     }
                 } else {
+                    if (do_x) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
-                                   IDESC_XY, kk != 0);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk),
+                                       HI, IDESC_XY, kk != 0);
+                    }
+                    if (do_y) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss_lh(tmem + Y_COL + HW * h, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
-                                   IDESC_XY, kk != 0);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lh(tmem + Y_COL + HW * h, r2_lo + kstep(kk), c2 + kstep_c(kk),
+                                       HI, IDESC_XY, kk != 0);
+                    }
                 }
                 umma_commit(&xy_full[h]);
             };
@@ -738,6 +759,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     const bool x_tmem = !KV || kind == 0;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
+                        if (!do_x) break;
                         if (x_tmem)
                             umma_ts_lh(tmem + X_COL, tmem + A_COL + 8 * kk, c1 + kstep_c(kk), HI,
                                        IDESC_XYT, kk != 0);
@@ -745,7 +767,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
                                        IDESC_XYT, kk != 0);
                     }
-                    if (!KV || kind == 1) {
+                    if (do_y && (!KV || kind == 1)) {
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             if (KV)
@@ -757,14 +779,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         }
                     }
                 } else {
+                    if (do_x) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
-                                   IDESC_XYT, kk != 0);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lh(tmem + X_COL, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                                       IDESC_XYT, kk != 0);
+                    }
+                    if (do_y) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss_lh(tmem + Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
-                                   IDESC_XYT, kk != 0);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lh(tmem + Y_COL, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                                       IDESC_XYT, kk != 0);
+                    }
                 }
                 umma_commit(&xy_full[0]);
                 umma_commit(&xy_full[1]);
@@ -791,13 +817,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (KV) {
                         // dv += P^T dout (P^T at X), dk += dS^T q (dS^T at Y); at
                         // d = 256 the dv unit does the first, the dk unit the second
-                        if (!AT || kind == 0)
+                        if (do_x && (!AT || kind == 0))
                             umma_ts_lh(tmem + 0, tmem + X_COL + zc, c2_mn + bstep, HI, IDESC_ACC,
                                        acc);
-                        if (!AT || kind == 1)
+                        if (do_y && (!AT || kind == 1))
                             umma_ts_lh(tmem + (AT ? 0 : ACC_N), tmem + Y_COL + zc, c1_mn + bstep,
                                        HI, IDESC_ACC, acc);
-                    } else {
+                    } else if (do_x) {
                         // dq += dS K (dS at X)
                         umma_ts_lh(tmem + 0, tmem + X_COL + zc, c1_mn + bstep, HI, IDESC_ACC,
                                    acc);
@@ -878,8 +904,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
         __syncwarp();
     }
-    else {
+    else if (warp < BW_WARP_PRODUCER) {
         // ------------------------------------------------------------ elementwise + epilogue
+        // (warps 0-7 only: warp 10 is idle when one thread issues the UMMAs)
         // Warps w and w+4 share TMEM lane quadrant w%4 (rows 32(w%4)..+31);
         // warp w takes columns 0..HW-1 of X and Y, warp w+4 columns HW..2HW-1.
         // KV mode: row = key, column = query row (head 2g + column/CQ). Q mode:
