@@ -481,7 +481,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* acc_free = bars + 11; // epilogue read the accumulators (8 warp arrivals)
     uint64_t* drain = bars + 12;
     uint64_t* ra_full = bars + 13;  // d = 256: the unit's TMEM-resident operand written (8 warps)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+    // d = 256 dv units: X double-buffered in the X and Y columns (a dv unit
+    // has no Y); xb_full[b] = X of the next tile of buffer b is in TMEM
+    uint64_t* xb_full = bars + 14;  // [2]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     // varlen tables: cum[num_seqs + 1] (unit prefix in rank order), order[], work[]
     int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
@@ -505,6 +508,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         mbar_init(acc_free, BW_EW_THREADS / 32);
         mbar_init(drain, C::ISSUERS);
         mbar_init(ra_full, BW_EW_THREADS / 32);
+        for (int b = 0; b < 2; ++b) mbar_init(&xb_full[b], C::ISSUERS);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -693,7 +697,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
             constexpr uint32_t CTILE_STEP = C::CTILE_BYTES >> 4;
             constexpr uint32_t HALF_ROWS = (HW * 128) >> 4;  // rows HW.. of a column tile
-            uint32_t ct = 0;
+            uint32_t ct = 0;   // column tiles (slot ring)
+            uint32_t bt = 0;   // column tiles of d = 256 dv units (X buffers)
             int uw = 0;
             bool ok = true;
             auto kstep = [](int kk) -> uint32_t {
@@ -835,6 +840,32 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             // that half's P / dS only after the accumulation reading them was
             // issued; UMMAs of one thread execute in issue order. With whole-
             // tile X / Y (TILE_XY): XY(c) | z_0 | ACC_0(c) | z_1 | ACC_1(c) XY(c+1).
+            // d = 256 dv unit: X of the tile in slot sl into X buffer b (TMEM
+            // columns X_COL + 64 b; a dv unit computes no Y), and the dv
+            // accumulation over that buffer's P
+            auto issue_x_buf = [&](int sl, uint32_t b) {
+                constexpr uint32_t IDESC_XYT = idesc_bf16(128, C::CR, false);
+                const uint32_t c1 = slot_lo + sl * SLOT_STEP;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    if (!do_x) break;
+                    umma_ts_lh(tmem + X_COL + C::CR * b, tmem + A_COL + 8 * kk, c1 + kstep_c(kk),
+                               HI, IDESC_XYT, kk != 0);
+                }
+                umma_commit(&xb_full[b]);
+            };
+            auto issue_acc_buf = [&](int sl, int h, uint32_t b, bool first) {
+                const uint32_t c2_mn = slot_lo_mn + sl * SLOT_STEP + CTILE_STEP;
+                constexpr int KS = HW / 16;
+#pragma unroll
+                for (int k4 = 0; k4 < KS; ++k4) {
+                    if (!do_x) break;
+                    const int kk = KS * h + k4;
+                    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                    umma_ts_lh(tmem + 0, tmem + X_COL + C::CR * b + HW * h + 8 * k4,
+                               c2_mn + kk * ((16 * 128) >> 4), HI, IDESC_ACC, acc);
+                }
+            };
             for (int r = 0; ok && r * G < num_units; ++r) {
                 const int u = bw_sched(r, cta, G);
                 if (u >= num_units) continue;
@@ -848,6 +879,54 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (!ok) break;
                 }
                 tc_fence_after();
+                if (AT && KV && U.dh == 0) {
+                    // dv unit, X double-buffered: X(c+1) runs while the
+                    // elementwise warps work on tile c; X(c+2) goes into
+                    // tile c's buffer once the accumulation over it is issued
+                    ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_x_buf(ct & 1, bt & 1);
+                    if (U.ncols > 1) {
+                        ok = mbar_wait(&c_full[(ct + 1) & 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
+                                       SITE_BW_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_x_buf((ct + 1) & 1, (bt + 1) & 1);
+                    }
+                    for (int c = 0; c < U.ncols; ++c) {
+                        const int sl = ct & 1;
+                        const uint32_t b = bt & 1;
+                        ok = mbar_wait(&z_full[0], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                        if (!ok) break;
+                        if (c == 0 && uw > 0) {
+                            ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim,
+                                           SITE_BW_MMA_ACC);
+                            if (!ok) break;
+                        }
+                        tc_fence_after();
+                        issue_acc_buf(sl, 0, b, c == 0);
+                        ok = mbar_wait(&z_full[1], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_acc_buf(sl, 1, b, false);
+                        umma_commit(&c_empty[sl]);
+                        if (c + 2 < U.ncols) {  // tile c+2 is in slot sl again
+                            ok = mbar_wait(&c_full[sl], ((ct + 2) >> 1) & 1, abort_flag, lim,
+                                           SITE_BW_MMA);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_x_buf(sl, b);
+                        }
+                        ++ct;
+                        ++bt;
+                    }
+                    if (!ok) break;
+                    umma_commit(acc_done);
+                    umma_commit(r_empty);
+                    ++uw;
+                    continue;
+                }
                 ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
                 tc_fence_after();
@@ -916,7 +995,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const int r = (qd << 5) | lane;
         const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
         const int col0 = part * HW;
-        uint32_t ct = 0;
+        uint32_t ct = 0;   // column tiles (slot ring; z_full phases)
+        uint32_t xt = 0;   // column tiles on xy_full (all but d = 256 dv units)
+        uint32_t bt = 0;   // column tiles of d = 256 dv units (X buffers, xb_full)
         int uw = 0;
         bool ok = true;
         for (int rr = 0; ok && rr * G < num_units; ++rr) {
@@ -985,9 +1066,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ra_full);
             }
+            // d = 256 dv unit: X alternates between buffers at X_COL and Y_COL
+            const bool xbuf = AT && KV && U.dh == 0;
             for (int c = 0; c < U.ncols; ++c) {
                 const int sl = ct & 1;
-                ok = mbar_wait(&xy_full[part], ct & 1, abort_flag, lim, SITE_BW_EW);
+                const uint32_t x_col = xbuf ? X_COL + C::CR * (bt & 1) : X_COL;
+                if (xbuf)
+                    ok = mbar_wait(&xb_full[bt & 1], (bt >> 1) & 1, abort_flag, lim, SITE_BW_EW);
+                else
+                    ok = mbar_wait(&xy_full[part], xt & 1, abort_flag, lim, SITE_BW_EW);
                 if (KV && ok)  // the column tile's lse2 / D, copied with its operands
                     ok = mbar_wait(&c_full[sl], (ct >> 1) & 1, abort_flag, lim, SITE_BW_EW);
                 ok = __all_sync(0xffffffffu, ok);
@@ -1037,7 +1124,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     uint32_t xv[CHUNK], yv[CHUNK];
                     // d = 256 dv unit: P only (no Y; dS is not formed)
                     const bool want_y = !(AT && KV && U.dh == 0);
-                    bw_ld_async<CHUNK>(tmem + lane_addr + X_COL + cb, xv);
+                    bw_ld_async<CHUNK>(tmem + lane_addr + x_col + cb, xv);
                     if (want_y) {
                         bw_ld_async<CHUNK>(tmem + lane_addr + Y_COL + cb, yv);
                     } else {
@@ -1184,7 +1271,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (KV) {
                         // d = 256: the dv unit needs P^T only, the dk unit dS^T only
                         if (!AT || U.dh == 0)
-                            bw_st<CHUNK / 2>(tmem + lane_addr + X_COL + zc, pp);  // P^T
+                            bw_st<CHUNK / 2>(tmem + lane_addr + x_col + zc, pp);  // P^T
                         if (!AT || U.dh == 1)
                             bw_st<CHUNK / 2>(tmem + lane_addr + Y_COL + zc, pd);  // dS^T
                     } else {
@@ -1196,6 +1283,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&z_full[part]);
                 ++ct;
+                if (xbuf) ++bt; else ++xt;
             }
             if (!ok) break;
             // ---- epilogue: accumulators -> bf16 gradients
