@@ -24,8 +24,10 @@
 //   bwd_sm100<D, BW_Q>   one unit = 64 query positions x 2 heads: q and dout
 //                 stay, the CK-key tiles stream; X = q K^T, Y = dout V^T,
 //                 dq += dS K.
-// Column tiles are 128 rows for d <= 128 and 64 rows at d = 256 (BwCfg).
-// TMEM (512 columns), d <= 128: accumulators at 0..255, X at 256, Y at 384.
+// Column tiles are 64 rows (BwCfg): 32 positions x 2 heads, or 64 keys.
+// TMEM (512 columns), d <= 128: accumulators at 0..2d-1; X and Y double-
+// buffered, buffer b at 256 + 128 b (X) and 320 + 128 b (Y), so that the X / Y
+// of the next column tiles run while the elementwise warps work on this one.
 // d = 256: one 256-column accumulator at 0, one resident operand held in TMEM
 // at 256..383 (read by the UMMAs as their A operand, so its bytes never cross
 // shared memory again), X at 384 and Y at 448. The dk/dv kernel then runs
@@ -44,7 +46,7 @@ constexpr int BW_THREADS = 352;          // 8 elementwise warps, producer, 2 UMM
 constexpr int BW_EW_THREADS = 256;
 constexpr int BW_WARP_PRODUCER = 8;
 constexpr int BW_WARP_MMA = 9;           // issuer 0: X and the accumulation reading X; TMEM owner
-constexpr int BW_WARP_MMA2 = 10;         // issuer 1 (d = 256): Y and the accumulation reading Y
+constexpr int BW_WARP_MMA2 = 10;         // issuer 1: Y and the accumulation reading Y
 constexpr int BW_QPOS = 64;              // query positions per column/row tile (x 2 heads)
 constexpr int BW_KEYS = 128;             // keys per tile
 constexpr int BW_X_COL = 256;
@@ -53,41 +55,50 @@ constexpr uint32_t BW_TMEM_COLS = 512;
 
 // Tile shapes per head size. The resident (row) tiles are always 128 rows:
 // 128 keys (KV mode) or 64 positions x 2 heads (Q mode). The streamed column
-// tiles are CR rows: CQ positions x 2 heads (KV) or CK keys (Q), split into
-// two halves of HW columns, one per column part of the elementwise warps. At
-// d = 256 the column tiles shrink to 32 rows so that two slots still fit
-// next to the 128 KB resident pair, and the dk/dv kernel splits d into two
-// halves (DSPLIT units per key tile) so that its accumulators fit TMEM.
+// tiles are CR = 64 rows: CQ = 32 positions x 2 heads (KV) or CK = 64 keys
+// (Q), split into two halves of HW columns, one per column part of the
+// elementwise warps. X and Y are whole-tile N = 64 UMMAs issued by two
+// threads: one thread issues a tcgen05.mma only about every 67 cycles, which
+// is more than the math of an M = 128, N = 64, K = 16 product (32 cycles).
+// d <= 128: K and V (or q and dout) stay in shared memory, four slots of
+// column tiles stream, and X / Y are double-buffered in TMEM. d = 256: one
+// resident operand lives in TMEM (see the file header), two slots stream, and
+// the dk/dv kernel splits each key tile into a dv and a dk unit (DSPLIT) so
+// that its accumulator fits TMEM; only the dv units double-buffer X.
 template <int D>
 struct BwCfg {
     static_assert(D == 64 || D == 128 || D == 256, "backward kernels: d = 64, 128, 256");
-    // d = 256: one resident operand in TMEM instead of shared memory (see the
-    // file header), which leaves room for 64-row column tiles
     static constexpr bool A_TMEM = D == 256;
-    static constexpr int CQ = D == 256 ? 32 : BW_QPOS;  // KV column tile: positions per head
-    static constexpr int CK = D == 256 ? 64 : BW_KEYS;  // Q column tile: keys
+    static constexpr bool DB = !A_TMEM;                  // X / Y double-buffered for every unit
+    static constexpr int CQ = 32;                        // KV column tile: positions per head
+    static constexpr int CK = 64;                        // Q column tile: keys
     static constexpr int CR = 2 * CQ;                    // column tile rows (both modes)
     static_assert(CR == CK, "column tiles of both modes have CR rows");
     static constexpr int HW = CR / 2;                    // columns per half (per warp part)
     static constexpr int CHUNK = HW < 32 ? HW : 32;      // columns per TMEM round trip
     static constexpr int DSPLIT_KV = D == 256 ? 2 : 1;   // dk/dv kernel: units per key tile
     static constexpr int RES_TILES = A_TMEM ? 1 : 2;     // resident tiles in shared memory
-    // UMMA issuing threads: two at d = 256 (measured 7-8% faster); at d <= 128
-    // a second issuer measured 4-6% slower than one issuing everything in the
-    // X / Y / accumulation order of the column-half pipeline
-    static constexpr int ISSUERS = A_TMEM ? 2 : 1;
+    static constexpr int ISSUERS = 2;                    // UMMA issuing threads
+    static constexpr int NSLOT = A_TMEM ? 2 : 4;         // column-tile slots
     static constexpr int TILE_BYTES = 128 * D * 2;       // one 128-row resident tile
     static constexpr int CTILE_BYTES = CR * D * 2;       // one streamed column tile
     static constexpr int VEC_BYTES = 1024;               // -lse2, -D of the tile's query rows
     static constexpr int VEC_TX = 2 * CR * 4;            //   (bytes copied: CR rows, two arrays)
     static constexpr int SLOT_BYTES = 2 * CTILE_BYTES + VEC_BYTES;
     static_assert(SLOT_BYTES % 1024 == 0 && VEC_TX <= VEC_BYTES, "slot layout");
-    static constexpr int SMEM_TILES = RES_TILES * TILE_BYTES + 2 * SLOT_BYTES;  // R1 (R2), 2 slots
+    static constexpr int SMEM_TILES = RES_TILES * TILE_BYTES + NSLOT * SLOT_BYTES;
     // TMEM columns: accumulators at 0, the resident A operand (d = 256), X, Y
     static constexpr uint32_t A_COL = 256;
     static constexpr uint32_t X_COL = A_TMEM ? 384 : BW_X_COL;
     static constexpr uint32_t Y_COL = A_TMEM ? 448 : BW_Y_COL;
+    // double buffers: X of buffer b at XB0 + XB_STEP b, Y (d <= 128) at YB0 + XB_STEP b
+    // (d = 256 dv units: X alternates between the X and Y columns)
+    static constexpr uint32_t XB0 = A_TMEM ? 384 : 256;
+    static constexpr uint32_t YB0 = A_TMEM ? 448 : 320;
+    static constexpr uint32_t XB_STEP = A_TMEM ? 64 : 128;
     static_assert(!A_TMEM || (X_COL + CR <= Y_COL && Y_COL + CR <= BW_TMEM_COLS), "TMEM columns");
+    static_assert(A_TMEM || (2 * D <= XB0 && YB0 + XB_STEP + CR <= BW_TMEM_COLS),
+                  "TMEM columns (double-buffered X / Y)");
     static constexpr int MAX_SEQ_TABLE = 1024;                  // varlen: sequences per launch
     // varlen: per-sequence work, sequences ranked by it, unit prefix in rank order
     static constexpr int VL_BYTES = 4 * (3 * MAX_SEQ_TABLE + 1);
@@ -467,24 +478,30 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     // units) or dout (Q); the other operand is in TMEM.
     uint8_t* sR1 = base;
     uint8_t* sR2 = base + C::TILE_BYTES;
-    uint8_t* sSlot = base + C::RES_TILES * C::TILE_BYTES;  // [2] x (C1, C2, lse2[CR], D[CR])
+    uint8_t* sSlot = base + C::RES_TILES * C::TILE_BYTES;  // [NSLOT] x (C1, C2, lse2[CR], D[CR])
+    constexpr int NS = C::NSLOT;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::SMEM_TILES);
     uint64_t* r_full = bars + 0;
     uint64_t* r_empty = bars + 1;
-    uint64_t* c_full = bars + 2;    // [2]
-    uint64_t* c_empty = bars + 4;   // [2]
-    // Column halves h = 0, 1 (columns HW h .. HW h + HW - 1 of X and Y, the
-    // column parts of the elementwise warps) run as a two-stage pipeline:
-    uint64_t* xy_full = bars + 6;   // [2] X and Y of half h of the current tile are in TMEM
-    uint64_t* z_full = bars + 8;    // [2] P / dS of half h written back (4 warp arrivals)
-    uint64_t* acc_done = bars + 10; // last accumulation of the unit completed
-    uint64_t* acc_free = bars + 11; // epilogue read the accumulators (8 warp arrivals)
-    uint64_t* drain = bars + 12;
-    uint64_t* ra_full = bars + 13;  // d = 256: the unit's TMEM-resident operand written (8 warps)
-    // d = 256 dv units: X double-buffered in the X and Y columns (a dv unit
-    // has no Y); xb_full[b] = X of the next tile of buffer b is in TMEM
-    uint64_t* xb_full = bars + 14;  // [2]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+    uint64_t* c_full = bars + 2;    // [NSLOT <= 4]
+    uint64_t* c_empty = bars + 6;   // [NSLOT <= 4]
+    // Single-buffered X / Y (d = 256 dk units and dq kernel), per column half
+    // h = 0, 1 (columns HW h .. HW h + HW - 1 of X and Y, the column parts of
+    // the elementwise warps):
+    uint64_t* xy_full = bars + 10;  // [2] X and Y of half h of the current tile are in TMEM
+    uint64_t* z_full = bars + 12;   // [2] P / dS of half h written back (4 warp arrivals)
+    uint64_t* acc_done = bars + 14; // last accumulation of the unit completed
+    uint64_t* acc_free = bars + 15; // epilogue read the accumulators (8 warp arrivals)
+    uint64_t* drain = bars + 16;
+    uint64_t* ra_full = bars + 17;  // d = 256: the unit's TMEM-resident operand written (8 warps)
+    // Double-buffered X / Y (every unit at d <= 128, dv units at d = 256), by
+    // buffer b: xb_full[b] = X and Y of the buffer's next tile are in TMEM;
+    // zb_full[2 b + h] = its half h's P / dS written back (4 warp arrivals).
+    // Each completes one phase per tile of its buffer, so that neither side
+    // can run two phases ahead of a waiter.
+    uint64_t* xb_full = bars + 18;  // [2]
+    uint64_t* zb_full = bars + 20;  // [4]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     // varlen tables: cum[num_seqs + 1] (unit prefix in rank order), order[], work[]
     int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
@@ -496,7 +513,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(r_full, 1);
         mbar_init(r_empty, C::ISSUERS);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(&c_full[i], 1);
             mbar_init(&c_empty[i], C::ISSUERS);
         }
@@ -509,6 +526,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         mbar_init(drain, C::ISSUERS);
         mbar_init(ra_full, BW_EW_THREADS / 32);
         for (int b = 0; b < 2; ++b) mbar_init(&xb_full[b], C::ISSUERS);
+        for (int i = 0; i < 4; ++i) mbar_init(&zb_full[i], BW_EW_THREADS / 64);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -624,8 +642,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     }
                 }
                 for (int c = 0; c < U.ncols; ++c) {
-                    const int sl = ct & 1;
-                    ok = mbar_wait(&c_empty[sl], ((ct >> 1) & 1) ^ 1, abort_flag, lim,
+                    const int sl = ct % NS;
+                    ok = mbar_wait(&c_empty[sl], ((ct / NS) & 1) ^ 1, abort_flag, lim,
                                    SITE_BW_PROD);
                     if (!ok) break;
                     uint8_t* slot = sSlot + sl * C::SLOT_BYTES;
@@ -657,10 +675,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 ++uw;
             }
             // Drain: every copy issued lands before the CTA exits.
-            const uint32_t last = ct < 2u ? ct : 2u;
+            const uint32_t last = ct < uint32_t(NS) ? ct : uint32_t(NS);
             for (uint32_t i = 0; i < last; ++i) {
                 const uint32_t f = ct - 1 - i;
-                mbar_wait_drain(&c_full[f & 1], (f >> 1) & 1, lim);
+                mbar_wait_drain(&c_full[f % NS], (f / NS) & 1, lim);
             }
             if (uw > 0) mbar_wait_drain(r_full, (uw - 1) & 1, lim);
         }
@@ -669,19 +687,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     else if (warp == BW_WARP_MMA || (C::ISSUERS == 2 && warp == BW_WARP_MMA2)) {
         // ------------------------------------------------------------ UMMA issuers
         // One thread issues a tcgen05.mma about every 67 cycles, less than the
-        // math of the N = 64 UMMAs at d = 256, so there two threads in
-        // different warps share the issue: issuer 0 X and the accumulation
-        // that reads X (dv, or dq), issuer 1 Y and the accumulation that reads
-        // Y (dk). Neither writes what the other's UMMAs read, and each keeps
-        // its own order (X(c+1) after the accumulation over X(c)'s P, Y(c+1)
-        // after the one over Y(c)'s dS). Both take every wait; the barriers
-        // their commits complete count both. At d <= 128 issuer 0 issues all.
+        // math of the N = 64 UMMAs, so two threads in different warps share
+        // the issue: issuer 0 X and the accumulation that reads X (dv, or dq),
+        // issuer 1 Y and the accumulation that reads Y (dk). Neither writes
+        // what the other's UMMAs read, and each keeps its own order (the X of
+        // a buffer after the accumulation over that buffer's P, its Y after
+        // the one over its dS). Both take every wait; the barriers their
+        // commits complete count both.
         const int role = warp - BW_WARP_MMA;
         const bool do_x = role == 0;
         const bool do_y = C::ISSUERS == 2 ? role == 1 : role == 0;
         if (lane == 0) {
             constexpr int HW = C::HW;
-            constexpr uint32_t IDESC_XY = idesc_bf16(128, HW, false);  // one column half
             constexpr uint32_t IDESC_ACC = idesc_bf16(128, ACC_N, true);
             constexpr uint32_t HI = sdesc_hi(1024);  // SBO 1024 B (8 rows x 128 B)
             // K-major operands (contraction over d): 64-column blocks of rows x
@@ -696,9 +713,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const uint32_t slot_lo_mn = sdesc_lo(smem_u32(sSlot), C::CR * 128);
             constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
             constexpr uint32_t CTILE_STEP = C::CTILE_BYTES >> 4;
-            constexpr uint32_t HALF_ROWS = (HW * 128) >> 4;  // rows HW.. of a column tile
             uint32_t ct = 0;   // column tiles (slot ring)
-            uint32_t bt = 0;   // column tiles of d = 256 dv units (X buffers)
+            uint32_t bt = 0;   // column tiles with double-buffered X / Y (xb_full, zb_full)
+            uint32_t xt = 0;   // column tiles with single-buffered X / Y (xy_full, z_full)
             int uw = 0;
             bool ok = true;
             auto kstep = [](int kk) -> uint32_t {
@@ -707,60 +724,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             auto kstep_c = [](int kk) -> uint32_t {
                 return ((kk * 16) / 64) * CBLOCK + (((kk * 16) % 64) / 16) * 2;
             };
-            // X, Y columns [HW h, HW h + HW) of the tile in slot sl: rows HW h..
-            // of the column tiles (N = HW), contraction over d
-            auto issue_xy = [&](int sl, int h, int kind) {
-                const uint32_t c1 = slot_lo + sl * SLOT_STEP + h * HALF_ROWS;
-                const uint32_t c2 = c1 + CTILE_STEP;
-                if constexpr (AT) {
-                    // d = 256, A operands: KV dv unit X: K in TMEM; KV dk unit
-                    // X: K in R1, Y: V in TMEM; Q: X: q in TMEM, Y: dout in R1
-                    const bool x_tmem = !KV || kind == 0;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        if (!do_x) break;
-                        if (x_tmem)
-                            umma_ts_lh(tmem + X_COL + HW * h, tmem + A_COL + 8 * kk,
-                                       c1 + kstep_c(kk), HI, IDESC_XY, kk != 0);
-                        else
-                            umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk),
-                                       HI, IDESC_XY, kk != 0);
-                    }
-                    if (do_y && (!KV || kind == 1)) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            if (KV)
-                                umma_ts_lh(tmem + Y_COL + HW * h, tmem + A_COL + 8 * kk,
-                                           c2 + kstep_c(kk), HI, IDESC_XY, kk != 0);
-                            else
-                                umma_ss_lh(tmem + Y_COL + HW * h, r1_lo + kstep(kk),
-                                           c2 + kstep_c(kk), HI, IDESC_XY, kk != 0);
-                        }
-                    }
-                } else {
-                    if (do_x) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            umma_ss_lh(tmem + X_COL + HW * h, r1_lo + kstep(kk), c1 + kstep_c(kk),
-                                       HI, IDESC_XY, kk != 0);
-                    }
-                    if (do_y) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            umma_ss_lh(tmem + Y_COL + HW * h, r2_lo + kstep(kk), c2 + kstep_c(kk),
-                                       HI, IDESC_XY, kk != 0);
-                    }
-                }
-                umma_commit(&xy_full[h]);
-            };
-            // Both halves of the tile in slot sl as one UMMA pair (N = CR): fewer,
-            // wider UMMAs, and a resident A tile in shared memory is read once
-            // per tile instead of once per half.
+            // Single-buffered X / Y of the tile in slot sl (d = 256 dk units and
+            // the dq kernel), each one N = CR UMMA per k-step. A operands: KV dk
+            // unit X: K in R1, Y: V in TMEM; Q: X: q in TMEM, Y: dout in R1.
             auto issue_xy_tile = [&](int sl, int kind) {
                 constexpr uint32_t IDESC_XYT = idesc_bf16(128, C::CR, false);
                 const uint32_t c1 = slot_lo + sl * SLOT_STEP;
                 const uint32_t c2 = c1 + CTILE_STEP;
-                if constexpr (AT) {  // A operands as in issue_xy
+                if constexpr (AT) {
                     const bool x_tmem = !KV || kind == 0;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -800,12 +771,6 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 umma_commit(&xy_full[0]);
                 umma_commit(&xy_full[1]);
             };
-            // Whole-tile X / Y at d = 256 (N = 64): one thread issues a
-            // tcgen05.mma about every 67 cycles however small it is, so N = 32
-            // halves (16 cycles of math each at M = 128) leave the tensor pipe
-            // mostly idle; at d <= 128 the N = 64 halves and their overlap with
-            // the elementwise warps measured faster.
-            constexpr bool TILE_XY = HW < 32 || AT;
             // accumulations over the half's HW rows (K indices HW h ..): A = the
             // bf16 operand the half's warps wrote at columns HW h + 8 k4; B =
             // the streamed tile read MN-major (all D columns)
@@ -835,36 +800,74 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     }
                 }
             };
-            // Issue order per tile c (slot sl): XY_0(c) XY_1(c) | z_0 | ACC_0(c)
-            // XY_0(c+1) | z_1 | ACC_1(c) XY_1(c+1). A half's X / Y overwrite
-            // that half's P / dS only after the accumulation reading them was
-            // issued; UMMAs of one thread execute in issue order. With whole-
-            // tile X / Y (TILE_XY): XY(c) | z_0 | ACC_0(c) | z_1 | ACC_1(c) XY(c+1).
-            // d = 256 dv unit: X of the tile in slot sl into X buffer b (TMEM
-            // columns X_COL + 64 b; a dv unit computes no Y), and the dv
-            // accumulation over that buffer's P
-            auto issue_x_buf = [&](int sl, uint32_t b) {
+            // Single-buffered order per tile c: XY(c) | z_0 | ACC_0(c) | z_1 |
+            // ACC_1(c) XY(c+1): X / Y overwrite P / dS only after the
+            // accumulation reading them was issued, and UMMAs of one thread
+            // execute in issue order. Double-buffered: X / Y of tile c into buffer b = c & 1, the
+            // accumulation over buffer b, then X / Y of tile c+2 into it again,
+            // so that X / Y(c+1) run while the elementwise warps work on tile c.
+            // X / Y of the tile in slot sl into buffer b (d = 256 dv units: X
+            // only, K in TMEM)
+            auto issue_xy_buf = [&](int sl, uint32_t b) {
                 constexpr uint32_t IDESC_XYT = idesc_bf16(128, C::CR, false);
                 const uint32_t c1 = slot_lo + sl * SLOT_STEP;
+                const uint32_t c2 = c1 + CTILE_STEP;
+                const uint32_t xc = C::XB0 + C::XB_STEP * b, yc = C::YB0 + C::XB_STEP * b;
+                if constexpr (AT) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    if (!do_x) break;
-                    umma_ts_lh(tmem + X_COL + C::CR * b, tmem + A_COL + 8 * kk, c1 + kstep_c(kk),
-                               HI, IDESC_XYT, kk != 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        if (!do_x) break;
+                        umma_ts_lh(tmem + xc, tmem + A_COL + 8 * kk, c1 + kstep_c(kk), HI,
+                                   IDESC_XYT, kk != 0);
+                    }
+                } else {
+                    if (do_x) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lh(tmem + xc, r1_lo + kstep(kk), c1 + kstep_c(kk), HI,
+                                       IDESC_XYT, kk != 0);
+                    }
+                    if (do_y) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lh(tmem + yc, r2_lo + kstep(kk), c2 + kstep_c(kk), HI,
+                                       IDESC_XYT, kk != 0);
+                    }
                 }
                 umma_commit(&xb_full[b]);
             };
+            // accumulations over half h of buffer b: dv (issuer 0, P^T at X) and
+            // dk (issuer 1, dS^T at Y) in KV mode, dq (issuer 0, dS at X) in Q
+            // mode; d = 256 dv units: dv only
             auto issue_acc_buf = [&](int sl, int h, uint32_t b, bool first) {
-                const uint32_t c2_mn = slot_lo_mn + sl * SLOT_STEP + CTILE_STEP;
+                const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
+                const uint32_t c2_mn = c1_mn + CTILE_STEP;
+                const uint32_t xc = C::XB0 + C::XB_STEP * b, yc = C::YB0 + C::XB_STEP * b;
                 constexpr int KS = HW / 16;
 #pragma unroll
                 for (int k4 = 0; k4 < KS; ++k4) {
-                    if (!do_x) break;
                     const int kk = KS * h + k4;
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    umma_ts_lh(tmem + 0, tmem + X_COL + C::CR * b + HW * h + 8 * k4,
-                               c2_mn + kk * ((16 * 128) >> 4), HI, IDESC_ACC, acc);
+                    const uint32_t bstep = kk * ((16 * 128) >> 4);
+                    const uint32_t zc = HW * h + 8 * k4;
+                    if (KV) {
+                        if (do_x)
+                            umma_ts_lh(tmem + 0, tmem + xc + zc, c2_mn + bstep, HI, IDESC_ACC, acc);
+                        if (do_y && !AT)
+                            umma_ts_lh(tmem + ACC_N, tmem + yc + zc, c1_mn + bstep, HI, IDESC_ACC,
+                                       acc);
+                    } else if (do_x) {
+                        umma_ts_lh(tmem + 0, tmem + xc + zc, c1_mn + bstep, HI, IDESC_ACC, acc);
+                    }
                 }
+            };
+            // X / Y of column tile t (slot ring position t) into buffer b
+            auto load_xy_buf = [&](uint32_t t, uint32_t b) -> bool {
+                if (!mbar_wait(&c_full[t % NS], (t / NS) & 1, abort_flag, lim, SITE_BW_MMA))
+                    return false;
+                tc_fence_after();
+                issue_xy_buf(static_cast<int>(t % NS), b);
+                return true;
             };
             for (int r = 0; ok && r * G < num_units; ++r) {
                 const int u = bw_sched(r, cta, G);
@@ -879,25 +882,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (!ok) break;
                 }
                 tc_fence_after();
-                if (AT && KV && U.dh == 0) {
-                    // dv unit, X double-buffered: X(c+1) runs while the
-                    // elementwise warps work on tile c; X(c+2) goes into
-                    // tile c's buffer once the accumulation over it is issued
-                    ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
+                if (C::DB || (KV && U.dh == 0)) {
+                    // double-buffered X / Y (d = 256: dv units, X only)
+                    ok = load_xy_buf(ct, bt & 1);
+                    if (ok && U.ncols > 1) ok = load_xy_buf(ct + 1, (bt + 1) & 1);
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_x_buf(ct & 1, bt & 1);
-                    if (U.ncols > 1) {
-                        ok = mbar_wait(&c_full[(ct + 1) & 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
-                                       SITE_BW_MMA);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_x_buf((ct + 1) & 1, (bt + 1) & 1);
-                    }
                     for (int c = 0; c < U.ncols; ++c) {
-                        const int sl = ct & 1;
+                        const int sl = static_cast<int>(ct % NS);
                         const uint32_t b = bt & 1;
-                        ok = mbar_wait(&z_full[0], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                        ok = mbar_wait(&zb_full[2 * b], (bt >> 1) & 1, abort_flag, lim,
+                                       SITE_BW_MMA_Z);
                         if (!ok) break;
                         if (c == 0 && uw > 0) {
                             ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim,
@@ -906,17 +900,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         }
                         tc_fence_after();
                         issue_acc_buf(sl, 0, b, c == 0);
-                        ok = mbar_wait(&z_full[1], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                        ok = mbar_wait(&zb_full[2 * b + 1], (bt >> 1) & 1, abort_flag, lim,
+                                       SITE_BW_MMA_Z);
                         if (!ok) break;
                         tc_fence_after();
                         issue_acc_buf(sl, 1, b, false);
                         umma_commit(&c_empty[sl]);
-                        if (c + 2 < U.ncols) {  // tile c+2 is in slot sl again
-                            ok = mbar_wait(&c_full[sl], ((ct + 2) >> 1) & 1, abort_flag, lim,
-                                           SITE_BW_MMA);
+                        if (c + 2 < U.ncols) {  // tile c+2 goes into buffer b again
+                            ok = load_xy_buf(ct + 2, b);
                             if (!ok) break;
-                            tc_fence_after();
-                            issue_x_buf(sl, b);
                         }
                         ++ct;
                         ++bt;
@@ -927,19 +919,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     ++uw;
                     continue;
                 }
-                ok = mbar_wait(&c_full[ct & 1], (ct >> 1) & 1, abort_flag, lim, SITE_BW_MMA);
+                if constexpr (!AT) continue;  // (every unit above)
+                // single-buffered X / Y (d = 256 dk units and dq kernel)
+                ok = mbar_wait(&c_full[ct % NS], (ct / NS) & 1, abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
                 tc_fence_after();
-                if constexpr (TILE_XY) {
-                    issue_xy_tile(ct & 1, U.dh);
-                } else {
-                    issue_xy(ct & 1, 0, U.dh);
-                    issue_xy(ct & 1, 1, U.dh);
-                }
+                issue_xy_tile(static_cast<int>(ct % NS), U.dh);
                 for (int c = 0; c < U.ncols; ++c) {
-                    const int sl = ct & 1;
-                    const bool next = c + 1 < U.ncols;
-                    ok = mbar_wait(&z_full[0], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                    const int sl = static_cast<int>(ct % NS);
+                    ok = mbar_wait(&z_full[0], xt & 1, abort_flag, lim, SITE_BW_MMA_Z);
                     if (!ok) break;
                     if (c == 0 && uw > 0) {
                         ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim, SITE_BW_MMA_ACC);
@@ -947,30 +935,20 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     }
                     tc_fence_after();
                     issue_acc(sl, 0, U.dh, c == 0);
-                    if (next && !TILE_XY) {
-                        ok = mbar_wait(&c_full[sl ^ 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
-                                       SITE_BW_MMA);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_xy(sl ^ 1, 0, U.dh);
-                    }
-                    ok = mbar_wait(&z_full[1], ct & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                    ok = mbar_wait(&z_full[1], xt & 1, abort_flag, lim, SITE_BW_MMA_Z);
                     if (!ok) break;
                     tc_fence_after();
                     issue_acc(sl, 1, U.dh, false);
                     umma_commit(&c_empty[sl]);
-                    if (next) {
-                        if constexpr (TILE_XY) {
-                            ok = mbar_wait(&c_full[sl ^ 1], ((ct + 1) >> 1) & 1, abort_flag, lim,
-                                           SITE_BW_MMA);
-                            if (!ok) break;
-                            tc_fence_after();
-                            issue_xy_tile(sl ^ 1, U.dh);
-                        } else {
-                            issue_xy(sl ^ 1, 1, U.dh);
-                        }
+                    if (c + 1 < U.ncols) {
+                        ok = mbar_wait(&c_full[(ct + 1) % NS], ((ct + 1) / NS) & 1, abort_flag,
+                                       lim, SITE_BW_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_xy_tile(static_cast<int>((ct + 1) % NS), U.dh);
                     }
                     ++ct;
+                    ++xt;
                 }
                 if (!ok) break;
                 umma_commit(acc_done);
@@ -985,7 +963,6 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     }
     else if (warp < BW_WARP_PRODUCER) {
         // ------------------------------------------------------------ elementwise + epilogue
-        // (warps 0-7 only: warp 10 is idle when one thread issues the UMMAs)
         // Warps w and w+4 share TMEM lane quadrant w%4 (rows 32(w%4)..+31);
         // warp w takes columns 0..HW-1 of X and Y, warp w+4 columns HW..2HW-1.
         // KV mode: row = key, column = query row (head 2g + column/CQ). Q mode:
@@ -995,9 +972,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const int r = (qd << 5) | lane;
         const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
         const int col0 = part * HW;
-        uint32_t ct = 0;   // column tiles (slot ring; z_full phases)
-        uint32_t xt = 0;   // column tiles on xy_full (all but d = 256 dv units)
-        uint32_t bt = 0;   // column tiles of d = 256 dv units (X buffers, xb_full)
+        uint32_t ct = 0;   // column tiles (slot ring)
+        uint32_t xt = 0;   // column tiles with single-buffered X / Y (xy_full, z_full)
+        uint32_t bt = 0;   // column tiles with double-buffered X / Y (xb_full, zb_full)
         int uw = 0;
         bool ok = true;
         for (int rr = 0; ok && rr * G < num_units; ++rr) {
@@ -1066,17 +1043,20 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ra_full);
             }
-            // d = 256 dv unit: X alternates between buffers at X_COL and Y_COL
-            const bool xbuf = AT && KV && U.dh == 0;
+            // double-buffered X / Y (d <= 128; d = 256 dv units: X only, in
+            // the X and Y columns alternately)
+            const bool xbuf = C::DB || (KV && U.dh == 0);
             for (int c = 0; c < U.ncols; ++c) {
-                const int sl = ct & 1;
-                const uint32_t x_col = xbuf ? X_COL + C::CR * (bt & 1) : X_COL;
+                const int sl = static_cast<int>(ct % NS);
+                const uint32_t b = bt & 1;
+                const uint32_t x_col = xbuf ? C::XB0 + C::XB_STEP * b : X_COL;
+                const uint32_t y_col = xbuf ? C::YB0 + C::XB_STEP * b : Y_COL;
                 if (xbuf)
-                    ok = mbar_wait(&xb_full[bt & 1], (bt >> 1) & 1, abort_flag, lim, SITE_BW_EW);
+                    ok = mbar_wait(&xb_full[b], (bt >> 1) & 1, abort_flag, lim, SITE_BW_EW);
                 else
                     ok = mbar_wait(&xy_full[part], xt & 1, abort_flag, lim, SITE_BW_EW);
                 if (KV && ok)  // the column tile's lse2 / D, copied with its operands
-                    ok = mbar_wait(&c_full[sl], (ct >> 1) & 1, abort_flag, lim, SITE_BW_EW);
+                    ok = mbar_wait(&c_full[sl], (ct / NS) & 1, abort_flag, lim, SITE_BW_EW);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
@@ -1126,7 +1106,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     const bool want_y = !(AT && KV && U.dh == 0);
                     bw_ld_async<CHUNK>(tmem + lane_addr + x_col + cb, xv);
                     if (want_y) {
-                        bw_ld_async<CHUNK>(tmem + lane_addr + Y_COL + cb, yv);
+                        bw_ld_async<CHUNK>(tmem + lane_addr + y_col + cb, yv);
                     } else {
 #pragma unroll
                         for (int i = 0; i < CHUNK; ++i) yv[i] = 0u;
@@ -1273,15 +1253,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         if (!AT || U.dh == 0)
                             bw_st<CHUNK / 2>(tmem + lane_addr + x_col + zc, pp);  // P^T
                         if (!AT || U.dh == 1)
-                            bw_st<CHUNK / 2>(tmem + lane_addr + Y_COL + zc, pd);  // dS^T
+                            bw_st<CHUNK / 2>(tmem + lane_addr + y_col + zc, pd);  // dS^T
                     } else {
-                        bw_st<CHUNK / 2>(tmem + lane_addr + X_COL + zc, pd);  // dS
+                        bw_st<CHUNK / 2>(tmem + lane_addr + x_col + zc, pd);  // dS
                     }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&z_full[part]);
+                if (lane == 0) mbar_arrive(xbuf ? &zb_full[2 * b + part] : &z_full[part]);
                 ++ct;
                 if (xbuf) ++bt; else ++xt;
             }
