@@ -352,6 +352,27 @@ int noalloc_scratch(void** out) {
     return G2ATTN_OK;
 }
 
+// The gradients' series for tanh(u), u = alpha x / C, |u| <= 1/4: the same
+// window as the forward's fast path, with the coefficients of the Taylor
+// series (1, -1/3, 2/15, -17/315) times (alpha/C)^(2k+1) so that the kernels
+// evaluate it in powers of the raw accumulator x. Off when the smallest folded
+// coefficient is not a comfortably normal float.
+void fill_bwd_series(float query_scale, float softcap, g2::BwParams& P) {
+    g2::PfParams F{};
+    fill_poly(query_scale, softcap, F);
+    P.u_scale = F.u_scale;
+    P.poly_acc_max = F.poly_acc_max;
+    const float us = F.u_scale, us2 = us * us;
+    const float c[4] = {1.0f, -1.0f / 3.0f, 2.0f / 15.0f, -17.0f / 315.0f};
+    float pw = us;
+    for (int i = 0; i < 4; ++i) {
+        P.th_c[i] = c[i] * pw;
+        pw *= us2;
+    }
+    if (!(fabsf(P.th_c[3]) > 1e-30f) || !isfinite(P.th_c[3]) || !isfinite(P.th_c[0]))
+        P.poly_acc_max = 0.f;
+}
+
 // Backward: query-side positions padded to whole 64-position tiles in the
 // workspace (-lse*log2(e) and -D, fp32 each).
 long long bwd_tp(int T) { return (static_cast<long long>(T) + 63) / 64 * 64; }
@@ -528,12 +549,7 @@ int g2attn_prefill_varlen_backward(const void* q, const void* k, const void* v, 
     fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, has_cap);
     P.has_cap = has_cap;
     P.query_scale = query_scale;
-    {  // the same series window as the forward's fast path
-        g2::PfParams F{};
-        fill_poly(query_scale, softcap, F);
-        P.u_scale = F.u_scale;
-        P.poly_acc_max = F.poly_acc_max;
-    }
+    fill_bwd_series(query_scale, softcap, P);
     P.timeout_ns = wait_limit_ns();
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 64)
@@ -590,12 +606,7 @@ int g2attn_prefill_backward(const void* q, const void* k, const void* v, const v
     fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, has_cap);
     P.has_cap = has_cap;
     P.query_scale = query_scale;
-    {  // the same series window as the forward's fast path
-        g2::PfParams F{};
-        fill_poly(query_scale, softcap, F);
-        P.u_scale = F.u_scale;
-        P.poly_acc_max = F.poly_acc_max;
-    }
+    fill_bwd_series(query_scale, softcap, P);
     P.timeout_ns = wait_limit_ns();
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d == 64) return launch_backward<64>(q, k, v, out, lse, dout, P, st);

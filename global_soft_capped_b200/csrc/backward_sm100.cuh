@@ -42,11 +42,16 @@ namespace g2 {
 
 constexpr int BW_KV = 0;
 constexpr int BW_Q = 1;
-constexpr int BW_THREADS = 352;          // 8 elementwise warps, producer, 2 UMMA issuers
-constexpr int BW_EW_THREADS = 256;
-constexpr int BW_WARP_PRODUCER = 8;
-constexpr int BW_WARP_MMA = 9;           // issuer 0: X and the accumulation reading X; TMEM owner
-constexpr int BW_WARP_MMA2 = 10;         // issuer 1: Y and the accumulation reading Y
+// Elementwise warps: BW_NPART column parts x 4 TMEM lane quadrants. Their
+// per-tile work is bound by instruction issue, not latency: four parts (16
+// warps) measured 5% slower than two at d = 128 and d = 256.
+constexpr int BW_NPART = 2;
+constexpr int BW_EW_WARPS = 4 * BW_NPART;
+constexpr int BW_EW_THREADS = 32 * BW_EW_WARPS;
+constexpr int BW_WARP_PRODUCER = BW_EW_WARPS;
+constexpr int BW_WARP_MMA = BW_EW_WARPS + 1;   // issuer 0: X and the accumulation reading X; TMEM owner
+constexpr int BW_WARP_MMA2 = BW_EW_WARPS + 2;  // issuer 1: Y and the accumulation reading Y
+constexpr int BW_THREADS = 32 * (BW_EW_WARPS + 3);  // elementwise warps, producer, 2 UMMA issuers
 constexpr int BW_QPOS = 64;              // query positions per column/row tile (x 2 heads)
 constexpr int BW_KEYS = 128;             // keys per tile
 constexpr int BW_X_COL = 256;
@@ -56,7 +61,7 @@ constexpr uint32_t BW_TMEM_COLS = 512;
 // Tile shapes per head size. The resident (row) tiles are always 128 rows:
 // 128 keys (KV mode) or 64 positions x 2 heads (Q mode). The streamed column
 // tiles are CR = 64 rows: CQ = 32 positions x 2 heads (KV) or CK = 64 keys
-// (Q), split into two halves of HW columns, one per column part of the
+// (Q), split into BW_NPART parts of HW columns, one per column part of the
 // elementwise warps. X and Y are whole-tile N = 64 UMMAs issued by two
 // threads: one thread issues a tcgen05.mma only about every 67 cycles, which
 // is more than the math of an M = 128, N = 64, K = 16 product (32 cycles).
@@ -74,7 +79,7 @@ struct BwCfg {
     static constexpr int CK = 64;                        // Q column tile: keys
     static constexpr int CR = 2 * CQ;                    // column tile rows (both modes)
     static_assert(CR == CK, "column tiles of both modes have CR rows");
-    static constexpr int HW = CR / 2;                    // columns per half (per warp part)
+    static constexpr int HW = CR / BW_NPART;             // columns per warp part
     static constexpr int CHUNK = HW < 32 ? HW : 32;      // columns per TMEM round trip
     static constexpr int DSPLIT_KV = D == 256 ? 2 : 1;   // dk/dv kernel: units per key tile
     static constexpr int RES_TILES = A_TMEM ? 1 : 2;     // resident tiles in shared memory
@@ -135,6 +140,7 @@ struct BwParams {
     float scale_l2;     // alpha log2(e)
     float query_scale;
     float u_scale;       // alpha / C              (cap on)
+    float th_c[4];       // series of tanh(alpha x / C) in x: (alpha/C)^(2k+1) c_k (cap on)
     float poly_acc_max;  // largest |q.k| with |alpha q.k / C| <= 1/4 (0: series off)
     int has_cap;
     unsigned long long timeout_ns;
@@ -214,8 +220,8 @@ __device__ __forceinline__ int bw_row_tiles(int T, int S) {
 
 // Units. Dense: row tiles in the order of bw_tile_cols, then batch, then KV
 // head. Varlen: sequence by sequence, heaviest first (`order`, with the unit
-// prefix `cum` in that order), within a sequence as dense. The d-halves of a
-// key tile (dk/dv kernel at d = 256) are consecutive units.
+// prefix `cum` in that order), within a sequence as dense. The dv and dk
+// units of a key tile (dk/dv kernel at d = 256) are consecutive units.
 template <int D, int MODE>
 __device__ __forceinline__ void bw_unit(const BwParams& P, const int* cum, const int* order,
                                         int u, BwUnit& U) {
@@ -385,35 +391,41 @@ __device__ __forceinline__ void bw_load_tile(uint8_t* dst, const CUtensorMap* ma
     for (int c = 0; c < D / 64; ++c) tma_load_3d(dst + c * rows * 128, map, bar, c * 64, row, head);
 }
 
-// HALF (= D/2) accumulator columns of this thread's row, times f, as bf16 to
-// dst (when valid): all loads in flight before one wait.
-template <int HALF>
+// TMEM round trips of N columns (32 lanes x 32 bit): loads of 16 or 32
+// columns (complete with tmem_wait_ld, then bw_fence before use) and stores of
+// 8 or 16.
+template <int N>
+__device__ __forceinline__ void bw_ld_async(uint32_t taddr, uint32_t (&r)[N]);
+template <int N>
+__device__ __forceinline__ void bw_fence(uint32_t (&r)[N]);
+
+// NC accumulator columns of this thread's row (a multiple of 16), times f, as
+// bf16 to dst (when valid): all loads in flight before one wait.
+template <int NC>
 __device__ __forceinline__ void bw_store_acc(uint32_t taddr, __nv_bfloat16* dst, float f,
                                              bool valid) {
-    static_assert(HALF % 32 == 0, "accumulator chunks");
-    uint32_t v[HALF / 32][32];
+    constexpr int W = NC % 32 == 0 ? 32 : 16;  // columns per TMEM load
+    static_assert(NC % W == 0, "accumulator chunks");
+    uint32_t v[NC / W][W];
 #pragma unroll
-    for (int j = 0; j < HALF / 32; ++j) tmem_ld32_async(taddr + 32 * j, v[j]);
+    for (int j = 0; j < NC / W; ++j) bw_ld_async<W>(taddr + W * j, v[j]);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < HALF / 32; ++j) {
-        tmem_reg_fence(v[j]);
-        uint32_t pk[16];
+    for (int j = 0; j < NC / W; ++j) {
+        bw_fence<W>(v[j]);
+        uint32_t pk[W / 2];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < W / 2; ++i)
             pk[i] = pack_bf16x2(__uint_as_float(v[j][2 * i]) * f, __uint_as_float(v[j][2 * i + 1]) * f);
         if (valid) {
-            uint4* o = reinterpret_cast<uint4*>(dst + 32 * j);
+            uint4* o = reinterpret_cast<uint4*>(dst + W * j);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
+            for (int q4 = 0; q4 < W / 8; ++q4)
                 o[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
     }
 }
 
-// TMEM round trips of N columns (32 lanes x 32 bit): loads of 16 or 32
-// columns (complete with tmem_wait_ld, then bw_fence before use) and stores of
-// 8 or 16.
 template <int N>
 __device__ __forceinline__ void bw_ld_async(uint32_t taddr, uint32_t (&r)[N]) {
     static_assert(N == 16 || N == 32, "TMEM load width");
@@ -485,23 +497,23 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint64_t* r_empty = bars + 1;
     uint64_t* c_full = bars + 2;    // [NSLOT <= 4]
     uint64_t* c_empty = bars + 6;   // [NSLOT <= 4]
-    // Single-buffered X / Y (d = 256 dk units and dq kernel), per column half
-    // h = 0, 1 (columns HW h .. HW h + HW - 1 of X and Y, the column parts of
-    // the elementwise warps):
-    uint64_t* xy_full = bars + 10;  // [2] X and Y of half h of the current tile are in TMEM
-    uint64_t* z_full = bars + 12;   // [2] P / dS of half h written back (4 warp arrivals)
-    uint64_t* acc_done = bars + 14; // last accumulation of the unit completed
-    uint64_t* acc_free = bars + 15; // epilogue read the accumulators (8 warp arrivals)
-    uint64_t* drain = bars + 16;
-    uint64_t* ra_full = bars + 17;  // d = 256: the unit's TMEM-resident operand written (8 warps)
+    // Single-buffered X / Y (d = 256 dk units and dq kernel), per column part
+    // h (columns HW h .. HW h + HW - 1 of X and Y, the column parts of the
+    // elementwise warps):
+    uint64_t* xy_full = bars + 10;  // [NPART] X and Y of the current tile are in TMEM
+    uint64_t* z_full = bars + 14;   // [NPART] P / dS of part h written back (4 warp arrivals)
+    uint64_t* acc_done = bars + 18; // last accumulation of the unit completed
+    uint64_t* acc_free = bars + 19; // epilogue read the accumulators (one arrival per warp)
+    uint64_t* drain = bars + 20;
+    uint64_t* ra_full = bars + 21;  // d = 256: the unit's TMEM-resident operand written
     // Double-buffered X / Y (every unit at d <= 128, dv units at d = 256), by
     // buffer b: xb_full[b] = X and Y of the buffer's next tile are in TMEM;
-    // zb_full[2 b + h] = its half h's P / dS written back (4 warp arrivals).
-    // Each completes one phase per tile of its buffer, so that neither side
-    // can run two phases ahead of a waiter.
-    uint64_t* xb_full = bars + 18;  // [2]
-    uint64_t* zb_full = bars + 20;  // [4]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
+    // zb_full[NPART b + h] = its part h's P / dS written back (4 warp
+    // arrivals). Each completes one phase per tile of its buffer, so that
+    // neither side can run two phases ahead of a waiter.
+    uint64_t* xb_full = bars + 22;  // [2]
+    uint64_t* zb_full = bars + 24;  // [2 NPART]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24 + 2 * BW_NPART);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     // varlen tables: cum[num_seqs + 1] (unit prefix in rank order), order[], work[]
     int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
@@ -517,16 +529,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             mbar_init(&c_full[i], 1);
             mbar_init(&c_empty[i], C::ISSUERS);
         }
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < BW_NPART; ++h) {
             mbar_init(&xy_full[h], C::ISSUERS);
-            mbar_init(&z_full[h], BW_EW_THREADS / 64);
+            mbar_init(&z_full[h], 4);  // the part's warp in each lane quadrant
         }
         mbar_init(acc_done, C::ISSUERS);
         mbar_init(acc_free, BW_EW_THREADS / 32);
         mbar_init(drain, C::ISSUERS);
         mbar_init(ra_full, BW_EW_THREADS / 32);
         for (int b = 0; b < 2; ++b) mbar_init(&xb_full[b], C::ISSUERS);
-        for (int i = 0; i < 4; ++i) mbar_init(&zb_full[i], BW_EW_THREADS / 64);
+        for (int i = 0; i < 2 * BW_NPART; ++i) mbar_init(&zb_full[i], 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -768,16 +780,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                        IDESC_XYT, kk != 0);
                     }
                 }
-                umma_commit(&xy_full[0]);
-                umma_commit(&xy_full[1]);
+#pragma unroll
+                for (int h = 0; h < BW_NPART; ++h) umma_commit(&xy_full[h]);
             };
-            // accumulations over the half's HW rows (K indices HW h ..): A = the
-            // bf16 operand the half's warps wrote at columns HW h + 8 k4; B =
+            // accumulations over part h's HW rows (K indices HW h ..): A = the
+            // bf16 operand the part's warps wrote at columns HW h + 8 k4; B =
             // the streamed tile read MN-major (all D columns)
             auto issue_acc = [&](int sl, int h, int kind, bool first) {
                 const uint32_t c1_mn = slot_lo_mn + sl * SLOT_STEP;
                 const uint32_t c2_mn = c1_mn + CTILE_STEP;
-                constexpr int KS = HW / 16;  // K steps per half
+                constexpr int KS = HW / 16;  // K steps per part
 #pragma unroll
                 for (int k4 = 0; k4 < KS; ++k4) {
                     const int kk = KS * h + k4;
@@ -801,11 +813,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
             };
             // Single-buffered order per tile c: XY(c) | z_0 | ACC_0(c) | z_1 |
-            // ACC_1(c) XY(c+1): X / Y overwrite P / dS only after the
+            // ACC_1(c) | ... XY(c+1): X / Y overwrite P / dS only after the
             // accumulation reading them was issued, and UMMAs of one thread
-            // execute in issue order. Double-buffered: X / Y of tile c into buffer b = c & 1, the
-            // accumulation over buffer b, then X / Y of tile c+2 into it again,
-            // so that X / Y(c+1) run while the elementwise warps work on tile c.
+            // execute in issue order. Double-buffered: X / Y of tile c into
+            // buffer b = c & 1, the accumulation over buffer b, then X / Y of
+            // tile c+2 into it again, so that X / Y(c+1) run while the
+            // elementwise warps work on tile c.
             // X / Y of the tile in slot sl into buffer b (d = 256 dv units: X
             // only, K in TMEM)
             auto issue_xy_buf = [&](int sl, uint32_t b) {
@@ -836,7 +849,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
                 umma_commit(&xb_full[b]);
             };
-            // accumulations over half h of buffer b: dv (issuer 0, P^T at X) and
+            // accumulations over part h of buffer b: dv (issuer 0, P^T at X) and
             // dk (issuer 1, dS^T at Y) in KV mode, dq (issuer 0, dS at X) in Q
             // mode; d = 256 dv units: dv only
             auto issue_acc_buf = [&](int sl, int h, uint32_t b, bool first) {
@@ -890,21 +903,20 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     for (int c = 0; c < U.ncols; ++c) {
                         const int sl = static_cast<int>(ct % NS);
                         const uint32_t b = bt & 1;
-                        ok = mbar_wait(&zb_full[2 * b], (bt >> 1) & 1, abort_flag, lim,
-                                       SITE_BW_MMA_Z);
-                        if (!ok) break;
                         if (c == 0 && uw > 0) {
                             ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim,
                                            SITE_BW_MMA_ACC);
                             if (!ok) break;
                         }
-                        tc_fence_after();
-                        issue_acc_buf(sl, 0, b, c == 0);
-                        ok = mbar_wait(&zb_full[2 * b + 1], (bt >> 1) & 1, abort_flag, lim,
-                                       SITE_BW_MMA_Z);
+#pragma unroll
+                        for (int h = 0; h < BW_NPART; ++h) {
+                            ok = mbar_wait(&zb_full[BW_NPART * b + h], (bt >> 1) & 1, abort_flag,
+                                           lim, SITE_BW_MMA_Z);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_acc_buf(sl, h, b, c == 0);
+                        }
                         if (!ok) break;
-                        tc_fence_after();
-                        issue_acc_buf(sl, 1, b, false);
                         umma_commit(&c_empty[sl]);
                         if (c + 2 < U.ncols) {  // tile c+2 goes into buffer b again
                             ok = load_xy_buf(ct + 2, b);
@@ -927,18 +939,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 issue_xy_tile(static_cast<int>(ct % NS), U.dh);
                 for (int c = 0; c < U.ncols; ++c) {
                     const int sl = static_cast<int>(ct % NS);
-                    ok = mbar_wait(&z_full[0], xt & 1, abort_flag, lim, SITE_BW_MMA_Z);
-                    if (!ok) break;
                     if (c == 0 && uw > 0) {
                         ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim, SITE_BW_MMA_ACC);
                         if (!ok) break;
                     }
-                    tc_fence_after();
-                    issue_acc(sl, 0, U.dh, c == 0);
-                    ok = mbar_wait(&z_full[1], xt & 1, abort_flag, lim, SITE_BW_MMA_Z);
+#pragma unroll
+                    for (int h = 0; h < BW_NPART; ++h) {
+                        ok = mbar_wait(&z_full[h], xt & 1, abort_flag, lim, SITE_BW_MMA_Z);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_acc(sl, h, U.dh, c == 0);
+                    }
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_acc(sl, 1, U.dh, false);
                     umma_commit(&c_empty[sl]);
                     if (c + 1 < U.ncols) {
                         ok = mbar_wait(&c_full[(ct + 1) % NS], ((ct + 1) / NS) & 1, abort_flag,
@@ -963,8 +975,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     }
     else if (warp < BW_WARP_PRODUCER) {
         // ------------------------------------------------------------ elementwise + epilogue
-        // Warps w and w+4 share TMEM lane quadrant w%4 (rows 32(w%4)..+31);
-        // warp w takes columns 0..HW-1 of X and Y, warp w+4 columns HW..2HW-1.
+        // Warps w, w+4, ... share TMEM lane quadrant w%4 (rows 32(w%4)..+31);
+        // warp w takes the columns HW (w/4) .. HW (w/4) + HW - 1 of X and Y.
         // KV mode: row = key, column = query row (head 2g + column/CQ). Q mode:
         // row = query row (head 2g + row/64), column = key.
         constexpr int HW = C::HW, CQ = C::CQ, CHUNK = C::CHUNK;
@@ -987,9 +999,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 // query sees at least its own key)
                 if (KV && r < U.rvalid) {
                     const size_t row = (static_cast<size_t>(U.kbase) + U.row0 + r) * P.Hkv + U.g;
-                    const size_t c0 = row * D + part * (D / 2);
+                    const size_t c0 = row * D + part * (D / BW_NPART);
 #pragma unroll
-                    for (int c = 0; c < D / 2; c += 8) {
+                    for (int c = 0; c < D / BW_NPART; c += 8) {
                         if (!AT || U.dh == 0)
                             *reinterpret_cast<uint4*>(P.dv + c0 + c) = make_uint4(0u, 0u, 0u, 0u);
                         if (!AT || U.dh == 1)
@@ -1011,8 +1023,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const int key_row = U.row0 + r;  // KV mode
             if constexpr (AT) {
                 // This thread's row of the unit's TMEM-resident operand (KV dv
-                // unit: K, dk unit: V; Q: q), its part's half of the d columns
-                // as bf16 pairs at TMEM columns A_COL + 64 part ..; rows past
+                // unit: K, dk unit: V; Q: q), its part's D / NPART of the d
+                // columns as bf16 pairs at TMEM columns A_COL + (D / NPART / 2)
+                // part ..; rows past
                 // the sequence are zeros. The previous unit's UMMAs, which read
                 // these columns, completed before its epilogue (acc_done).
                 const __nv_bfloat16* src = nullptr;
@@ -1023,20 +1036,22 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 } else if (t_row < U.T) {
                     src = P.q + ((static_cast<size_t>(U.qbase) + t_row) * P.H + 2 * U.g + hl_row) * D;
                 }
+                constexpr int PD = D / BW_NPART;  // d values of this part
+                static_assert(PD % 64 == 0, "resident operand: 32 TMEM columns per store");
 #pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {  // 2 x 32 columns = 128 d values
+                for (int hc = 0; hc < PD / 64; ++hc) {  // 32 columns = 64 d values
                     uint32_t w[32];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         uint4 x = make_uint4(0u, 0u, 0u, 0u);
                         if (src)
-                            x = __ldg(reinterpret_cast<const uint4*>(src + part * (D / 2) + 64 * hc) + i);
+                            x = __ldg(reinterpret_cast<const uint4*>(src + part * PD + 64 * hc) + i);
                         w[4 * i] = x.x;
                         w[4 * i + 1] = x.y;
                         w[4 * i + 2] = x.z;
                         w[4 * i + 3] = x.w;
                     }
-                    tmem_st32(tmem + lane_addr + A_COL + 64 * part + 32 * hc, w);
+                    tmem_st32(tmem + lane_addr + A_COL + (PD / 2) * part + 32 * hc, w);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -1115,10 +1130,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     bw_fence<CHUNK>(xv);
                     bw_fence<CHUNK>(yv);
                     // the cap's tanh by series when every |u| of this warp's chunk <= 1/4
-                    float amax = 0.f;
+                    float am[2] = {0.f, 0.f};
 #pragma unroll
-                    for (int i = 0; i < CHUNK; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(xv[i])));
-                    const bool poly = __all_sync(0xffffffffu, amax <= P.poly_acc_max);
+                    for (int i = 0; i < CHUNK; i += 2)
+                        am[(i >> 1) & 1] = fmax3f(am[(i >> 1) & 1], fabsf(__uint_as_float(xv[i])),
+                                                  fabsf(__uint_as_float(xv[i + 1])));
+                    const bool poly =
+                        __all_sync(0xffffffffu, fmaxf(am[0], am[1]) <= P.poly_acc_max);
                     uint32_t pp[CHUNK / 2], pd[CHUNK / 2];
                     // -lse2 / -D of the column pair i, i+1 (KV: per column, from
                     // the slot; Q: this row's)
@@ -1131,11 +1149,23 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             nd = make_float2(row_nd, row_nd);
                         }
                     };
+                    // -lse2 / -D of columns i .. i+3 (KV: one 16-byte shared load each)
+                    auto vec_quad = [&](int i, float4& nl4, float4& nd4) {
+                        if (KV) {
+                            nl4 = *reinterpret_cast<const float4*>(vec + cb + i);
+                            nd4 = *reinterpret_cast<const float4*>(vec + C::CR + cb + i);
+                        } else {
+                            nl4 = make_float4(row_nl2, row_nl2, row_nl2, row_nl2);
+                            nd4 = make_float4(row_nd, row_nd, row_nd, row_nd);
+                        }
+                    };
                     // fast path, packed pairs: P = 2^(s2 - lse2), dS = P (dP - D) (1 - tanh^2);
                     // on tiles that cross the band's edges each weight outside
-                    // [vlo, vhi] is replaced by 0 after its exp2
-                    auto fast = [&](auto mask_tag) {
+                    // [vlo, vhi] is replaced by 0 after its exp2. d = 256 dv units
+                    // need P only (want_y false: no dS).
+                    auto fast = [&](auto mask_tag, auto ds_tag) {
                         constexpr bool MASK = decltype(mask_tag)::value;
+                        constexpr bool DS = decltype(ds_tag)::value;
                         auto keep = [&](int i, int e, float p) {
                             if constexpr (MASK) {
                                 const int idx = (KV ? ((cb + i + e) & (CQ - 1)) : cb + i + e) + ccol0;
@@ -1146,54 +1176,83 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         };
                         const float2 one = make_float2(1.f, 1.f), mone = make_float2(-1.f, -1.f);
                         if (P.has_cap) {
-                            const float2 us = make_float2(P.u_scale, P.u_scale);
-                            const float2 c3 = make_float2(-17.0f / 315.0f, -17.0f / 315.0f);
-                            const float2 c2 = make_float2(2.0f / 15.0f, 2.0f / 15.0f);
-                            const float2 c1 = make_float2(-1.0f / 3.0f, -1.0f / 3.0f);
+                            // tanh(alpha x / C) = x (t0 + t1 x^2 + t2 x^4 + t3 x^6): the
+                            // series in u = alpha x / C with the powers of alpha / C
+                            // folded into its coefficients
+                            const float2 T0 = make_float2(P.th_c[0], P.th_c[0]);
+                            const float2 T1 = make_float2(P.th_c[1], P.th_c[1]);
+                            const float2 T2 = make_float2(P.th_c[2], P.th_c[2]);
+                            const float2 T3 = make_float2(P.th_c[3], P.th_c[3]);
                             const float2 cl2 = make_float2(P.cap_l2, P.cap_l2);
 #pragma unroll
-                            for (int i = 0; i < CHUNK; i += 2) {
-                                float2 nl2, nd;
-                                vec_pair(i, nl2, nd);
-                                const float2 x = make_float2(__uint_as_float(xv[i]),
-                                                             __uint_as_float(xv[i + 1]));
-                                const float2 y = make_float2(__uint_as_float(yv[i]),
-                                                             __uint_as_float(yv[i + 1]));
-                                const float2 u = mul2(x, us);
-                                const float2 u2 = mul2(u, u);
-                                float2 q = fma2(u2, c3, c2);
-                                q = fma2(u2, q, c1);
-                                q = fma2(u2, q, one);
-                                const float2 th = mul2(u, q);              // tanh(alpha x / C)
-                                const float2 e2 = fma2(th, cl2, nl2);       // s2 - lse2
-                                const float2 dcap = fma2(mul2(th, th), mone, one);
-                                const float p0 = keep(i, 0, ex2_approx(e2.x));
-                                const float p1 = keep(i, 1, ex2_approx(e2.y));
-                                const float2 ds = mul2(mul2(make_float2(p0, p1), add2(y, nd)), dcap);
-                                pp[i / 2] = pack_bf16x2(p0, p1);
-                                pd[i / 2] = pack_bf16x2(ds.x, ds.y);
+                            for (int i = 0; i < CHUNK; i += 4) {
+                                float4 nl4, nd4;
+                                vec_quad(i, nl4, nd4);
+#pragma unroll
+                                for (int j = 0; j < 4; j += 2) {
+                                    const int c = i + j;
+                                    const float2 nl2 = j ? make_float2(nl4.z, nl4.w)
+                                                         : make_float2(nl4.x, nl4.y);
+                                    const float2 nd = j ? make_float2(nd4.z, nd4.w)
+                                                        : make_float2(nd4.x, nd4.y);
+                                    const float2 x = make_float2(__uint_as_float(xv[c]),
+                                                                 __uint_as_float(xv[c + 1]));
+                                    const float2 x2 = mul2(x, x);
+                                    float2 q = fma2(x2, T3, T2);
+                                    q = fma2(x2, q, T1);
+                                    q = fma2(x2, q, T0);
+                                    const float2 th = mul2(x, q);             // tanh(alpha x / C)
+                                    const float2 e2 = fma2(th, cl2, nl2);      // s2 - lse2
+                                    const float p0 = keep(c, 0, ex2_approx(e2.x));
+                                    const float p1 = keep(c, 1, ex2_approx(e2.y));
+                                    pp[c / 2] = pack_bf16x2(p0, p1);
+                                    if constexpr (DS) {
+                                        const float2 y = make_float2(__uint_as_float(yv[c]),
+                                                                     __uint_as_float(yv[c + 1]));
+                                        const float2 dcap = fma2(mul2(th, th), mone, one);
+                                        const float2 ds =
+                                            mul2(mul2(make_float2(p0, p1), add2(y, nd)), dcap);
+                                        pd[c / 2] = pack_bf16x2(ds.x, ds.y);
+                                    }
+                                }
                             }
                         } else {
                             const float2 sl2 = make_float2(P.scale_l2, P.scale_l2);
 #pragma unroll
-                            for (int i = 0; i < CHUNK; i += 2) {
-                                float2 nl2, nd;
-                                vec_pair(i, nl2, nd);
-                                const float2 x = make_float2(__uint_as_float(xv[i]),
-                                                             __uint_as_float(xv[i + 1]));
-                                const float2 y = make_float2(__uint_as_float(yv[i]),
-                                                             __uint_as_float(yv[i + 1]));
-                                const float2 e2 = fma2(x, sl2, nl2);
-                                const float p0 = keep(i, 0, ex2_approx(e2.x));
-                                const float p1 = keep(i, 1, ex2_approx(e2.y));
-                                const float2 ds = mul2(make_float2(p0, p1), add2(y, nd));
-                                pp[i / 2] = pack_bf16x2(p0, p1);
-                                pd[i / 2] = pack_bf16x2(ds.x, ds.y);
+                            for (int i = 0; i < CHUNK; i += 4) {
+                                float4 nl4, nd4;
+                                vec_quad(i, nl4, nd4);
+#pragma unroll
+                                for (int j = 0; j < 4; j += 2) {
+                                    const int c = i + j;
+                                    const float2 nl2 = j ? make_float2(nl4.z, nl4.w)
+                                                         : make_float2(nl4.x, nl4.y);
+                                    const float2 nd = j ? make_float2(nd4.z, nd4.w)
+                                                        : make_float2(nd4.x, nd4.y);
+                                    const float2 x = make_float2(__uint_as_float(xv[c]),
+                                                                 __uint_as_float(xv[c + 1]));
+                                    const float2 e2 = fma2(x, sl2, nl2);
+                                    const float p0 = keep(c, 0, ex2_approx(e2.x));
+                                    const float p1 = keep(c, 1, ex2_approx(e2.y));
+                                    pp[c / 2] = pack_bf16x2(p0, p1);
+                                    if constexpr (DS) {
+                                        const float2 y = make_float2(__uint_as_float(yv[c]),
+                                                                     __uint_as_float(yv[c + 1]));
+                                        const float2 ds = mul2(make_float2(p0, p1), add2(y, nd));
+                                        pd[c / 2] = pack_bf16x2(ds.x, ds.y);
+                                    }
+                                }
                             }
                         }
                     };
                     if (poly || !P.has_cap) {
-                        if (interior) fast(BwMask<false>{}); else fast(BwMask<true>{});
+                        if (want_y) {
+                            if (interior) fast(BwMask<false>{}, BwMask<true>{});
+                            else fast(BwMask<true>{}, BwMask<true>{});
+                        } else {
+                            if (interior) fast(BwMask<false>{}, BwMask<false>{});
+                            else fast(BwMask<true>{}, BwMask<false>{});
+                        }
                     } else {
                         // general path: per-element mask, exact cap when |u| > 1/4
 #pragma unroll
@@ -1261,7 +1320,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(xbuf ? &zb_full[2 * b + part] : &z_full[part]);
+                if (lane == 0) mbar_arrive(xbuf ? &zb_full[BW_NPART * b + part] : &z_full[part]);
                 ++ct;
                 if (xbuf) ++bt; else ++xt;
             }
@@ -1271,8 +1330,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            constexpr int HALF = ACC_N / 2;           // accumulator columns per warp
-            constexpr int SEG = HALF < 64 ? HALF : 64;  // columns per TMEM round trip
+            constexpr int PCOLS = ACC_N / BW_NPART;       // accumulator columns per warp
+            constexpr int SEG = PCOLS < 32 ? PCOLS : 32;  // columns per TMEM round trip
             if (KV) {
                 const bool valid = r < U.rvalid;
                 const size_t row = (static_cast<size_t>(U.kbase) + key_row) * P.Hkv + U.g;
@@ -1282,19 +1341,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (AT && a != U.dh) continue;
                     const float f = a ? P.query_scale : 1.0f;
                     const uint32_t acol = AT ? 0u : static_cast<uint32_t>(a * ACC_N);
-                    __nv_bfloat16* dst = (a ? P.dk : P.dv) + row * D + part * HALF;
+                    __nv_bfloat16* dst = (a ? P.dk : P.dv) + row * D + part * PCOLS;
 #pragma unroll
-                    for (int sg = 0; sg < HALF / SEG; ++sg)
-                        bw_store_acc<SEG>(tmem + lane_addr + acol + part * HALF + SEG * sg,
+                    for (int sg = 0; sg < PCOLS / SEG; ++sg)
+                        bw_store_acc<SEG>(tmem + lane_addr + acol + part * PCOLS + SEG * sg,
                                           dst + SEG * sg, f, valid);
                 }
             } else {
                 const bool valid = pr_row < U.rvalid;
                 const size_t row = (static_cast<size_t>(U.qbase) + t_row) * P.H + 2 * U.g + hl_row;
-                __nv_bfloat16* dst = P.dq + row * D + part * HALF;
+                __nv_bfloat16* dst = P.dq + row * D + part * PCOLS;
 #pragma unroll
-                for (int sg = 0; sg < HALF / SEG; ++sg)
-                    bw_store_acc<SEG>(tmem + lane_addr + part * HALF + SEG * sg, dst + SEG * sg,
+                for (int sg = 0; sg < PCOLS / SEG; ++sg)
+                    bw_store_acc<SEG>(tmem + lane_addr + part * PCOLS + SEG * sg, dst + SEG * sg,
                                       P.query_scale, valid);
             }
             tc_fence_before();
