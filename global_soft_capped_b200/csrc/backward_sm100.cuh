@@ -91,7 +91,14 @@ struct BwCfg {
     static constexpr int VEC_TX = 2 * CR * 4;            //   (bytes copied: CR rows, two arrays)
     static constexpr int SLOT_BYTES = 2 * CTILE_BYTES + VEC_BYTES;
     static_assert(SLOT_BYTES % 1024 == 0 && VEC_TX <= VEC_BYTES, "slot layout");
-    static constexpr int SMEM_TILES = RES_TILES * TILE_BYTES + NSLOT * SLOT_BYTES;
+    // Layout, d <= 128: R1, R2, then the NSLOT slots. d = 256: the slots, then
+    // the one resident tile in a slot-sized region, so that a dv unit (which
+    // keeps nothing in shared memory) can stream through it as a third slot.
+    static constexpr int RES_BYTES = A_TMEM ? SLOT_BYTES : RES_TILES * TILE_BYTES;
+    static_assert(!A_TMEM || SLOT_BYTES >= TILE_BYTES, "resident region holds a slot");
+    static constexpr int NRING_MAX = A_TMEM ? NSLOT + 1 : NSLOT;  // slots of the widest ring
+    static_assert(NRING_MAX <= 4, "slot barriers");
+    static constexpr int SMEM_TILES = NSLOT * SLOT_BYTES + RES_BYTES;
     // TMEM columns: accumulators at 0, the resident A operand (d = 256), X, Y
     static constexpr uint32_t A_COL = 256;
     static constexpr uint32_t X_COL = A_TMEM ? 384 : BW_X_COL;
@@ -374,6 +381,56 @@ __global__ void __launch_bounds__(256) bwd_prep_varlen(
     }
 }
 
+// Slot ring of the column tiles; producer, issuers and elementwise warps keep
+// identical copies. Fixed ring (VAR false): every unit uses the same NMAX
+// slots, and tiles are numbered across units. Variable ring (d = 256: dv
+// units stream through one more slot than dk units): every unit starts with
+// all slots free (the producer waits for the previous unit's UMMAs to
+// complete before its first load), so tile c of a unit goes to slot c % n,
+// n the unit's ring size, and the barrier phases continue per slot.
+template <int NMAX, bool VAR>
+struct BwRing {
+    static_assert(NMAX >= 1 && NMAX <= 4, "up to four slots");
+    static_assert(VAR || (NMAX & (NMAX - 1)) == 0, "a fixed ring has a power-of-two size");
+    static constexpr int SLOTS = NMAX;
+    uint32_t base;            // fixed ring: tiles before the current unit
+    uint32_t u0, u1, u2, u3;  // variable ring: fills of each slot before the unit
+    int n;                    // variable ring: slots in the current unit's ring
+    __device__ __forceinline__ void init() {
+        base = u0 = u1 = u2 = u3 = 0;
+        n = NMAX;
+    }
+    // c / n and c % n for n in {1, 2, 3, 4} without a general division
+    __device__ __forceinline__ int quot(int c) const {
+        return n == 3 ? c / 3 : (n == 4 ? c >> 2 : (n == 2 ? c >> 1 : c));
+    }
+    __device__ __forceinline__ uint32_t uses(int p) const {
+        if constexpr (!VAR)
+            return base > static_cast<uint32_t>(p) ? (base - 1 - p) / NMAX + 1 : 0u;
+        else
+            return p == 0 ? u0 : (p == 1 ? u1 : (p == 2 ? u2 : u3));
+    }
+    __device__ __forceinline__ int slot(int c) const {
+        if constexpr (!VAR) return static_cast<int>((base + c) % NMAX);
+        else return c - n * quot(c);
+    }
+    __device__ __forceinline__ uint32_t phase(int c) const {
+        if constexpr (!VAR) return ((base + c) / NMAX) & 1u;
+        else return (uses(slot(c)) + static_cast<uint32_t>(quot(c))) & 1u;
+    }
+    __device__ __forceinline__ void end_unit(int ncols) {
+        if constexpr (!VAR) {
+            base += static_cast<uint32_t>(ncols);
+        } else {
+            const int q = quot(ncols), rem = ncols - n * q;
+            u0 += static_cast<uint32_t>(q + (0 < rem));
+            if (n > 1) u1 += static_cast<uint32_t>(q + (1 < rem));
+            if (n > 2) u2 += static_cast<uint32_t>(q + (2 < rem));
+            if (n > 3) u3 += static_cast<uint32_t>(q + (3 < rem));
+        }
+    }
+};
+
 // Static persistent schedule (as the forward): round r gives CTA c unit
 // r*G + c on even rounds and r*G + G-1-c on odd rounds.
 __device__ __forceinline__ int bw_sched(int r, int c, int G) {
@@ -488,15 +545,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     // d <= 128: R1 = K (KV) or q (Q), R2 = V or dout. d = 256: R1 = K (KV, dk
     // units) or dout (Q); the other operand is in TMEM.
-    uint8_t* sR1 = base;
-    uint8_t* sR2 = base + C::TILE_BYTES;
-    uint8_t* sSlot = base + C::RES_TILES * C::TILE_BYTES;  // [NSLOT] x (C1, C2, lse2[CR], D[CR])
+    // [NSLOT] x (C1, C2, lse2[CR], D[CR]); d = 256 dv units: + R1 as one more slot
+    uint8_t* sSlot = AT ? base : base + C::RES_BYTES;
+    uint8_t* sR1 = AT ? base + C::NSLOT * C::SLOT_BYTES : base;
+    uint8_t* sR2 = sR1 + C::TILE_BYTES;
     constexpr int NS = C::NSLOT;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::SMEM_TILES);
     uint64_t* r_full = bars + 0;
     uint64_t* r_empty = bars + 1;
-    uint64_t* c_full = bars + 2;    // [NSLOT <= 4]
-    uint64_t* c_empty = bars + 6;   // [NSLOT <= 4]
+    uint64_t* c_full = bars + 2;    // [NRING_MAX <= 4]
+    uint64_t* c_empty = bars + 6;   // [NRING_MAX <= 4]
     // Single-buffered X / Y (d = 256 dk units and dq kernel), per column part
     // h (columns HW h .. HW h + HW - 1 of X and Y, the column parts of the
     // elementwise warps):
@@ -525,7 +583,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(r_full, 1);
         mbar_init(r_empty, C::ISSUERS);
-        for (int i = 0; i < NS; ++i) {
+        for (int i = 0; i < C::NRING_MAX; ++i) {
             mbar_init(&c_full[i], 1);
             mbar_init(&c_empty[i], C::ISSUERS);
         }
@@ -614,11 +672,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const int cta = blockIdx.x;
     const uint64_t lim = P.timeout_ns;
     const int num_units = P.varlen ? min(P.num_units, cum[P.num_seqs] * DS) : P.num_units;
+    // slots in a unit's ring: d = 256 dv units also stream through R1
+    auto ring_size = [](const BwUnit& U) { return (AT && KV && U.dh == 0) ? NS + 1 : NS; };
+    using Ring = BwRing<(AT && KV) ? C::NRING_MAX : NS, AT && KV>;
 
     if (warp == BW_WARP_PRODUCER) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            uint32_t ct = 0;  // column tiles loaded so far
+            Ring ring;
+            ring.init();
             int uw = 0;       // units with work so far
             bool ok = true;
             for (int r = 0; ok && r * G < num_units; ++r) {
@@ -653,10 +715,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         bw_load_tile<D>(sR2, &tmO, r_full, U.qbase + U.row0, 2 * U.g);
                     }
                 }
+                ring.n = ring_size(U);
                 for (int c = 0; c < U.ncols; ++c) {
-                    const int sl = ct % NS;
-                    ok = mbar_wait(&c_empty[sl], ((ct / NS) & 1) ^ 1, abort_flag, lim,
-                                   SITE_BW_PROD);
+                    const int sl = ring.slot(c);
+                    ok = mbar_wait(&c_empty[sl], ring.phase(c) ^ 1, abort_flag, lim, SITE_BW_PROD);
                     if (!ok) break;
                     uint8_t* slot = sSlot + sl * C::SLOT_BYTES;
                     if (KV) {
@@ -682,16 +744,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         bw_load_tile<D>(slot + C::CTILE_BYTES, &tmV, &c_full[sl], U.kbase + key0,
                                         U.g, C::CR);
                     }
-                    ++ct;
                 }
+                if (!ok) break;
+                ring.end_unit(U.ncols);
                 ++uw;
             }
-            // Drain: every copy issued lands before the CTA exits.
-            const uint32_t last = ct < uint32_t(NS) ? ct : uint32_t(NS);
-            for (uint32_t i = 0; i < last; ++i) {
-                const uint32_t f = ct - 1 - i;
-                mbar_wait_drain(&c_full[f % NS], (f / NS) & 1, lim);
-            }
+            // Drain: every copy issued lands before the CTA exits (the last
+            // fill of each slot).
+#pragma unroll
+            for (int p = 0; p < Ring::SLOTS; ++p)
+                if (ring.uses(p) > 0) mbar_wait_drain(&c_full[p], (ring.uses(p) - 1) & 1, lim);
             if (uw > 0) mbar_wait_drain(r_full, (uw - 1) & 1, lim);
         }
         __syncwarp();
@@ -725,7 +787,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const uint32_t slot_lo_mn = sdesc_lo(smem_u32(sSlot), C::CR * 128);
             constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
             constexpr uint32_t CTILE_STEP = C::CTILE_BYTES >> 4;
-            uint32_t ct = 0;   // column tiles (slot ring)
+            Ring ring;         // column-tile slots
+            ring.init();
             uint32_t bt = 0;   // column tiles with double-buffered X / Y (xb_full, zb_full)
             uint32_t xt = 0;   // column tiles with single-buffered X / Y (xy_full, z_full)
             int uw = 0;
@@ -874,12 +937,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     }
                 }
             };
-            // X / Y of column tile t (slot ring position t) into buffer b
-            auto load_xy_buf = [&](uint32_t t, uint32_t b) -> bool {
-                if (!mbar_wait(&c_full[t % NS], (t / NS) & 1, abort_flag, lim, SITE_BW_MMA))
+            // X / Y of the unit's column tile c into buffer b
+            auto load_xy_buf = [&](int c, uint32_t b) -> bool {
+                if (!mbar_wait(&c_full[ring.slot(c)], ring.phase(c), abort_flag, lim, SITE_BW_MMA))
                     return false;
                 tc_fence_after();
-                issue_xy_buf(static_cast<int>(t % NS), b);
+                issue_xy_buf(ring.slot(c), b);
                 return true;
             };
             for (int r = 0; ok && r * G < num_units; ++r) {
@@ -895,13 +958,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (!ok) break;
                 }
                 tc_fence_after();
+                ring.n = ring_size(U);
                 if (C::DB || (KV && U.dh == 0)) {
                     // double-buffered X / Y (d = 256: dv units, X only)
-                    ok = load_xy_buf(ct, bt & 1);
-                    if (ok && U.ncols > 1) ok = load_xy_buf(ct + 1, (bt + 1) & 1);
+                    ok = load_xy_buf(0, bt & 1);
+                    if (ok && U.ncols > 1) ok = load_xy_buf(1, (bt + 1) & 1);
                     if (!ok) break;
                     for (int c = 0; c < U.ncols; ++c) {
-                        const int sl = static_cast<int>(ct % NS);
+                        const int sl = ring.slot(c);
                         const uint32_t b = bt & 1;
                         if (c == 0 && uw > 0) {
                             ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim,
@@ -919,13 +983,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                         if (!ok) break;
                         umma_commit(&c_empty[sl]);
                         if (c + 2 < U.ncols) {  // tile c+2 goes into buffer b again
-                            ok = load_xy_buf(ct + 2, b);
+                            ok = load_xy_buf(c + 2, b);
                             if (!ok) break;
                         }
-                        ++ct;
                         ++bt;
                     }
                     if (!ok) break;
+                    ring.end_unit(U.ncols);
                     umma_commit(acc_done);
                     umma_commit(r_empty);
                     ++uw;
@@ -933,12 +997,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
                 if constexpr (!AT) continue;  // (every unit above)
                 // single-buffered X / Y (d = 256 dk units and dq kernel)
-                ok = mbar_wait(&c_full[ct % NS], (ct / NS) & 1, abort_flag, lim, SITE_BW_MMA);
+                ok = mbar_wait(&c_full[ring.slot(0)], ring.phase(0), abort_flag, lim, SITE_BW_MMA);
                 if (!ok) break;
                 tc_fence_after();
-                issue_xy_tile(static_cast<int>(ct % NS), U.dh);
+                issue_xy_tile(ring.slot(0), U.dh);
                 for (int c = 0; c < U.ncols; ++c) {
-                    const int sl = static_cast<int>(ct % NS);
+                    const int sl = ring.slot(c);
                     if (c == 0 && uw > 0) {
                         ok = mbar_wait(acc_free, (uw - 1) & 1, abort_flag, lim, SITE_BW_MMA_ACC);
                         if (!ok) break;
@@ -953,16 +1017,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     if (!ok) break;
                     umma_commit(&c_empty[sl]);
                     if (c + 1 < U.ncols) {
-                        ok = mbar_wait(&c_full[(ct + 1) % NS], ((ct + 1) / NS) & 1, abort_flag,
+                        ok = mbar_wait(&c_full[ring.slot(c + 1)], ring.phase(c + 1), abort_flag,
                                        lim, SITE_BW_MMA);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_xy_tile(static_cast<int>((ct + 1) % NS), U.dh);
+                        issue_xy_tile(ring.slot(c + 1), U.dh);
                     }
-                    ++ct;
                     ++xt;
                 }
                 if (!ok) break;
+                ring.end_unit(U.ncols);
                 umma_commit(acc_done);
                 umma_commit(r_empty);
                 ++uw;
@@ -984,7 +1048,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const int r = (qd << 5) | lane;
         const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
         const int col0 = part * HW;
-        uint32_t ct = 0;   // column tiles (slot ring)
+        Ring ring;         // column-tile slots
+        ring.init();
         uint32_t xt = 0;   // column tiles with single-buffered X / Y (xy_full, z_full)
         uint32_t bt = 0;   // column tiles with double-buffered X / Y (xb_full, zb_full)
         int uw = 0;
@@ -1061,8 +1126,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             // double-buffered X / Y (d <= 128; d = 256 dv units: X only, in
             // the X and Y columns alternately)
             const bool xbuf = C::DB || (KV && U.dh == 0);
+            ring.n = ring_size(U);
             for (int c = 0; c < U.ncols; ++c) {
-                const int sl = static_cast<int>(ct % NS);
+                const int sl = ring.slot(c);
                 const uint32_t b = bt & 1;
                 const uint32_t x_col = xbuf ? C::XB0 + C::XB_STEP * b : X_COL;
                 const uint32_t y_col = xbuf ? C::YB0 + C::XB_STEP * b : Y_COL;
@@ -1071,7 +1137,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 else
                     ok = mbar_wait(&xy_full[part], xt & 1, abort_flag, lim, SITE_BW_EW);
                 if (KV && ok)  // the column tile's lse2 / D, copied with its operands
-                    ok = mbar_wait(&c_full[sl], (ct / NS) & 1, abort_flag, lim, SITE_BW_EW);
+                    ok = mbar_wait(&c_full[sl], ring.phase(c), abort_flag, lim, SITE_BW_EW);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
@@ -1321,10 +1387,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(xbuf ? &zb_full[BW_NPART * b + part] : &z_full[part]);
-                ++ct;
                 if (xbuf) ++bt; else ++xt;
             }
             if (!ok) break;
+            ring.end_unit(U.ncols);
             // ---- epilogue: accumulators -> bf16 gradients
             ok = mbar_wait(acc_done, uw & 1, abort_flag, lim, SITE_BW_EW_ACC);
             ok = __all_sync(0xffffffffu, ok);
