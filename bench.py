@@ -144,16 +144,60 @@ def ncu_traffic(kernel_key, units_now):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled through NVML every 2 ms
+    by a background thread; stop() keeps the samples taken inside the timed
+    region (mark_begin / mark_end). Falls back to nvidia-smi at 100 ms."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index):
-        self.dev = device_index
+    def __init__(self, device):
+        self.device = device
+        self.dev = device.index if device.index is not None else 0
         self.proc = None
+        self.thread = None
+        self.samples = []
+        self.t0 = self.t1 = None
         self.path = os.path.join("/tmp", f"g2attn_clocks_{os.getpid()}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop_flag = False
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+
+            def run():
+                while not self.stop_flag:
+                    t = time.perf_counter()
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = int(get_reasons(h)) if get_reasons else 0
+                        self.samples.append((t, sm, pw, rs))
+                    except Exception:
+                        pass
+                    time.sleep(0.002)
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            time.sleep(0.02)  # the sampler is running before the timed region starts
+            return
+        except Exception:
+            self.thread = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -162,9 +206,26 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def mark_begin(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            inside = [x for x in self.samples if self.t0 is not None and self.t0 <= x[0] <= self.t1]
+            reasons = sorted({n for x in inside for bit, n in self.REASONS.items() if x[3] & bit})
+            sms = [x[1] for x in inside]
+            return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": self.max_mhz,
+                    "sm_mhz_min": min(sms) if sms else None,
+                    "power_w_median": round(statistics.median([x[2] for x in inside]), 1) if inside else None,
+                    "samples_in_timed_region": len(inside), "sampler": "NVML every 2 ms",
+                    "reasons": reasons}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -190,7 +251,8 @@ class ClockSampler:
                     reasons.add(n)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
-                "samples_under_load": len(sms), "reasons": sorted(reasons)}
+                "samples_under_load": len(sms), "sampler": "nvidia-smi every 100 ms",
+                "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------------------
@@ -238,11 +300,12 @@ def run_ours(args, rank, world, dev):
 
     nsteps = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks = ClockSampler(dev)
+    clocks.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks.start()
+    clocks.mark_begin()
     t_wall = time.perf_counter()
     for i in range(nsteps):
         flush.zero_()
@@ -253,6 +316,7 @@ def run_ours(args, rank, world, dev):
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
+    clocks.mark_end()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
