@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/g2attn.h"
@@ -266,7 +267,9 @@ int decode_common(g2::DecParams& P, const g2::DecLayoutParams& LP, const void* q
     P.Hkv = Hkv;
     P.window = window;
     P.chunk = chunk;
-    P.max_splits = splits;
+    // a local layer sees at most `window` keys per sequence: no more splits than
+    // that range needs (the workspace, sized for max_cache_len, stays large enough)
+    P.max_splits = window > 0 ? std::min(splits, (window + chunk - 1) / chunk) : splits;
     fill_cap(query_scale, softcap, P.k_exp, P.cap_l2, P.scale_l2, P.has_cap);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (d) {
