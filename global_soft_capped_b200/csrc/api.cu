@@ -169,8 +169,6 @@ bool use_pairs() {
 
 int dispatch_prefill(int d, const void* q, const void* k, const void* v, long long tq,
                      long long tk, g2::PfParams& P, cudaStream_t st) {
-    // rows of d bf16 (128 B or more) stay 32-byte aligned when the base is
-    P.out_align32 = (reinterpret_cast<uintptr_t>(P.out) & 31u) == 0;
     switch (d) {
         case 64: return launch_prefill<64, 1>(q, k, v, tq, tk, P, st);
         case 128: return launch_prefill<128, 1>(q, k, v, tq, tk, P, st);

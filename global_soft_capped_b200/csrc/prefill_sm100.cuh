@@ -129,7 +129,6 @@ struct PfParams {
     // softmax is invariant to the shift, so no running max is needed.
     int fixed_ref_on;
     float fixed_ref;
-    int out_align32;  // out is 32-byte aligned: the epilogue stores 32 bytes at a time
     unsigned long long timeout_ns;
 };
 
