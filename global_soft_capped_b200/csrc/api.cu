@@ -378,8 +378,17 @@ void fill_bwd_series(float query_scale, float softcap, g2::BwParams& P) {
 // workspace (-lse*log2(e) and -D, fp32 each).
 long long bwd_tp(int T) { return (static_cast<long long>(T) + 63) / 64 * 64; }
 
-size_t bwd_ws_bytes(int B, int T, int H) {
+// Then a 256-byte block holding the unit counters of the two gradient kernels
+// (zeroed by the pass that runs before them).
+constexpr size_t kBwdSchedBytes = 256;
+
+size_t bwd_ws_rows_bytes(int B, int T, int H) {
     return 2ull * static_cast<size_t>(B) * static_cast<size_t>(H) * bwd_tp(T) * sizeof(float);
+}
+
+size_t bwd_ws_bytes(int B, int T, int H) {
+    const size_t rows = bwd_ws_rows_bytes(B, T, H);
+    return rows == 0 ? 0 : rows + kBwdSchedBytes;
 }
 
 template <int D, int MODE>
@@ -427,11 +436,14 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
     // -D = -(dout . out) and -lse * log2(e) per (b, h, position)
     const long long rows = static_cast<long long>(P.B) * P.H * P.Tp;
     const long long threads = rows * (D / 8);
+    // the unit counters follow the rows in the workspace
+    unsigned int* sched = reinterpret_cast<unsigned int*>(
+        reinterpret_cast<char*>(const_cast<float*>(P.nlse2)) + bwd_ws_rows_bytes(P.B, P.T, P.H));
     const long long blocks = (threads + 255) / 256;
     if (blocks > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
     g2::bwd_prep<D><<<static_cast<int>(blocks), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse,
-        const_cast<float*>(P.nlse2), const_cast<float*>(P.ndvec), P.B, P.T, P.H, P.Tp);
+        const_cast<float*>(P.nlse2), const_cast<float*>(P.ndvec), P.B, P.T, P.H, P.Tp, sched);
     if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
     const int BG = P.B * P.Hkv;
     const int key_tiles = (P.S + g2::BW_KEYS - 1) / g2::BW_KEYS;
@@ -439,10 +451,12 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
     P.row_tiles = key_tiles;
     const long long kv_units = static_cast<long long>(key_tiles) * BG * g2::BwCfg<D>::DSPLIT_KV;
     if (kv_units > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    P.sched = sched;
     int rc = launch_bwd<D, g2::BW_KV>(m.q_kv, m.o_kv, m.k_kv, m.v_kv, P,
                                       static_cast<int>(kv_units), sms, st);
     if (rc) return rc;
     P.row_tiles = q_tiles;
+    P.sched = sched + 1;
     return launch_bwd<D, g2::BW_Q>(m.q_q, m.o_q, m.k_q, m.v_q, P, q_tiles * BG, sms, st);
 }
 
@@ -452,9 +466,14 @@ long long bwd_vl_wmax(int num_seqs, int total_q) {
     return (static_cast<long long>(total_q) + 64ll * num_seqs + 63) / 64 * 64;
 }
 
+size_t bwd_vl_ws_head_bytes(int num_seqs, int total_q, int H) {
+    const size_t b = 2ull * H * bwd_vl_wmax(num_seqs, total_q) * sizeof(float) +
+                     (static_cast<size_t>(num_seqs) + 1) * sizeof(int);
+    return (b + kBwdSchedBytes - 1) / kBwdSchedBytes * kBwdSchedBytes;
+}
+
 size_t bwd_vl_ws_bytes(int num_seqs, int total_q, int H) {
-    return 2ull * H * bwd_vl_wmax(num_seqs, total_q) * sizeof(float) +
-           (static_cast<size_t>(num_seqs) + 1) * sizeof(int);
+    return bwd_vl_ws_head_bytes(num_seqs, total_q, H) + kBwdSchedBytes;
 }
 
 template <int D>
@@ -465,7 +484,11 @@ int launch_backward_varlen(const void* q, const void* k, const void* v, const vo
     if (!make_bw_maps<D>(m, q, k, v, dout, total_q, total_k, P.H, P.Hkv)) return G2ATTN_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return G2ATTN_ERR_CUDA;
-    g2::bwd_wq_prefix<<<1, 32, 0, st>>>(P.cu_q, P.num_seqs, total_q, const_cast<int*>(P.wq));
+    unsigned int* sched = reinterpret_cast<unsigned int*>(
+        reinterpret_cast<char*>(const_cast<float*>(P.nlse2)) +
+        bwd_vl_ws_head_bytes(P.num_seqs, total_q, P.H));
+    g2::bwd_wq_prefix<<<1, 32, 0, st>>>(P.cu_q, P.num_seqs, total_q, const_cast<int*>(P.wq),
+                                       sched);
     if (cudaGetLastError() != cudaSuccess) return G2ATTN_ERR_CUDA;
     const long long threads = static_cast<long long>(P.H) * P.wmax * (D / 8);
     const long long blocks = (threads + 255) / 256;
@@ -481,9 +504,11 @@ int launch_backward_varlen(const void* q, const void* k, const void* v, const vo
                             g2::BwCfg<D>::DSPLIT_KV;
     const long long q_ub = (static_cast<long long>(total_q) / g2::BW_QPOS + P.num_seqs) * P.Hkv;
     if (kv_ub > INT32_MAX || q_ub > INT32_MAX) return G2ATTN_ERR_UNSUPPORTED;
+    P.sched = sched;
     int rc = launch_bwd<D, g2::BW_KV>(m.q_kv, m.o_kv, m.k_kv, m.v_kv, P, static_cast<int>(kv_ub),
                                       sms, st);
     if (rc) return rc;
+    P.sched = sched + 1;
     return launch_bwd<D, g2::BW_Q>(m.q_q, m.o_q, m.k_q, m.v_q, P, static_cast<int>(q_ub), sms, st);
 }
 

@@ -151,6 +151,11 @@ struct BwParams {
     float poly_acc_max;  // largest |q.k| with |alpha q.k / C| <= 1/4 (0: series off)
     int has_cap;
     unsigned long long timeout_ns;
+    // Unit counter of this launch in the caller's workspace, zeroed by the
+    // pass that runs before it: the CTAs take units in order from it (a
+    // dynamic list schedule, longest units first). nullptr: the static
+    // zig-zag schedule.
+    unsigned int* sched;
 };
 
 // tanh(u) for |u| <= 1/4: Taylor series through u^7 (coefficients -1/3, 2/15,
@@ -276,7 +281,10 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict__ out,
                                                 const __nv_bfloat16* __restrict__ dout,
                                                 const float* __restrict__ lse, float* nlse2,
-                                                float* ndvec, int B, int T, int H, int Tp) {
+                                                float* ndvec, int B, int T, int H, int Tp,
+                                                unsigned int* sched) {
+    // the gradient kernels' unit counters, for the launches that follow
+    if (blockIdx.x == 0 && threadIdx.x < 2) sched[threadIdx.x] = 0u;
     constexpr int LPR = D / 8;  // lanes per row
     const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / LPR;
     const int sub = threadIdx.x % LPR;
@@ -310,8 +318,10 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict_
 // Varlen: wq[s] = sum over s' < s of T_s' rounded up to 64 (the workspace
 // column where sequence s starts), wq[num_seqs] = the total. One block.
 __global__ void __launch_bounds__(32) bwd_wq_prefix(const int* __restrict__ cu_q, int num_seqs,
-                                                    int total_q, int* wq) {
+                                                    int total_q, int* wq, unsigned int* sched) {
     const int lane = threadIdx.x;
+    // the gradient kernels' unit counters, for the launches that follow
+    if (lane < 2) sched[lane] = 0u;
     int carry = 0;
     for (int s0 = 0; s0 < num_seqs; s0 += 32) {
         const int q = s0 + lane;
@@ -571,8 +581,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     // neither side can run two phases ahead of a waiter.
     uint64_t* xb_full = bars + 22;  // [2]
     uint64_t* zb_full = bars + 24;  // [2 NPART]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24 + 2 * BW_NPART);
+    // dynamic schedule: the producer publishes each unit it takes in a ring of
+    // four (sq_full: published; sq_empty: read by both issuers and every
+    // elementwise warp)
+    uint64_t* sq_full = bars + 24 + 2 * BW_NPART;   // [4]
+    uint64_t* sq_empty = sq_full + 4;               // [4]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sq_empty + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* sq_ring = reinterpret_cast<volatile int*>(tmem_holder + 4);  // [4], 16-byte aligned
     // varlen tables: cum[num_seqs + 1] (unit prefix in rank order), order[], work[]
     int* cum = reinterpret_cast<int*>(base + C::SMEM_TILES + 1024);
     int* order = cum + C::MAX_SEQ_TABLE + 1;
@@ -597,6 +613,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         mbar_init(ra_full, BW_EW_THREADS / 32);
         for (int b = 0; b < 2; ++b) mbar_init(&xb_full[b], C::ISSUERS);
         for (int i = 0; i < 2 * BW_NPART; ++i) mbar_init(&zb_full[i], 4);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&sq_full[i], 1);
+            mbar_init(&sq_empty[i], C::ISSUERS + BW_EW_THREADS / 32);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -672,6 +692,39 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const int cta = blockIdx.x;
     const uint64_t lim = P.timeout_ns;
     const int num_units = P.varlen ? min(P.num_units, cum[P.num_seqs] * DS) : P.num_units;
+    // Unit of round r for this CTA, or -1 when it has no more. Static: the
+    // zig-zag schedule. Dynamic: the producer takes the next unit from the
+    // launch's counter and publishes it in sq_ring; the issuers and the
+    // elementwise warps read it there in the same order. Every role sees the
+    // same sequence of units, ending with one past num_units.
+    auto take_unit = [&](int r, bool& ok) -> int {
+        if (P.sched == nullptr) return r * G < num_units ? bw_sched(r, cta, G) : -1;
+        const int i = r & 3;
+        if (!mbar_wait(&sq_empty[i], ((r >> 2) & 1) ^ 1, abort_flag, lim, SITE_BW_PROD)) {
+            ok = false;
+            return -1;
+        }
+        const int u = static_cast<int>(atomicAdd(P.sched, 1u));
+        sq_ring[i] = u;
+        mbar_arrive(&sq_full[i]);  // release: the ring entry is visible to the waiters
+        return u < num_units ? u : -1;
+    };
+    // a consumer's copy; `warp_wide`: every lane of the warp calls it and one
+    // arrival is made for the warp
+    auto read_unit = [&](int r, bool& ok, bool warp_wide) -> int {
+        if (P.sched == nullptr) return r * G < num_units ? bw_sched(r, cta, G) : -1;
+        const int i = r & 3;
+        bool w = mbar_wait(&sq_full[i], (r >> 2) & 1, abort_flag, lim, SITE_BW_MMA);
+        if (warp_wide) w = __all_sync(0xffffffffu, w);
+        if (!w) {
+            ok = false;
+            return -1;
+        }
+        const int u = sq_ring[i];
+        if (warp_wide) __syncwarp();
+        if (!warp_wide || lane == 0) mbar_arrive(&sq_empty[i]);
+        return u < num_units ? u : -1;
+    };
     // slots in a unit's ring: d = 256 dv units also stream through R1
     auto ring_size = [](const BwUnit& U) { return (AT && KV && U.dh == 0) ? NS + 1 : NS; };
     using Ring = BwRing<(AT && KV) ? C::NRING_MAX : NS, AT && KV>;
@@ -683,9 +736,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             ring.init();
             int uw = 0;       // units with work so far
             bool ok = true;
-            for (int r = 0; ok && r * G < num_units; ++r) {
-                const int u = bw_sched(r, cta, G);
-                if (u >= num_units) continue;
+            for (int r = 0; ok; ++r) {
+                const int u = take_unit(r, ok);
+                if (u < 0) break;
                 BwUnit U;
                 bw_unit<D, MODE>(P, cum, order, u, U);
                 if (U.ncols == 0) continue;
@@ -945,9 +998,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 issue_xy_buf(ring.slot(c), b);
                 return true;
             };
-            for (int r = 0; ok && r * G < num_units; ++r) {
-                const int u = bw_sched(r, cta, G);
-                if (u >= num_units) continue;
+            for (int r = 0; ok; ++r) {
+                const int u = read_unit(r, ok, false);
+                if (u < 0) break;
                 BwUnit U;
                 bw_unit<D, MODE>(P, cum, order, u, U);
                 if (U.ncols == 0) continue;
@@ -1054,9 +1107,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         uint32_t bt = 0;   // column tiles with double-buffered X / Y (xb_full, zb_full)
         int uw = 0;
         bool ok = true;
-        for (int rr = 0; ok && rr * G < num_units; ++rr) {
-            const int u = bw_sched(rr, cta, G);
-            if (u >= num_units) continue;
+        for (int rr = 0; ok; ++rr) {
+            const int u = read_unit(rr, ok, true);
+            if (u < 0) break;
             BwUnit U;
             bw_unit<D, MODE>(P, cum, order, u, U);
             if (U.ncols == 0) {

@@ -249,7 +249,9 @@ G2ATTN_API size_t g2attn_backward_workspace_size(int B, int T, int H);
  *     full (keys that no query sees get zero gradients).
  *   workspace: device memory of at least
  *     g2attn_backward_workspace_size(B, T, H) bytes, 16-byte aligned, owned by
- *     the caller and overwritten.
+ *     the caller and overwritten: -lse*log2(e) and -D per (b, h, position),
+ *     then the two gradient kernels' unit counters (the CTAs take their units
+ *     in order from a counter, longest first; the first pass zeroes them).
  * Supported: d = 64, 128 and 256. At d = 256 one of the two resident tiles of
  * each gradient kernel is held in tensor memory (it is read by the UMMAs as
  * their A operand), the streamed tiles are 64 rows, and the dk/dv kernel runs
@@ -282,7 +284,8 @@ G2ATTN_API size_t g2attn_varlen_backward_workspace_size(int num_seqs, int total_
  * packed like q.
  *   dq like q, dk and dv like k and v (bf16), written in full.
  *   workspace: at least g2attn_varlen_backward_workspace_size(num_seqs,
- *     total_q, H) bytes, 16-byte aligned, overwritten.
+ *     total_q, H) bytes, 16-byte aligned, overwritten (per-row vectors, the
+ *     padded prefix of the sequences, the unit counters).
  * Sequence rows derived from cu_seqlens are clamped into [0, total_q) and
  * [0, total_k): malformed offsets give undefined results but no access
  * outside the tensors. Supported: d = 64, 128 and 256; num_seqs <= 1024.

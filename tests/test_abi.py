@@ -149,10 +149,13 @@ def test_paged_prefill_rejects_before_launch(lib):
     assert g2.g2attn_prefill_paged(*bad) == g2.G2ATTN_ERR_INVALID_ARG
 
 
+SCHED_BYTES = 256  # the gradient kernels' unit counters, after the per-row vectors
+
+
 def test_backward_workspace_size(lib):
     a = g2.g2attn_backward_workspace_size(1, 8192, 32)
-    assert a == 2 * 1 * 32 * 8192 * 4
-    assert g2.g2attn_backward_workspace_size(2, 65, 4) == 2 * 2 * 4 * 128 * 4  # 64-padded
+    assert a == 2 * 1 * 32 * 8192 * 4 + SCHED_BYTES
+    assert g2.g2attn_backward_workspace_size(2, 65, 4) == 2 * 2 * 4 * 128 * 4 + SCHED_BYTES
     assert g2.g2attn_backward_workspace_size(0, 64, 4) == 0
 
 
@@ -183,7 +186,9 @@ def test_backward_rejects_before_launch(lib, kw, status):
 
 def test_varlen_backward_workspace_size(lib):
     wmax = (100 + 64 * 3 + 63) // 64 * 64      # every sequence padded to whole tiles
-    assert g2.g2attn_varlen_backward_workspace_size(3, 100, 8) == 2 * 8 * wmax * 4 + 4 * 4
+    head = 2 * 8 * wmax * 4 + 4 * 4                # -lse2, -D, then the prefix wq[4]
+    head = (head + SCHED_BYTES - 1) // SCHED_BYTES * SCHED_BYTES
+    assert g2.g2attn_varlen_backward_workspace_size(3, 100, 8) == head + SCHED_BYTES
     assert g2.g2attn_varlen_backward_workspace_size(0, 100, 8) == 0
     assert g2.g2attn_varlen_backward_workspace_size(3, 0, 8) == 0
 
