@@ -44,6 +44,7 @@ enum WaitSite : unsigned int {
     SITE_BW_EW_ACC = 18,    // backward elementwise: accumulation finished
     SITE_EPI_O_DONE = 19,   // forward epilogue: the unit's last PV completed
     SITE_EPI_STATS = 20,    // forward epilogue: row statistics handed over
+    SITE_SCHED = 21,        // forward, dynamic schedule: a unit published / released
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -385,6 +386,53 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
+}
+
+// The same with cluster-scope release: orders this thread's earlier ordinary
+// shared-memory accesses, the other CTA's included, before the arrival.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// Bounded wait on a local mbarrier with cluster-scope acquire: ordinary
+// shared-memory writes that the other CTA made before its releasing arrival
+// are visible after it. Gives up like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity,
+                                                          volatile int* abort_flag,
+                                                          uint64_t limit_ns, unsigned int site) {
+    auto try_once = [&]() -> bool {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        return ok != 0;
+    };
+    if (try_once()) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (try_once()) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            raise_timeout(abort_flag, site);
+            return false;
+        }
+    }
+}
+
+// Store a 32-bit value at a cluster-window shared address (either CTA).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long grid_launch_id() {
+    unsigned long long g;
+    asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+    return g;
 }
 
 // Tiled load into this CTA's shared memory whose completion is counted on an

@@ -286,6 +286,14 @@ __device__ __forceinline__ void pf_store_rows(uint32_t (&w)[EC / 2], int lane, R
     }
 }
 
+// Dynamic schedule of packed sequences: per-launch unit counters (next unit,
+// CTAs finished) at slot %gridid mod PF_SCHED_SLOTS. The CTA pairs take units
+// in order from `next` (list scheduling, heaviest sequences first); the last
+// CTA of a launch to finish zeroes its slot, so the slot is clean for the
+// launch that reuses it (launches in flight at once use distinct grid ids).
+constexpr int PF_SCHED_SLOTS = 4096;
+__device__ unsigned int g_pf_sched[PF_SCHED_SLOTS][2];
+
 // Static persistent schedule: round r gives CTA c unit r*G + c (even rounds)
 // or r*G + G-1-c (odd rounds), so the longest units spread evenly.
 __device__ __forceinline__ int pf_sched(int r, int c, int G) {
@@ -322,8 +330,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     uint64_t* xbar = bars + 11 + 2 * C::NSLOT;
     // row statistics of a unit handed to the epilogue warps, by unit parity [2]
     uint64_t* stat_full = xbar + 8;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(stat_full + 2);
+    // dynamic schedule (packed sequences): the even CTA's producer publishes
+    // each unit it takes in a ring of four in both CTAs (sq_full, one arrival);
+    // every other role of both CTAs releases the entry on the even CTA's
+    // sq_empty
+    uint64_t* sq_full = stat_full + 2;   // [4]
+    uint64_t* sq_empty = sq_full + 4;    // [4]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sq_empty + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* sq_ring = reinterpret_cast<volatile int*>(tmem_holder + 2);  // [4]
     // partial row maxima of the column parts, by tile parity: [2][NSPLIT][128]
     float* xmax = reinterpret_cast<float*>(base + C::SMEM_TILES + 1024);
     // partial (l, lr) row sums of the parts at the end of a unit, by unit
@@ -353,6 +368,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         mbar_init(o_free, CG * PF_EPI_WARPS);
         for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], PF_NSPLIT);
         for (int i = 0; i < 2; ++i) mbar_init(&stat_full[i], PF_SOFTMAX_THREADS / 32);
+        // readers per CTA: softmax and epilogue warps, and the issuer (even
+        // CTA) or the producer (odd CTA)
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&sq_full[i], 1);
+            mbar_init(&sq_empty[i], CG * (PF_SOFTMAX_THREADS / 32 + PF_EPI_WARPS + 1));
+        }
         mbar_init(drain, 1);
         mbar_init(o_last, 1);
         for (int i = 0; i < C::NSLOT; ++i) {
@@ -445,6 +466,59 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     // pair signal (data arrival, P ready, O read).
     const uint32_t l_q_full = PAIR ? mapa_shared(smem_u32(q_full), 0) : 0u;
     const uint32_t l_o_free = PAIR ? mapa_shared(smem_u32(o_free), 0) : 0u;
+    // Units of this CTA (pair), round by round; -1 when there are no more.
+    // Dense: the static zig-zag rounds. Packed sequences: the dynamic schedule
+    // (the even CTA's producer takes each unit and publishes it; the other
+    // roles of both CTAs read it from their ring in the same order).
+    const bool dyn = P.varlen != 0;
+    unsigned int* sched = g_pf_sched[grid_launch_id() % PF_SCHED_SLOTS];
+    auto ring_addr = [&](int i) {
+        return smem_u32(reinterpret_cast<const void*>(const_cast<const int*>(sq_ring + i)));
+    };
+    auto static_unit = [&](int r) -> int {
+        if (r * G >= num_units) return -1;
+        const int u = pf_sched(r, cta, G);
+        return u < num_units ? u : -1;
+    };
+    auto take_unit = [&](int r, bool& ok) -> int {  // the even CTA's producer
+        if (!dyn) return static_unit(r);
+        const int i = r & 3;
+        if (!mbar_wait(&sq_empty[i], ((r >> 2) & 1) ^ 1, abort_flag, lim, SITE_SCHED)) {
+            ok = false;
+            return -1;
+        }
+        const int u = static_cast<int>(atomicAdd(&sched[0], 1u));
+        sq_ring[i] = u;
+        if constexpr (PAIR) {
+            st_shared_cluster_u32(mapa_shared(ring_addr(i), 1), static_cast<uint32_t>(u));
+            mbar_arrive_release_cluster(mapa_shared(smem_u32(&sq_full[i]), 1));
+        }
+        mbar_arrive(&sq_full[i]);
+        return u < num_units ? u : -1;
+    };
+    // `warp_wide`: every lane calls it, one arrival per warp
+    auto read_unit = [&](int r, bool& ok, bool warp_wide) -> int {
+        if (!dyn) return static_unit(r);
+        const int i = r & 3;
+        bool w = (PAIR && !leader)
+                     ? mbar_wait_acquire_cluster(&sq_full[i], (r >> 2) & 1, abort_flag, lim,
+                                                 SITE_SCHED)
+                     : mbar_wait(&sq_full[i], (r >> 2) & 1, abort_flag, lim, SITE_SCHED);
+        if (warp_wide) w = __all_sync(0xffffffffu, w);
+        if (!w) {
+            ok = false;
+            return -1;
+        }
+        const int u = sq_ring[i];
+        if (warp_wide) __syncwarp();
+        if (!warp_wide || lane == 0) {
+            if (PAIR && !leader)
+                mbar_arrive_release_cluster(mapa_shared(smem_u32(&sq_empty[i]), 0));
+            else
+                mbar_arrive(&sq_empty[i]);
+        }
+        return u < num_units ? u : -1;
+    };
 
     if (warp == PF_WARP_PRODUCER) {
         // ------------------------------------------------------------ producer
@@ -457,9 +531,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             int unit_it = 0;
             int q_armed = 0;    // Q loads issued so far
             bool ok = true;
-            for (int r = 0; ok && r * G < num_units; ++r) {
-                const int u = pf_sched(r, cta, G);
-                if (u >= num_units) continue;
+            for (int r = 0; ok; ++r) {
+                const int u = leader ? take_unit(r, ok) : read_unit(r, ok, false);
+                if (u < 0) break;
                 PfUnit U;
                 pf_unit<CG>(P, vt, u, U, rank);
                 if (unit_it > 0) {
@@ -641,9 +715,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 return true;
             };
 
-            for (int r = 0; ok && r * G < num_units; ++r) {
-                const int u = pf_sched(r, cta, G);
-                if (u >= num_units) continue;
+            for (int r = 0; ok; ++r) {
+                const int u = read_unit(r, ok, false);
+                if (u < 0) break;
                 PfUnit U;
                 pf_unit<CG>(P, vt, u, U, rank);
                 ok = mbar_wait(q_full, unit_it & 1, abort_flag, lim, SITE_MMA_Q_FULL);
@@ -711,9 +785,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         uint32_t tile = 0;
         int unit_it = 0;
         bool ok = true;
-        for (int rr = 0; ok && rr * G < num_units; ++rr) {
-            const int u = pf_sched(rr, cta, G);
-            if (u >= num_units) continue;
+        for (int rr = 0; ok; ++rr) {
+            const int u = read_unit(rr, ok, true);
+            if (u < 0) break;
             PfUnit U;
             pf_unit<CG>(P, vt, u, U, rank);
             const int p = U.p_min + pr;  // absolute query position of this row
@@ -955,9 +1029,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         uint32_t tile = 0;
         int unit_it = 0;
         bool ok = true;
-        for (int rr = 0; ok && rr * G < num_units; ++rr) {
-            const int u = pf_sched(rr, cta, G);
-            if (u >= num_units) continue;
+        for (int rr = 0; ok; ++rr) {
+            const int u = read_unit(rr, ok, true);
+            if (u < 0) break;
             PfUnit U;
             pf_unit<CG>(P, vt, u, U, rank);
             // PV(gl) completing implies every earlier UMMA of this CTA completed.
@@ -1043,6 +1117,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         tc_fence_after();
         if constexpr (PAIR) tmem_dealloc_pair(tmem, PF_TMEM_COLS);
         else tmem_dealloc(tmem, PF_TMEM_COLS);
+    }
+    // dynamic schedule: every unit of this launch was taken (each even CTA's
+    // producer took one past the last before the barrier above); the last CTA
+    // to get here zeroes the slot
+    if (dyn && threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&sched[1], 1u) == gridDim.x - 1) {
+            atomicExch(&sched[0], 0u);
+            atomicExch(&sched[1], 0u);
+        }
     }
 }
 
