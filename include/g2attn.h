@@ -29,6 +29,11 @@
  *    argument error nothing is launched and nothing is written.
  *  - The host never reads device memory; cu_seqlens arrays stay on the device.
  *  - Return value: a g2attn_status code.
+ *  - Library state on the device: the sticky error word, the scratch array of
+ *    g2attn_decode_noalloc, and the unit counters of the packed-sequence
+ *    prefill launches (slot = the launch's grid id mod 4096; each launch's
+ *    last CTA zeroes its slot, so concurrent launches only interfere if 4096
+ *    of them are in flight at once).
  */
 #ifndef G2ATTN_H
 #define G2ATTN_H
