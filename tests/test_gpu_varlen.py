@@ -81,3 +81,38 @@ def test_9b_varlen_sampled(layer):
         rl_all.append(rl)
     check(torch.stack(go), np.concatenate(ro_all), torch.stack(gl), np.concatenate(rl_all),
           f"9b varlen {layer}")
+
+
+def test_concurrent_launches_on_two_streams_are_independent():
+    """Packed launches take their units from a per-launch counter slot chosen
+    by the launch's grid id: launches running at the same time on two streams
+    must not share units. Each stream's results equal those of the same call
+    run alone (bitwise: the units compute the same sums whatever CTA runs
+    them), over several rounds of overlapping launches."""
+    lens_a = [(700, 700), (1200, 1200), (300, 300), (900, 900)]
+    lens_b = [(1000, 1000), (64, 64), (1500, 1500)]
+    H, Hkv, d, W = 4, 2, 256, 256
+    dev = torch.device("cuda")
+    a = varlen_inputs(0, 0, 0, H, Hkv, d, seed=71, seq_lens=lens_a)
+    b = varlen_inputs(0, 0, 0, H, Hkv, d, seed=72, seq_lens=lens_b)
+    ga = [t.to(dev) for t in a[2:]]
+    gb = [t.to(dev) for t in b[2:]]
+    kw = dict(query_scale=0.0625, softcap=50.0, window=W)
+
+    def launch(g, Ts, Ss, stream=None):
+        cq, ck, q, k, v = g
+        return g2.prefill_varlen(q, k, v, cq, ck, max(Ts), max(Ss), stream=stream, **kw)
+
+    ref_a = launch(ga, a[0], a[1])
+    ref_b = launch(gb, b[0], b[1])
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(8):
+        with torch.cuda.stream(s1):
+            oa = launch(ga, a[0], a[1], stream=s1)
+        with torch.cuda.stream(s2):
+            ob = launch(gb, b[0], b[1], stream=s2)
+        torch.cuda.synchronize()
+        assert torch.equal(oa[0], ref_a[0]) and torch.equal(oa[1], ref_a[1])
+        assert torch.equal(ob[0], ref_b[0]) and torch.equal(ob[1], ref_b[1])
+    assert g2.g2attn_get_device_error() == g2.G2ATTN_OK
