@@ -67,9 +67,10 @@ constexpr uint32_t BW_TMEM_COLS = 512;
 // is more than the math of an M = 128, N = 64, K = 16 product (32 cycles).
 // d <= 128: K and V (or q and dout) stay in shared memory, four slots of
 // column tiles stream, and X / Y are double-buffered in TMEM. d = 256: one
-// resident operand lives in TMEM (see the file header), two slots stream, and
-// the dk/dv kernel splits each key tile into a dv and a dk unit (DSPLIT) so
-// that its accumulator fits TMEM; only the dv units double-buffer X.
+// resident operand lives in TMEM (see the file header), two slots stream (dv
+// units: three, the third in the resident region), and the dk/dv kernel
+// splits each key tile into a dv and a dk unit (DSPLIT) so that its
+// accumulator fits TMEM; only the dv units double-buffer X.
 template <int D>
 struct BwCfg {
     static_assert(D == 64 || D == 128 || D == 256, "backward kernels: d = 64, 128, 256");
