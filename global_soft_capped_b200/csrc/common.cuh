@@ -563,6 +563,18 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
     return d;
 }
 
+// acc.x += low bf16 of pk, acc.y += high bf16 of pk, each in fp32 (sm_100
+// mixed-precision add: the bf16 operand widens exactly, one rounding per add).
+__device__ __forceinline__ float2 add_bf16x2_f32(float2 acc, uint32_t pk) {
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(pk));
+    return acc;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -948,8 +948,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         ls[i & 1] = add2(ls[i & 1], e);
                         pk[i] = pack_bf16x2(e.x, e.y);
-                        lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
-                                                                  __uint_as_float(pk[i] & 0xFFFF0000u)));
+                        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
                     }
                 } else if (fast) {
                     const float2 B0 = make_float2(b0, b0), B1 = make_float2(b1, b1);
@@ -965,8 +964,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         ls[i & 1] = add2(ls[i & 1], e);
                         pk[i] = pack_bf16x2(e.x, e.y);
-                        lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
-                                                                  __uint_as_float(pk[i] & 0xFFFF0000u)));
+                        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
                     }
                 } else {
 #pragma unroll
@@ -975,8 +973,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         ls[i & 1] = add2(ls[i & 1], e);
                         pk[i] = pack_bf16x2(e.x, e.y);
-                        lrs[i & 1] = add2(lrs[i & 1], make_float2(__uint_as_float(pk[i] << 16),
-                                                                  __uint_as_float(pk[i] & 0xFFFF0000u)));
+                        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
                     }
                 }
                 // P of this part's HC keys as bf16 pairs: HC/2 columns at the
