@@ -300,7 +300,12 @@ __device__ __forceinline__ int pf_sched(int r, int c, int G) {
     return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-template <int D, int CG = 1>
+// FIX: the fixed softmax shift (PfParams::fixed_ref_on, cap on). The host
+// launches FIX = true exactly when fixed_ref_on is set, so that the softmax
+// of the capped layers carries no running-max exchange or uncapped code:
+// compiled in beside the fixed-shift loop, those cold branches cost that loop
+// about 15% at the 128-register bound.
+template <int D, int CG, bool FIX>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -819,8 +824,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // Raw accumulator range of this warp's columns (the running max
                 // needs the tile max; with the fixed shift only max |x| is
                 // needed, for the series check).
+                const bool cap = FIX || P.has_cap;  // FIX implies the cap
                 float amx, amn;
-                if (P.fixed_ref_on) {
+                if constexpr (FIX) {
                     float ma[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) ma[k] = fabsf(s[k]);
@@ -847,16 +853,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // one packed FMA below.
                 // Without the cap the map is the plain scale: the same fused path.
                 const bool fast = __all_sync(
-                    0xffffffffu, !boundary && (!P.has_cap ||
+                    0xffffffffu, !boundary && (!cap ||
                                                fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max));
                 float mt = 0.f;
                 if (fast) {
-                    if (!P.fixed_ref_on)
+                    if constexpr (!FIX)
                         mt = P.has_cap ? fmaxf(series_s2(amx), series_s2(amn))
                                        : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
                 } else {
                     // general path: capped logits in log2 units, then the mask
-                    if (P.has_cap) {
+                    if (cap) {
                         if (__all_sync(0xffffffffu,
                                        fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max)) {
 #pragma unroll
@@ -880,7 +886,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         for (int i = 0; i < HC; ++i)
                             if (i > hi || i < lo) s[i] = -INFINITY;
                     }
-                    if (!P.fixed_ref_on) {
+                    if constexpr (!FIX) {
                         float mx[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) mx[k] = s[k];
@@ -890,7 +896,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                     }
                 }
-                if (P.fixed_ref_on) {
+                if constexpr (FIX) {
                     // fixed shift: no running max, no exchange, no rescaling
                     m_ref = P.fixed_ref;
                 } else {
@@ -940,7 +946,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 uint32_t pk[HC / 2];
-                if (fast && !P.has_cap) {
+                if (!cap && fast) {
                     const float2 B0 = make_float2(b0, b0);
 #pragma unroll
                     for (int i = 0; i < HC / 2; ++i) {
