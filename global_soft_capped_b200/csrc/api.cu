@@ -400,11 +400,11 @@ size_t bwd_ws_bytes(int B, int T, int H) {
     return rows == 0 ? 0 : rows + kBwdSchedBytes;
 }
 
-template <int D, int MODE>
-int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mo, const CUtensorMap& mk,
-               const CUtensorMap& mv, g2::BwParams P, int units, int sms, cudaStream_t st) {
+template <int D, int MODE, bool CAP>
+int launch_bwd_kernel(const CUtensorMap& mq, const CUtensorMap& mo, const CUtensorMap& mk,
+                      const CUtensorMap& mv, g2::BwParams P, int units, int sms, cudaStream_t st) {
     using C = g2::BwCfg<D>;
-    auto kern = g2::bwd_sm100<D, MODE>;
+    auto kern = g2::bwd_sm100<D, MODE, CAP>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return G2ATTN_ERR_CUDA;
@@ -412,6 +412,14 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mo, const CUtensorMap& 
     const int grid = units < sms ? units : sms;
     kern<<<grid, g2::BW_THREADS, C::SMEM_BYTES, st>>>(mq, mo, mk, mv, P);
     return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
+}
+
+// The capped or the uncapped instantiation, as the parameters say.
+template <int D, int MODE>
+int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mo, const CUtensorMap& mk,
+               const CUtensorMap& mv, g2::BwParams P, int units, int sms, cudaStream_t st) {
+    return P.has_cap ? launch_bwd_kernel<D, MODE, true>(mq, mo, mk, mv, P, units, sms, st)
+                     : launch_bwd_kernel<D, MODE, false>(mq, mo, mk, mv, P, units, sms, st);
 }
 
 // Tensor maps of the two gradient kernels: the dk/dv kernel keeps 128-key K/V

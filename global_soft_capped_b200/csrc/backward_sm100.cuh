@@ -540,7 +540,10 @@ __device__ __forceinline__ void bw_st(uint32_t taddr, const uint32_t (&r)[N]) {
     }
 }
 
-template <int D, int MODE>
+// CAP: the soft-cap is on (BwParams::has_cap). The host launches the
+// instantiation that matches, so that the elementwise pass of either kind
+// of layer carries only its own loops.
+template <int D, int MODE, bool CAP>
 __global__ void __launch_bounds__(BW_THREADS, 1)
     bwd_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -1250,13 +1253,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     bw_fence<CHUNK>(xv);
                     bw_fence<CHUNK>(yv);
                     // the cap's tanh by series when every |u| of this warp's chunk <= 1/4
-                    float am[2] = {0.f, 0.f};
+                    bool poly = false;
+                    if constexpr (CAP) {
+                        float am[2] = {0.f, 0.f};
 #pragma unroll
-                    for (int i = 0; i < CHUNK; i += 2)
-                        am[(i >> 1) & 1] = fmax3f(am[(i >> 1) & 1], fabsf(__uint_as_float(xv[i])),
-                                                  fabsf(__uint_as_float(xv[i + 1])));
-                    const bool poly =
-                        __all_sync(0xffffffffu, fmaxf(am[0], am[1]) <= P.poly_acc_max);
+                        for (int i = 0; i < CHUNK; i += 2)
+                            am[(i >> 1) & 1] =
+                                fmax3f(am[(i >> 1) & 1], fabsf(__uint_as_float(xv[i])),
+                                       fabsf(__uint_as_float(xv[i + 1])));
+                        poly = __all_sync(0xffffffffu, fmaxf(am[0], am[1]) <= P.poly_acc_max);
+                    }
                     uint32_t pp[CHUNK / 2], pd[CHUNK / 2];
                     // -lse2 / -D of the column pair i, i+1 (KV: per column, from
                     // the slot; Q: this row's)
@@ -1295,7 +1301,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             }
                         };
                         const float2 one = make_float2(1.f, 1.f), mone = make_float2(-1.f, -1.f);
-                        if (P.has_cap) {
+                        if constexpr (CAP) {
                             // tanh(alpha x / C) = x (t0 + t1 x^2 + t2 x^4 + t3 x^6): the
                             // series in u = alpha x / C with the powers of alpha / C
                             // folded into its coefficients
@@ -1365,7 +1371,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                             }
                         }
                     };
-                    if (poly || !P.has_cap) {
+                    if (poly || !CAP) {
                         if (want_y) {
                             if (interior) fast(BwMask<false>{}, BwMask<true>{});
                             else fast(BwMask<true>{}, BwMask<true>{});
@@ -1399,7 +1405,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                                                  (t < U.T) && (j < U.S);
                                 const float x = __uint_as_float(xv[i + e]);
                                 float s2, dcap;
-                                if (P.has_cap) {
+                                if constexpr (CAP) {
                                     float th;
                                     if (poly) {
                                         th = bw_tanh_series(x * P.u_scale);
