@@ -112,7 +112,7 @@ void fill_poly(float query_scale, float softcap, g2::PfParams& P) {
 
 // CG = 2 launches clusters of two CTAs (one unit of 128 query positions per
 // pair); the grid holds as many pairs as can be resident at once.
-template <int D, int CG, bool FIX>
+template <int D, int CG, int SM>
 int launch_prefill_kernel(const void* q, const void* k, const void* v, long long total_q,
                           long long total_k, g2::PfParams& P, cudaStream_t stream) {
     using C = g2::PfCfg<D, CG>;
@@ -123,7 +123,7 @@ int launch_prefill_kernel(const void* q, const void* k, const void* v, long long
         return G2ATTN_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return G2ATTN_ERR_CUDA;
-    auto kern = g2::prefill_fwd_sm100<D, CG, FIX>;
+    auto kern = g2::prefill_fwd_sm100<D, CG, SM>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return G2ATTN_ERR_CUDA;
@@ -157,13 +157,17 @@ int launch_prefill_kernel(const void* q, const void* k, const void* v, long long
     return cudaGetLastError() == cudaSuccess ? G2ATTN_OK : G2ATTN_ERR_CUDA;
 }
 
-// The fixed-shift instantiation exactly when the parameters turn the fixed
-// shift on (see PfParams::fixed_ref_on).
+// The softmax variant the parameters call for: the fixed shift whenever it
+// is on (see PfParams::fixed_ref_on), else the running max with or without
+// the cap.
 template <int D, int CG>
 int launch_prefill(const void* q, const void* k, const void* v, long long total_q,
                    long long total_k, g2::PfParams& P, cudaStream_t stream) {
-    return P.fixed_ref_on ? launch_prefill_kernel<D, CG, true>(q, k, v, total_q, total_k, P, stream)
-                          : launch_prefill_kernel<D, CG, false>(q, k, v, total_q, total_k, P, stream);
+    if (P.fixed_ref_on)
+        return launch_prefill_kernel<D, CG, g2::PF_SM_FIXED>(q, k, v, total_q, total_k, P, stream);
+    if (P.has_cap)
+        return launch_prefill_kernel<D, CG, g2::PF_SM_CAP>(q, k, v, total_q, total_k, P, stream);
+    return launch_prefill_kernel<D, CG, g2::PF_SM_NOCAP>(q, k, v, total_q, total_k, P, stream);
 }
 
 // d = 256 runs on CTA pairs unless G2ATTN_PREFILL_PAIR=0 selects the

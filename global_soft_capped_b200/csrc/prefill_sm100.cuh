@@ -65,6 +65,10 @@ constexpr float PF_POLY_U_MAX = 0.25f;  // |x / C| bound of the series path
 // Largest C log2(e) for which the fixed softmax shift keeps every weight a
 // normal float: 2^(-2 C log2(e) + 64) >= 2^-126.
 constexpr float PF_FIXED_REF_MAX = 95.0f;
+// softmax variants of the forward kernel (template parameter SM)
+constexpr int PF_SM_FIXED = 0;  // cap on, fixed softmax shift
+constexpr int PF_SM_CAP = 1;    // cap on, running max
+constexpr int PF_SM_NOCAP = 2;  // no cap, running max
 
 // CG = 1: one CTA per unit of 64 query positions. CG = 2 (d = 256 only): a CTA
 // pair per unit of 128 positions, 64 per CTA; each CTA stages half of every
@@ -300,12 +304,13 @@ __device__ __forceinline__ int pf_sched(int r, int c, int G) {
     return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-// FIX: the fixed softmax shift (PfParams::fixed_ref_on, cap on). The host
-// launches FIX = true exactly when fixed_ref_on is set, so that the softmax
-// of the capped layers carries no running-max exchange or uncapped code:
-// compiled in beside the fixed-shift loop, those cold branches cost that loop
-// about 15% at the 128-register bound.
-template <int D, int CG, bool FIX>
+// SM, the softmax variant: PF_SM_FIXED (cap on, fixed shift:
+// PfParams::fixed_ref_on), PF_SM_CAP (cap on, running max) or PF_SM_NOCAP
+// (running max). The host launches the one the parameters call for, so that
+// each softmax carries only its own loops: compiled in beside the fixed-shift
+// loop, the running-max exchange and the uncapped loop cost it about 15% at
+// the 128-register bound.
+template <int D, int CG, int SM>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -824,7 +829,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // Raw accumulator range of this warp's columns (the running max
                 // needs the tile max; with the fixed shift only max |x| is
                 // needed, for the series check).
-                const bool cap = FIX || P.has_cap;  // FIX implies the cap
+                constexpr bool FIX = SM == PF_SM_FIXED;
+                constexpr bool cap = SM != PF_SM_NOCAP;
                 float amx, amn;
                 if constexpr (FIX) {
                     float ma[4];
@@ -858,11 +864,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float mt = 0.f;
                 if (fast) {
                     if constexpr (!FIX)
-                        mt = P.has_cap ? fmaxf(series_s2(amx), series_s2(amn))
-                                       : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
+                        mt = cap ? fmaxf(series_s2(amx), series_s2(amn))
+                                 : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
                 } else {
                     // general path: capped logits in log2 units, then the mask
-                    if (cap) {
+                    if constexpr (cap) {
                         if (__all_sync(0xffffffffu,
                                        fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max)) {
 #pragma unroll

@@ -52,6 +52,10 @@ EDGE = [
     (1, 190, 190, 2, 1, 128, 0, 50, 0.0, 0.09, 1.0),      # no cap
     (1, 128, 128, 2, 1, 64, 0, 0, 50.0, 4.0, 1.0),        # logits well past the cap
     (1, 192, 192, 2, 1, 256, 0, 70, 50.0, 0.25, 1.0),
+    # cap above C log2(e) = 95, i.e. C > 65.8: running max with the cap on
+    (1, 300, 300, 2, 1, 128, 0, 0, 100.0, 0.09, 1.0),     # series range
+    (1, 200, 200, 2, 1, 256, 0, 64, 100.0, 4.0, 1.0),     # logits past the series range
+    (2, 150, 260, 4, 2, 64, 110, 0, 80.0, 0.5, 1.0),
 ]
 
 
