@@ -298,6 +298,77 @@ __device__ __forceinline__ void pf_store_rows(uint32_t (&w)[EC / 2], int lane, R
 constexpr int PF_SCHED_SLOTS = 4096;
 __device__ unsigned int g_pf_sched[PF_SCHED_SLOTS][2];
 
+// The general path of the fixed-shift softmax for one warp's PF_PHC columns of
+// an S tile: tiles on the band's edges (columns outside [lo, hi] are masked)
+// or with logits past the series range (series false: the exact cap). Out of
+// line, so that the fast tile loop of the same kernel is compiled without it:
+// inline, this rarely taken code cost the fast loop several percent at the
+// 128-register bound. It reads the columns at `cols` again from TMEM (P has
+// not been written over them yet), writes the bf16 weights at the start of
+// the same columns, and returns the sums of the fp32 weights (x, y) and of
+// the bf16-rounded ones (z, w), pair lanes as in the fast loop. Called by
+// whole warps (the tcgen05 loads and stores are warp-wide).
+__device__ __noinline__ float4 pf_softmax_general_fixed(uint32_t cols, int lo, int hi,
+                                                        bool series, float b0, float b1,
+                                                        float b2, float b3, float k_exp,
+                                                        float cap_l2, float m_use) {
+    constexpr int HC = PF_PHC;
+    float s[HC];
+    {
+        uint32_t v[HC / 32][32];
+#pragma unroll
+        for (int c = 0; c < HC / 32; ++c) tmem_ld32_async(cols + 32 * c, v[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < HC / 32; ++c) tmem_reg_fence(v[c]);
+#pragma unroll
+        for (int i = 0; i < HC; ++i) s[i] = __uint_as_float(v[i / 32][i % 32]);
+    }
+    // capped logits in log2 units, then the mask
+    if (series) {
+#pragma unroll
+        for (int i = 0; i < HC; ++i) {
+            const float x2 = s[i] * s[i];
+            float q = fmaf(x2, b3, b2);
+            q = fmaf(x2, q, b1);
+            q = fmaf(x2, q, b0);
+            s[i] = s[i] * q;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < HC; ++i) {
+            const float e = ex2_approx(s[i] * k_exp);
+            const float rc = rcp_approx(1.0f + e);
+            s[i] = fmaf(-2.0f * cap_l2, rc, cap_l2);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < HC; ++i)
+        if (i > hi || i < lo) s[i] = -INFINITY;
+    const float2 mneg = make_float2(-m_use, -m_use);
+    float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    uint32_t pk[HC / 2];
+#pragma unroll
+    for (int i = 0; i < HC / 2; ++i) {
+        const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
+        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        ls[i & 1] = add2(ls[i & 1], e);
+        pk[i] = pack_bf16x2(e.x, e.y);
+        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
+    }
+#pragma unroll
+    for (int c = 0; c < HC / 32; ++c) {
+        uint32_t pc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pc[i] = pk[16 * c + i];
+        tmem_st16(cols + 16 * c, pc);
+    }
+    const float2 lsum = add2(ls[0], ls[1]);
+    const float2 lrsum = add2(lrs[0], lrs[1]);
+    return make_float4(lsum.x, lsum.y, lrsum.x, lrsum.y);
+}
+
 // Static persistent schedule: round r gives CTA c unit r*G + c (even rounds)
 // or r*G + G-1-c (odd rounds), so the longest units spread evenly.
 __device__ __forceinline__ int pf_sched(int r, int c, int G) {
@@ -866,8 +937,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     if constexpr (!FIX)
                         mt = cap ? fmaxf(series_s2(amx), series_s2(amn))
                                  : fmaxf(amx * P.scale_l2, amn * P.scale_l2);
-                } else {
+                } else if constexpr (!FIX) {
                     // general path: capped logits in log2 units, then the mask
+                    // (the fixed shift's general path is out of line, below)
                     if constexpr (cap) {
                         if (__all_sync(0xffffffffu,
                                        fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max)) {
@@ -949,6 +1021,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // same rounded weights makes them sum to one exactly, so their
                 // rounding errors cancel against the row's mean value.
                 const float2 mneg = make_float2(-m_use, -m_use);
+                if (FIX && !fast) {
+                    // the band's edges or logits past the series range
+                    const int hi = boundary ? p - j0 - col0 : HC;  // visible local columns
+                    const int lo = (boundary && P.window > 0) ? p - P.window + 1 - j0 - col0 : -1;
+                    const bool series = __all_sync(
+                        0xffffffffu, fmaxf(fabsf(amx), fabsf(amn)) <= P.poly_acc_max);
+                    const float4 r4 = pf_softmax_general_fixed(s_addr + col0, lo, hi, series, b0,
+                                                               b1, b2, b3, P.k_exp, P.cap_l2,
+                                                               m_use);
+                    l += r4.x + r4.y;
+                    lr += r4.z + r4.w;
+                } else {
                 float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 uint32_t pk[HC / 2];
@@ -978,7 +1062,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         pk[i] = pack_bf16x2(e.x, e.y);
                         lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
                     }
-                } else {
+                } else if constexpr (!FIX) {
 #pragma unroll
                     for (int i = 0; i < HC / 2; ++i) {
                         const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
@@ -1002,6 +1086,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const float2 lrsum = add2(lrs[0], lrs[1]);
                 l += lsum.x + lsum.y;
                 lr += lrsum.x + lrsum.y;
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
