@@ -5,7 +5,8 @@ A fixed generator draws dense, varlen, gradient and decode cases. The ranges are
 * 1–3 KV heads with two query heads each, batch 1–3;
 * S up to 700, 1 <= T <= S, any valid q_offset;
 * no window, or any window size;
-* cap 50, 5 or off, several query scales;
+* cap 50, 5 or off, several query scales, and a few cases with the cap at 100 (above
+  C log2(e) = 95 the forward keeps a running max with the cap on);
 * varlen packings with empty and single-token sequences;
 * decode from linear, ring (power-of-two slots >= window) and paged (16-256-row
   blocks) caches, with 1-12 sequences of up to 3000 tokens.
@@ -44,7 +45,11 @@ def _dense_cases(n, seed):
     return cases
 
 
-DENSE = _dense_cases(24, 20261202)
+def _with_cap(cases, cap, i_cap):
+    return [c[:i_cap] + (cap,) + c[i_cap + 1:] for c in cases]
+
+
+DENSE = _dense_cases(24, 20261202) + _with_cap(_dense_cases(6, 31337), 100.0, 8)
 
 
 @pytest.mark.parametrize("case", DENSE, ids=[str(i) for i in range(len(DENSE))])
@@ -77,7 +82,7 @@ def _varlen_cases(n, seed):
     return cases
 
 
-VARLEN = _varlen_cases(8, 777)
+VARLEN = _varlen_cases(8, 777) + _with_cap(_varlen_cases(3, 4711), 100.0, 5)
 
 
 @pytest.mark.parametrize("case", VARLEN, ids=[str(i) for i in range(len(VARLEN))])
@@ -92,7 +97,8 @@ def test_random_varlen(case):
 
 
 BACKWARD = ([c for c in _dense_cases(40, 4242) if c[5] in (64, 128)][:8] +
-            [c for c in _dense_cases(40, 9898) if c[5] == 256][:6])
+            [c for c in _dense_cases(40, 9898) if c[5] == 256][:6] +
+            _with_cap(_dense_cases(2, 5353), 100.0, 8))
 
 
 @pytest.mark.parametrize("case", BACKWARD, ids=[str(i) for i in range(len(BACKWARD))])
