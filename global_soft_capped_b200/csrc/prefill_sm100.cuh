@@ -1033,59 +1033,59 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     l += r4.x + r4.y;
                     lr += r4.z + r4.w;
                 } else {
-                float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                uint32_t pk[HC / 2];
-                if (!cap && fast) {
-                    const float2 B0 = make_float2(b0, b0);
+                    float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    float2 lrs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    uint32_t pk[HC / 2];
+                    if (!cap && fast) {
+                        const float2 B0 = make_float2(b0, b0);
 #pragma unroll
-                    for (int i = 0; i < HC / 2; ++i) {
-                        const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), B0, mneg);
-                        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                        ls[i & 1] = add2(ls[i & 1], e);
-                        pk[i] = pack_bf16x2(e.x, e.y);
-                        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
+                        for (int i = 0; i < HC / 2; ++i) {
+                            const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), B0, mneg);
+                            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                            ls[i & 1] = add2(ls[i & 1], e);
+                            pk[i] = pack_bf16x2(e.x, e.y);
+                            lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
+                        }
+                    } else if (fast) {
+                        const float2 B0 = make_float2(b0, b0), B1 = make_float2(b1, b1);
+                        const float2 B2 = make_float2(b2, b2), B3 = make_float2(b3, b3);
+#pragma unroll
+                        for (int i = 0; i < HC / 2; ++i) {
+                            const float2 a = make_float2(s[2 * i], s[2 * i + 1]);
+                            const float2 x2 = mul2(a, a);
+                            float2 q = fma2(x2, B3, B2);
+                            q = fma2(x2, q, B1);
+                            q = fma2(x2, q, B0);
+                            const float2 x = fma2(a, q, mneg);  // s2 - m
+                            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                            ls[i & 1] = add2(ls[i & 1], e);
+                            pk[i] = pack_bf16x2(e.x, e.y);
+                            lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
+                        }
+                    } else if constexpr (!FIX) {
+#pragma unroll
+                        for (int i = 0; i < HC / 2; ++i) {
+                            const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
+                            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                            ls[i & 1] = add2(ls[i & 1], e);
+                            pk[i] = pack_bf16x2(e.x, e.y);
+                            lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
+                        }
                     }
-                } else if (fast) {
-                    const float2 B0 = make_float2(b0, b0), B1 = make_float2(b1, b1);
-                    const float2 B2 = make_float2(b2, b2), B3 = make_float2(b3, b3);
+                    // P of this part's HC keys as bf16 pairs: HC/2 columns at the
+                    // start of its own S columns, which it has already read (the
+                    // other part's S columns may still be unread)
 #pragma unroll
-                    for (int i = 0; i < HC / 2; ++i) {
-                        const float2 a = make_float2(s[2 * i], s[2 * i + 1]);
-                        const float2 x2 = mul2(a, a);
-                        float2 q = fma2(x2, B3, B2);
-                        q = fma2(x2, q, B1);
-                        q = fma2(x2, q, B0);
-                        const float2 x = fma2(a, q, mneg);  // s2 - m
-                        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                        ls[i & 1] = add2(ls[i & 1], e);
-                        pk[i] = pack_bf16x2(e.x, e.y);
-                        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
+                    for (int c = 0; c < HC / 32; ++c) {
+                        uint32_t pc[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pc[i] = pk[16 * c + i];
+                        tmem_st16(s_addr + part * HC + 16 * c, pc);
                     }
-                } else if constexpr (!FIX) {
-#pragma unroll
-                    for (int i = 0; i < HC / 2; ++i) {
-                        const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), mneg);
-                        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                        ls[i & 1] = add2(ls[i & 1], e);
-                        pk[i] = pack_bf16x2(e.x, e.y);
-                        lrs[i & 1] = add_bf16x2_f32(lrs[i & 1], pk[i]);
-                    }
-                }
-                // P of this part's HC keys as bf16 pairs: HC/2 columns at the
-                // start of its own S columns, which it has already read (the
-                // other part's S columns may still be unread)
-#pragma unroll
-                for (int c = 0; c < HC / 32; ++c) {
-                    uint32_t pc[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pc[i] = pk[16 * c + i];
-                    tmem_st16(s_addr + part * HC + 16 * c, pc);
-                }
-                const float2 lsum = add2(ls[0], ls[1]);
-                const float2 lrsum = add2(lrs[0], lrs[1]);
-                l += lsum.x + lsum.y;
-                lr += lrsum.x + lrsum.y;
+                    const float2 lsum = add2(ls[0], ls[1]);
+                    const float2 lrsum = add2(lrs[0], lrs[1]);
+                    l += lsum.x + lsum.y;
+                    lr += lrsum.x + lrsum.y;
                 }
                 tmem_wait_st();
                 tc_fence_before();
